@@ -1,0 +1,300 @@
+"""Plain CPU oracle for bitshift-trellis coded quantisation (TEST INFRASTRUCTURE).
+
+Only the test-suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product (the CUDA library and its
+Python binding) never imports, links or calls it, and it never imports the
+product: the two share nothing but the seeded input generators in
+``tcq_workloads``.
+
+The arithmetic lives in ``tcq_oracle.c`` (Viterbi, BCJR, the vector-Jacobian
+product, brute force), compiled with gcc without fast-math; this module wraps
+it with ctypes and adds the bitstream decode/pack, written with numpy bit
+arrays straight from the window formula.
+
+Sources (restated, not copied):
+  * QTIP blog post, "QTIP: Trellis-Coded Quantization Puts 2-Bit LLM Weights
+    10% Above the Rate-Distortion Bound ..." -- sections "The trellis: a
+    stateful codebook" (bitshift trellis, predecessor set, decode window,
+    Viterbi), "The codebook is computed" (1MAD), "Tail-biting is worth its
+    complexity" (tail-biting stream of exactly k*T bits), "What it buys end to
+    end" (each 16x16 tile is one 256-weight sequence).
+  * "BCJR-QAT: A Differentiable Relaxation of Trellis-Coded Weight
+    Quantization", abstract (soft codeword = Boltzmann expectation over walks).
+
+Pins: every function here is checked by ``tests/test_oracle_*.py`` against
+what the pages print (908 distinct 1MAD values, the free-start MSE by L, the
+monotone-code MSE), closed forms (Irwin-Hall moments, D(R)), brute force over
+all walks, an independent transfer-matrix route to log Z, finite differences
+and the pages' own window formula evaluated with Python integers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from functools import lru_cache
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tcq_oracle.c")
+_LIB = os.path.join(_HERE, "libtcq_oracle.so")
+
+TAILBITING = 0
+FREE_START = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile ``tcq_oracle.c`` into ``libtcq_oracle.so`` (IEEE, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([
+            "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+            "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+@lru_cache(maxsize=None)
+def _lib():
+    lib = ctypes.CDLL(build())
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    D = ctypes.c_double
+    lib.orc_1mad_bytesum.argtypes = [ctypes.c_uint32]
+    lib.orc_1mad_bytesum.restype = I
+    lib.orc_1mad_f64.argtypes = [ctypes.c_uint32]
+    lib.orc_1mad_f64.restype = D
+    lib.orc_1mad_f32.argtypes = [ctypes.c_uint32]
+    lib.orc_1mad_f32.restype = ctypes.c_float
+    lib.orc_codebook_1mad_f64.argtypes = [I, P]
+    lib.orc_codebook_1mad_f32.argtypes = [I, P]
+    lib.orc_viterbi_f32.argtypes = [I, I, I, P, P, P]
+    lib.orc_viterbi_f32.restype = ctypes.c_float
+    lib.orc_viterbi_f64.argtypes = [I, I, I, P, P, P, P]
+    lib.orc_viterbi_f64.restype = D
+    lib.orc_bcjr_f64.argtypes = [I, I, I, D, P, P, P, P, P, P]
+    lib.orc_bcjr_f64.restype = I
+    lib.orc_bcjr_vjp_f64.argtypes = [I, I, I, D, P, P, P, P, P]
+    lib.orc_bcjr_vjp_f64.restype = I
+    lib.orc_bruteforce_f64.argtypes = [I, I, I, D, P, P, P, P, P, P]
+    lib.orc_bruteforce_f64.restype = ctypes.c_int64
+    return lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --------------------------------------------------------------------------
+# 1MAD codebook
+# --------------------------------------------------------------------------
+def bytesum_1mad(x: int) -> int:
+    return int(_lib().orc_1mad_bytesum(int(x)))
+
+
+@lru_cache(maxsize=None)
+def codebook_f64(L: int) -> np.ndarray:
+    out = np.empty(1 << L, dtype=np.float64)
+    _lib().orc_codebook_1mad_f64(L, _ptr(out))
+    out.setflags(write=False)
+    return out
+
+
+@lru_cache(maxsize=None)
+def codebook_f32(L: int) -> np.ndarray:
+    out = np.empty(1 << L, dtype=np.float32)
+    _lib().orc_codebook_1mad_f32(L, _ptr(out))
+    out.setflags(write=False)
+    return out
+
+
+def codebook_f16(L: int) -> np.ndarray:
+    """fp16 value of each state: round-to-nearest-even of the fp64 1MAD value."""
+    return codebook_f64(L).astype(np.float16)
+
+
+# --------------------------------------------------------------------------
+# Viterbi
+# --------------------------------------------------------------------------
+def viterbi_f32(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None):
+    """fp32-canonical Viterbi on each row of ``s`` [n, T].
+
+    Returns (states uint16 [n, T], mse float32 [n]) with mse = min cost / T
+    computed in fp32."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    if s.ndim == 1:
+        s = s[None]
+    n, T = s.shape
+    code = codebook_f32(L) if code is None else np.ascontiguousarray(code, dtype=np.float32)
+    states = np.empty((n, T), dtype=np.uint16)
+    mse = np.empty(n, dtype=np.float32)
+    lib = _lib()
+    for i in range(n):
+        row = s[i]
+        st = states[i]
+        cost = lib.orc_viterbi_f32(L, k, T, _ptr(row), _ptr(code), _ptr(st))
+        mse[i] = np.float32(cost) / np.float32(T)
+    return states, mse
+
+
+def viterbi_f64(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None):
+    """fp64 Viterbi; returns (states [n, T], mse float64 [n], min_margin [n])."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    if s.ndim == 1:
+        s = s[None]
+    n, T = s.shape
+    code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
+    states = np.empty((n, T), dtype=np.uint16)
+    mse = np.empty(n, dtype=np.float64)
+    margin = np.empty(n, dtype=np.float64)
+    lib = _lib()
+    m = ctypes.c_double()
+    for i in range(n):
+        cost = lib.orc_viterbi_f64(L, k, T, _ptr(s[i]), _ptr(code), _ptr(states[i]), ctypes.byref(m))
+        mse[i] = cost / T
+        margin[i] = m.value
+    return states, mse, margin
+
+
+# --------------------------------------------------------------------------
+# BCJR soft codeword and its vector-Jacobian product
+# --------------------------------------------------------------------------
+def bcjr_soft(s: np.ndarray, L: int, temp: float, k: int = 2, code: np.ndarray | None = None,
+              return_tables: bool = False):
+    """Soft codeword E_p[code(x_t)] and log Z per row of ``s`` (fp64)."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    if s.ndim == 1:
+        s = s[None]
+    n, T = s.shape
+    code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
+    soft = np.empty((n, T), dtype=np.float64)
+    logz = np.empty(n, dtype=np.float64)
+    tables = []
+    lib = _lib()
+    lz = ctypes.c_double()
+    for i in range(n):
+        if return_tables:
+            al = np.empty((T, 1 << L)); be = np.empty((T, 1 << L))
+            pa, pb = _ptr(al), _ptr(be)
+        else:
+            pa = pb = None
+        rc = lib.orc_bcjr_f64(L, k, T, float(temp), _ptr(s[i]), _ptr(code), _ptr(soft[i]),
+                              ctypes.byref(lz), pa, pb)
+        assert rc == 0
+        logz[i] = lz.value
+        if return_tables:
+            tables.append((al, be))
+    if return_tables:
+        return soft, logz, tables
+    return soft, logz
+
+
+def bcjr_vjp(s: np.ndarray, v: np.ndarray, L: int, temp: float, k: int = 2,
+             code: np.ndarray | None = None):
+    """grad[u] = d/ds_u sum_t v_t soft_t per row (fp64); also returns soft."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    if s.ndim == 1:
+        s = s[None]; v = v[None]
+    n, T = s.shape
+    code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
+    grad = np.empty((n, T)); soft = np.empty((n, T))
+    lib = _lib()
+    for i in range(n):
+        rc = lib.orc_bcjr_vjp_f64(L, k, T, float(temp), _ptr(s[i]), _ptr(code), _ptr(v[i]),
+                                  _ptr(grad[i]), _ptr(soft[i]))
+        assert rc == 0
+    return grad, soft
+
+
+def bruteforce(s: np.ndarray, L: int, temp: float, k: int = 2, code: np.ndarray | None = None):
+    """Enumerate every walk of one sequence ``s`` [T] (tiny cases only).
+
+    Returns dict(min_energy, log_z, soft [T], second [T, T], walks)."""
+    s = np.ascontiguousarray(s, dtype=np.float64).ravel()
+    T = s.shape[0]
+    code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
+    soft = np.empty(T); second = np.empty((T, T))
+    emin = ctypes.c_double(); lz = ctypes.c_double()
+    W = _lib().orc_bruteforce_f64(L, k, T, float(temp), _ptr(s), _ptr(code), ctypes.byref(emin),
+                                  ctypes.byref(lz), _ptr(soft), _ptr(second))
+    if W < 0:
+        raise ValueError("too many walks for brute force")
+    return dict(min_energy=emin.value, log_z=lz.value, soft=soft, second=second, walks=W)
+
+
+# --------------------------------------------------------------------------
+# Bitstream: decode and pack (QTIP blog, "The trellis" decode window; the
+# tail-biting stream of exactly k*T bits).  Stream bit p of a sequence sits
+# in 32-bit word p // 32 at bit 31 - p % 32 (most significant first).
+# --------------------------------------------------------------------------
+def stream_nbits(L: int, k: int, T: int, layout: int) -> int:
+    return k * T if layout == TAILBITING else k * T + L - k
+
+
+def stream_words(L: int, k: int, T: int, layout: int) -> int:
+    return (stream_nbits(L, k, T, layout) + 31) // 32
+
+
+def _words_to_bits(words: np.ndarray) -> np.ndarray:
+    words = np.ascontiguousarray(words, dtype=np.uint32)
+    n = words.shape[0]
+    by = words.astype(">u4").view(np.uint8).reshape(n, -1)
+    return np.unpackbits(by, axis=1)          # bit p of the stream in column p
+
+
+def _bits_to_words(bits: np.ndarray) -> np.ndarray:
+    n = bits.shape[0]
+    by = np.packbits(bits.astype(np.uint8), axis=1)
+    return by.view(">u4").astype(np.uint32).reshape(n, -1)
+
+
+def windows(words: np.ndarray, L: int, k: int, T: int, layout: int) -> np.ndarray:
+    """State (L-bit window) of every weight: weight t reads stream bits
+    [k t, k t + L), most significant first; the tail-biting stream wraps."""
+    bits = _words_to_bits(words)
+    nb = stream_nbits(L, k, T, layout)
+    n = bits.shape[0]
+    out = np.zeros((n, T), dtype=np.int64)
+    for t in range(T):
+        for i in range(L):
+            p = k * t + i
+            if layout == TAILBITING:
+                p %= nb
+            out[:, t] |= bits[:, p].astype(np.int64) << (L - 1 - i)
+    return out
+
+
+def decode(words: np.ndarray, L: int, T: int, layout: int = TAILBITING, k: int = 2) -> np.ndarray:
+    """fp16 weights [n, T] (sequence order) decoded from packed streams."""
+    w = windows(words, L, k, T, layout)
+    return codebook_f16(L)[w]
+
+
+def decode_tiles(words: np.ndarray, rows: int, cols: int, L: int = 16, layout: int = TAILBITING,
+                 k: int = 2) -> np.ndarray:
+    """Decode into a [rows, cols] fp16 matrix: sequence r*(cols/16)+c fills the
+    16x16 tile whose top-left element is (16r, 16c), row-major inside the tile."""
+    seqs = decode(words, L, 256, layout, k)
+    nr, nc = rows // 16, cols // 16
+    return seqs.reshape(nr, nc, 16, 16).transpose(0, 2, 1, 3).reshape(rows, cols)
+
+
+def pack(states: np.ndarray, L: int, layout: int, k: int = 2) -> np.ndarray:
+    """Pack walks [n, T] into streams.  Bits [k t, k t + k) are the top k bits
+    of state t; a free-start stream ends with the remaining L - k bits of the
+    last state.  For a valid walk this is the inverse of ``windows``."""
+    states = np.asarray(states).astype(np.int64)
+    n, T = states.shape
+    nb = stream_nbits(L, k, T, layout)
+    nw = stream_words(L, k, T, layout)
+    bits = np.zeros((n, nw * 32), dtype=np.uint8)
+    for t in range(T):
+        for i in range(k):
+            bits[:, k * t + i] = (states[:, t] >> (L - 1 - i)) & 1
+    if layout == FREE_START:
+        for i in range(k, L):
+            bits[:, k * (T - 1) + i] = (states[:, T - 1] >> (L - 1 - i)) & 1
+    assert nb <= nw * 32
+    return _bits_to_words(bits)

@@ -1,0 +1,401 @@
+/*
+ * tcq_oracle.c -- plain, slow CPU oracle for bitshift-trellis coded quantisation.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file: only the test-suite, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or constant generator
+ * with the CUDA library; it is written from the pages' definitions, one
+ * sequence at a time, with no blocking, fusion or reordering.
+ *
+ * Sources (web pages restated here in our own code):
+ *   [QTIP-blog]  "QTIP: Trellis-Coded Quantization Puts 2-Bit LLM Weights 10%
+ *                Above the Rate-Distortion Bound ..." (mohakchugh.is-a.dev),
+ *                sections "The trellis: a stateful codebook",
+ *                "The codebook is computed", "Reproducing Table 1".
+ *   [BCJR-QAT]   "BCJR-QAT: A Differentiable Relaxation of Trellis-Coded
+ *                Weight Quantization", abstract (the BCJR relaxation).
+ *
+ * Conventions shared by every function below:
+ *   L      state width in bits (2^L states), k bits per step, V = 1.
+ *   T      sequence length (number of weights), s[0..T-1] the targets.
+ *   code   codebook table, code[j] = value of state j (2^L entries).
+ *   pred_a(j) = (j >> k) | (a << (L-k)),  a in [0, 2^k)     [QTIP-blog, trellis]
+ *   succ_b(i) = ((i << k) | b) & (2^L - 1), b in [0, 2^k)
+ *   Free start: every state may begin a walk with cost (code - s_0)^2.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off (no fast-math), so
+ * every float/double operation below is one IEEE-754 operation, correctly
+ * rounded, in the order written.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* 1MAD computed codebook   [QTIP-blog, "The codebook is computed"]          */
+/* A 32-bit LCG step, the sum of the four bytes of the result (Irwin-Hall,  */
+/* n = 4), then centre by 510 and scale by 147.8.                           */
+/* ------------------------------------------------------------------------ */
+int orc_1mad_bytesum(uint32_t x)
+{
+    uint32_t y = 34038481u * x + 76625530u;          /* arithmetic mod 2^32 */
+    return (int)(y & 255u) + (int)((y >> 8) & 255u) +
+           (int)((y >> 16) & 255u) + (int)((y >> 24) & 255u);
+}
+
+double orc_1mad_f64(uint32_t x)
+{
+    return ((double)orc_1mad_bytesum(x) - 510.0) / 147.8;
+}
+
+/* fp32 codebook value: the fp64 value of the pages rounded once to fp32. */
+float orc_1mad_f32(uint32_t x)
+{
+    return (float)orc_1mad_f64(x);
+}
+
+void orc_codebook_1mad_f64(int L, double *out)
+{
+    for (uint32_t j = 0; j < (1u << L); ++j) out[j] = orc_1mad_f64(j);
+}
+
+void orc_codebook_1mad_f32(int L, float *out)
+{
+    for (uint32_t j = 0; j < (1u << L); ++j) out[j] = orc_1mad_f32(j);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Viterbi, fp32 canonical arithmetic   [QTIP-blog, trellis section]         */
+/*   cost_0(j) = (code_j - s_0)^2                                            */
+/*   cost_t(j) = min_a cost_{t-1}(pred_a(j)) + (code_j - s_t)^2              */
+/* Each fp32 step is d = code - s, e = d * d, cost = best + e, every one     */
+/* rounded to fp32 (no fused multiply-add).  The argmin over a keeps the     */
+/* first (lowest a) minimum, like numpy's argmin; the final argmin keeps the */
+/* lowest state.  Returns the minimum total cost; states[0..T-1] the walk.   */
+/* ------------------------------------------------------------------------ */
+float orc_viterbi_f32(int L, int k, int T, const float *s, const float *code,
+                      uint16_t *states)
+{
+    const int N = 1 << L, A = 1 << k;
+    float *cost = (float *)malloc(sizeof(float) * N);
+    float *next = (float *)malloc(sizeof(float) * N);
+    int32_t *back = (int32_t *)malloc(sizeof(int32_t) * (size_t)T * N);
+
+    for (int j = 0; j < N; ++j) {
+        float d = code[j] - s[0];
+        cost[j] = d * d;
+    }
+    for (int t = 1; t < T; ++t) {
+        for (int j = 0; j < N; ++j) {
+            float best = INFINITY;
+            int bestp = -1;
+            for (int a = 0; a < A; ++a) {
+                int p = (j >> k) | (a << (L - k));
+                if (bestp < 0 || cost[p] < best) { best = cost[p]; bestp = p; }
+            }
+            float d = code[j] - s[t];
+            float e = d * d;
+            next[j] = best + e;
+            back[(size_t)t * N + j] = bestp;
+        }
+        float *tmp = cost; cost = next; next = tmp;
+    }
+    int st = 0;
+    for (int j = 1; j < N; ++j)
+        if (cost[j] < cost[st]) st = j;
+    float total = cost[st];
+    states[T - 1] = (uint16_t)st;
+    for (int t = T - 1; t > 0; --t) {
+        st = back[(size_t)t * N + st];
+        states[t - 1] = (uint16_t)st;
+    }
+    free(cost); free(next); free(back);
+    return total;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Viterbi in fp64, same recursion, plus the decision margin along the walk */
+/* it returns.  At every decision (each step's argmin over the 2^k          */
+/* predecessors of the chosen state, and the final argmin) the margin is    */
+/* (second distinct value - best) / max(|best|, 1e-30), where "second       */
+/* distinct" is the smallest candidate strictly above the best (exact ties  */
+/* are settled by index identically at any precision).  *min_margin gets   */
+/* the smallest such margin (INFINITY when no decision had two distinct     */
+/* candidates).  Returns the minimum total cost.                            */
+/* ------------------------------------------------------------------------ */
+static double rel_gap(double best, double second)
+{
+    double den = fabs(best) > 1e-30 ? fabs(best) : 1e-30;
+    return (second - best) / den;
+}
+
+double orc_viterbi_f64(int L, int k, int T, const double *s, const double *code,
+                       uint16_t *states, double *min_margin)
+{
+    const int N = 1 << L, A = 1 << k;
+    double *cost = (double *)malloc(sizeof(double) * (size_t)T * N); /* all steps kept */
+    int32_t *back = (int32_t *)malloc(sizeof(int32_t) * (size_t)T * N);
+
+    for (int j = 0; j < N; ++j) {
+        double d = code[j] - s[0];
+        cost[j] = d * d;
+    }
+    for (int t = 1; t < T; ++t) {
+        const double *prev = cost + (size_t)(t - 1) * N;
+        double *cur = cost + (size_t)t * N;
+        for (int j = 0; j < N; ++j) {
+            double best = INFINITY;
+            int bestp = -1;
+            for (int a = 0; a < A; ++a) {
+                int p = (j >> k) | (a << (L - k));
+                if (bestp < 0 || prev[p] < best) { best = prev[p]; bestp = p; }
+            }
+            double d = code[j] - s[t];
+            cur[j] = best + d * d;
+            back[(size_t)t * N + j] = bestp;
+        }
+    }
+    const double *last = cost + (size_t)(T - 1) * N;
+    int st = 0;
+    for (int j = 1; j < N; ++j)
+        if (last[j] < last[st]) st = j;
+    double total = last[st];
+
+    double margin = INFINITY;
+    {   /* final decision */
+        double second = INFINITY;
+        for (int j = 0; j < N; ++j)
+            if (last[j] > total && last[j] < second) second = last[j];
+        if (second < INFINITY) margin = fmin(margin, rel_gap(total, second));
+    }
+    states[T - 1] = (uint16_t)st;
+    for (int t = T - 1; t > 0; --t) {
+        const double *prev = cost + (size_t)(t - 1) * N;
+        int bestp = back[(size_t)t * N + st];
+        double best = prev[bestp], second = INFINITY;
+        for (int a = 0; a < A; ++a) {
+            int p = (st >> k) | (a << (L - k));
+            if (prev[p] > best && prev[p] < second) second = prev[p];
+        }
+        if (second < INFINITY) margin = fmin(margin, rel_gap(best, second));
+        st = bestp;
+        states[t - 1] = (uint16_t)st;
+    }
+    if (min_margin) *min_margin = margin;
+    free(cost); free(back);
+    return total;
+}
+
+/* ------------------------------------------------------------------------ */
+/* BCJR forward-backward at temperature temp, fp64, natural-log domain.     */
+/* [BCJR-QAT abstract]: the soft codeword is the Boltzmann expectation over */
+/* trellis paths.  Reading used here: a walk x has energy                   */
+/*   E(x) = sum_t (code[x_t] - s_t)^2    (the cost Viterbi minimises)       */
+/* and probability exp(-E/temp) / Z, with a free start (every first state)  */
+/* and a free end.  soft[t] = E_p[code[x_t]], *log_z = log Z.               */
+/*   alpha_0(j) = -e_0(j)/temp,  alpha_t(j) = LSE_a alpha_{t-1}(pred_a j)   */
+/*                                            - e_t(j)/temp                  */
+/*   beta_{T-1}(i) = 0,          beta_t(i) = LSE_b [beta_{t+1}(succ_b i)     */
+/*                                            - e_{t+1}(succ_b i)/temp]      */
+/*   gamma_t(j) = exp(alpha_t(j) + beta_t(j) - log Z)                        */
+/* If alpha_out/beta_out are non-NULL they receive the T x 2^L tables.      */
+/* ------------------------------------------------------------------------ */
+static double lse_array(const double *v, int n)
+{
+    double m = -INFINITY;
+    for (int i = 0; i < n; ++i) if (v[i] > m) m = v[i];
+    if (m == -INFINITY) return m;
+    double acc = 0.0;
+    for (int i = 0; i < n; ++i) acc += exp(v[i] - m);
+    return m + log(acc);
+}
+
+static double emis(const double *code, const double *s, int t, int j)
+{
+    double d = code[j] - s[t];
+    return d * d;
+}
+
+static void bcjr_tables(int L, int k, int T, double temp, const double *s,
+                        const double *code, double *alpha, double *beta)
+{
+    const int N = 1 << L, A = 1 << k;
+    double tmp[64];
+    for (int j = 0; j < N; ++j) alpha[j] = -emis(code, s, 0, j) / temp;
+    for (int t = 1; t < T; ++t)
+        for (int j = 0; j < N; ++j) {
+            for (int a = 0; a < A; ++a)
+                tmp[a] = alpha[(size_t)(t - 1) * N + ((j >> k) | (a << (L - k)))];
+            alpha[(size_t)t * N + j] = lse_array(tmp, A) - emis(code, s, t, j) / temp;
+        }
+    for (int i = 0; i < N; ++i) beta[(size_t)(T - 1) * N + i] = 0.0;
+    for (int t = T - 2; t >= 0; --t)
+        for (int i = 0; i < N; ++i) {
+            for (int b = 0; b < A; ++b) {
+                int nx = ((i << k) | b) & (N - 1);
+                tmp[b] = beta[(size_t)(t + 1) * N + nx] - emis(code, s, t + 1, nx) / temp;
+            }
+            beta[(size_t)t * N + i] = lse_array(tmp, A);
+        }
+}
+
+int orc_bcjr_f64(int L, int k, int T, double temp, const double *s, const double *code,
+                 double *soft, double *log_z, double *alpha_out, double *beta_out)
+{
+    const int N = 1 << L;
+    if (k > 6) return -1;
+    double *alpha = alpha_out ? alpha_out : (double *)malloc(sizeof(double) * (size_t)T * N);
+    double *beta = beta_out ? beta_out : (double *)malloc(sizeof(double) * (size_t)T * N);
+    bcjr_tables(L, k, T, temp, s, code, alpha, beta);
+    double lz = lse_array(alpha + (size_t)(T - 1) * N, N);
+    for (int t = 0; t < T; ++t) {
+        double acc = 0.0;
+        for (int j = 0; j < N; ++j)
+            acc += exp(alpha[(size_t)t * N + j] + beta[(size_t)t * N + j] - lz) * code[j];
+        soft[t] = acc;
+    }
+    if (log_z) *log_z = lz;
+    if (!alpha_out) free(alpha);
+    if (!beta_out) free(beta);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Vector-Jacobian product of the soft codeword, fp64.                      */
+/* grad[u] = d/ds_u sum_t v_t soft_t.  Differentiating the Boltzmann         */
+/* expectation (E is a sum of squares, so dE/ds_u = -2(code[x_u] - s_u)):   */
+/*   d soft_t / d s_u = (2/temp) Cov_p(code[x_t], code[x_u]),               */
+/*   grad[u] = (2/temp) (E_p[F code[x_u]] - E_p[F] soft_u),                 */
+/*   F = sum_t v_t code[x_t].                                               */
+/* E_p[F | x_u = j] is split by the Markov property into the prefix part    */
+/* phi_u(j) (which includes v_u code_j) and the suffix part psi_u(j):       */
+/*   phi_0(j) = v_0 code_j,                                                 */
+/*   phi_t(j) = sum_a w_a phi_{t-1}(pred_a j) + v_t code_j,                 */
+/*              w_a = softmax_a alpha_{t-1}(pred_a j)                       */
+/*   psi_{T-1}(i) = 0,                                                      */
+/*   psi_t(i) = sum_b r_b [v_{t+1} code(succ_b i) + psi_{t+1}(succ_b i)],   */
+/*              r_b = softmax_b [beta_{t+1}(succ_b i) - e_{t+1}(succ_b i)/temp] */
+/*   E_p[F code[x_u]] = sum_j gamma_u(j) code_j (phi_u(j) + psi_u(j)).      */
+/* soft_out (nullable) receives the soft codeword as a by-product.          */
+/* ------------------------------------------------------------------------ */
+int orc_bcjr_vjp_f64(int L, int k, int T, double temp, const double *s, const double *code,
+                     const double *v, double *grad, double *soft_out)
+{
+    const int N = 1 << L, A = 1 << k;
+    if (k > 6) return -1;
+    double *alpha = (double *)malloc(sizeof(double) * (size_t)T * N);
+    double *beta = (double *)malloc(sizeof(double) * (size_t)T * N);
+    double *phi = (double *)malloc(sizeof(double) * (size_t)T * N);
+    double *psi = (double *)malloc(sizeof(double) * (size_t)T * N);
+    double *soft = (double *)malloc(sizeof(double) * (size_t)T);
+    double tmp[64];
+    bcjr_tables(L, k, T, temp, s, code, alpha, beta);
+    double lz = lse_array(alpha + (size_t)(T - 1) * N, N);
+
+    for (int j = 0; j < N; ++j) phi[j] = v[0] * code[j];
+    for (int t = 1; t < T; ++t)
+        for (int j = 0; j < N; ++j) {
+            for (int a = 0; a < A; ++a)
+                tmp[a] = alpha[(size_t)(t - 1) * N + ((j >> k) | (a << (L - k)))];
+            double m = lse_array(tmp, A), acc = 0.0;
+            for (int a = 0; a < A; ++a)
+                acc += exp(tmp[a] - m) * phi[(size_t)(t - 1) * N + ((j >> k) | (a << (L - k)))];
+            phi[(size_t)t * N + j] = acc + v[t] * code[j];
+        }
+    for (int i = 0; i < N; ++i) psi[(size_t)(T - 1) * N + i] = 0.0;
+    for (int t = T - 2; t >= 0; --t)
+        for (int i = 0; i < N; ++i) {
+            for (int b = 0; b < A; ++b) {
+                int nx = ((i << k) | b) & (N - 1);
+                tmp[b] = beta[(size_t)(t + 1) * N + nx] - emis(code, s, t + 1, nx) / temp;
+            }
+            double m = lse_array(tmp, A), acc = 0.0;
+            for (int b = 0; b < A; ++b) {
+                int nx = ((i << k) | b) & (N - 1);
+                acc += exp(tmp[b] - m) * (v[t + 1] * code[nx] + psi[(size_t)(t + 1) * N + nx]);
+            }
+            psi[(size_t)t * N + i] = acc;
+        }
+    double ef = 0.0;
+    for (int t = 0; t < T; ++t) {
+        double acc = 0.0;
+        for (int j = 0; j < N; ++j)
+            acc += exp(alpha[(size_t)t * N + j] + beta[(size_t)t * N + j] - lz) * code[j];
+        soft[t] = acc;
+        ef += v[t] * acc;
+    }
+    for (int u = 0; u < T; ++u) {
+        double acc = 0.0;
+        for (int j = 0; j < N; ++j) {
+            double g = exp(alpha[(size_t)u * N + j] + beta[(size_t)u * N + j] - lz);
+            acc += g * code[j] * (phi[(size_t)u * N + j] + psi[(size_t)u * N + j]);
+        }
+        grad[u] = (2.0 / temp) * (acc - ef * soft[u]);
+    }
+    if (soft_out) memcpy(soft_out, soft, sizeof(double) * (size_t)T);
+    free(alpha); free(beta); free(phi); free(psi); free(soft);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Brute force over every walk (tiny L, T only): the plain definitions.     */
+/* A walk is a first state x_0 in [0, 2^L) and T-1 k-bit digits, with       */
+/* x_t = ((x_{t-1} << k) | digit_t) & (2^L - 1); there are 2^(L + k(T-1))   */
+/* of them.  Outputs: the minimum energy, the Boltzmann log Z at temp, the  */
+/* expectations soft[t] = E[code[x_t]] and (if non-NULL) the T x T matrix   */
+/* second[t*T+u] = E[code[x_t] code[x_u]].  Returns the walk count, or -1   */
+/* if it would exceed 2^24.                                                 */
+/* ------------------------------------------------------------------------ */
+int64_t orc_bruteforce_f64(int L, int k, int T, double temp, const double *s,
+                           const double *code, double *min_energy, double *log_z,
+                           double *soft, double *second)
+{
+    const int bits = L + k * (T - 1);
+    if (bits > 24 || T < 1 || T > 64) return -1;
+    const int64_t W = (int64_t)1 << bits;
+    const uint32_t mask = (1u << L) - 1u;
+    int xs[64];
+    double emin = INFINITY;
+    for (int pass = 0; pass < 2; ++pass) {
+        double z = 0.0;
+        if (pass == 1) {
+            for (int t = 0; t < T; ++t) soft[t] = 0.0;
+            if (second) for (int i = 0; i < T * T; ++i) second[i] = 0.0;
+        }
+        for (int64_t w = 0; w < W; ++w) {
+            /* decode the walk: x_0 is the top L bits of the index, each later   */
+            /* digit the next k bits (the bitstream read most-significant first) */
+            uint64_t code_bits = (uint64_t)w;
+            uint32_t x = (uint32_t)(code_bits >> (k * (T - 1))) & mask;
+            double E = 0.0;
+            for (int t = 0; t < T; ++t) {
+                if (t > 0) {
+                    uint32_t dgt = (uint32_t)(code_bits >> (k * (T - 1 - t))) & ((1u << k) - 1u);
+                    x = ((x << k) | dgt) & mask;
+                }
+                xs[t] = (int)x;
+                double d = code[x] - s[t];
+                E += d * d;
+            }
+            if (pass == 0) {
+                if (E < emin) emin = E;
+            } else {
+                double p = exp(-(E - emin) / temp);
+                z += p;
+                for (int t = 0; t < T; ++t) {
+                    soft[t] += p * code[xs[t]];
+                    if (second)
+                        for (int u = 0; u < T; ++u) second[t * T + u] += p * code[xs[t]] * code[xs[u]];
+                }
+            }
+        }
+        if (pass == 1) {
+            for (int t = 0; t < T; ++t) soft[t] /= z;
+            if (second) for (int i = 0; i < T * T; ++i) second[i] /= z;
+            *log_z = log(z) - emin / temp;
+        }
+    }
+    *min_energy = emin;
+    return W;
+}

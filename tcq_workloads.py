@@ -1,0 +1,118 @@
+"""Seeded synthetic inputs for the bitshift-trellis workloads.
+
+This module holds only input generation: random draws from numpy's PCG64
+``default_rng(seed)``, the random-sign Hadamard rotation that prepares the
+1024x1024 block, and the reshaping of a matrix into 256-weight sequences, one
+per 16x16 tile.  It holds none of the method's arithmetic (no codebook, no
+trellis search, no decode) and is the only module that both the CUDA path's
+tests/benchmark and the CPU oracle's tests use.
+
+Workloads (the pages' shapes and distributions):
+  * gaussian:   n x 256 fp32 weights i.i.d. N(0, 1)          (QTIP blog, Table 1)
+  * rht_block:  1024x1024 N(0,1) block after a seeded random-sign
+                Walsh-Hadamard transform on both sides, cut into 16x16 tiles
+                (QTIP blog, "The trellis" -- RHT from QuIP#; "What it buys end
+                to end" -- one tile = one 256-long sequence)
+  * student_t:  2048x8192 Student-t (nu = 5) rescaled to unit variance, tiled
+  * bitstream:  uniform random 32-bit words, 16 per sequence = a tail-biting
+                2-bit stream of 256 weights (QTIP blog, "Tail-biting")
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+SEQ_LEN = 256
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    L: int
+    n_seq: int
+    kind: str                      # gaussian | rht_block | student_t | bitstream
+    seed: int
+    temps: tuple = ()
+    rows: int = 0
+    cols: int = 0
+    ops: tuple = field(default=())
+
+
+# The five workloads, seeds 1..5.
+WORKLOADS = {
+    "l8_gauss64": Workload("l8_gauss64", 8, 64, "gaussian", 1, (1.0, 0.1),
+                           ops=("viterbi", "bcjr")),
+    "l12_gauss1024": Workload("l12_gauss1024", 12, 1024, "gaussian", 2, (0.05,),
+                              ops=("viterbi", "bcjr", "bcjr_grad")),
+    "l16_rht1024": Workload("l16_rht1024", 16, 4096, "rht_block", 3, (), 1024, 1024,
+                            ops=("viterbi",)),
+    "l16_studentt_2048x8192": Workload("l16_studentt_2048x8192", 16, 65536, "student_t", 4,
+                                       (1.0, 0.1, 0.01), 2048, 8192, ops=("bcjr",)),
+    "l16_decode_8192sq": Workload("l16_decode_8192sq", 16, 262144, "bitstream", 5, (),
+                                  8192, 8192, ops=("decode",)),
+}
+
+
+def tiles_to_sequences(m: np.ndarray) -> np.ndarray:
+    """[R, C] -> [(R/16)*(C/16), 256]: sequence r*(C/16)+c is the 16x16 tile
+    at (16r, 16c), read row-major."""
+    R, C = m.shape
+    assert R % 16 == 0 and C % 16 == 0
+    return np.ascontiguousarray(
+        m.reshape(R // 16, 16, C // 16, 16).transpose(0, 2, 1, 3).reshape(-1, 256))
+
+
+def gaussian(n_seq: int, seed: int, seq_len: int = SEQ_LEN) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((n_seq, seq_len)).astype(np.float32)
+
+
+def _sylvester(n: int) -> np.ndarray:
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def rht_block(seed: int, n: int = 1024) -> np.ndarray:
+    """H diag(sigma1) W diag(sigma2) H^T / n in fp64, cast to fp32 (H Sylvester
+    Hadamard, so H/sqrt(n) is orthonormal and the result stays N(0,1))."""
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((n, n))
+    s1 = rng.integers(0, 2, n) * 2 - 1
+    s2 = rng.integers(0, 2, n) * 2 - 1
+    h = _sylvester(n)
+    out = (h * s1[None, :]) @ w @ (s2[:, None] * h.T) / n
+    return out.astype(np.float32)
+
+
+def student_t_block(seed: int, rows: int = 2048, cols: int = 8192, nu: float = 5.0) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return (rng.standard_t(nu, (rows, cols)) * np.sqrt((nu - 2.0) / nu)).astype(np.float32)
+
+
+def bitstream(n_seq: int, seed: int, words: int = 16) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, 2 ** 32, (n_seq, words), dtype=np.uint32)
+
+
+def sequences(name: str, n_limit: int | None = None) -> np.ndarray:
+    """Target sequences [n, 256] fp32 of a weight workload (optionally the
+    first ``n_limit`` rows only, from the same draw)."""
+    w = WORKLOADS[name]
+    if w.kind == "gaussian":
+        out = gaussian(w.n_seq, w.seed)
+    elif w.kind == "rht_block":
+        out = tiles_to_sequences(rht_block(w.seed, w.rows))
+    elif w.kind == "student_t":
+        out = tiles_to_sequences(student_t_block(w.seed, w.rows, w.cols))
+    else:
+        raise ValueError(f"{name} is a bitstream workload")
+    return out if n_limit is None else np.ascontiguousarray(out[:n_limit])
+
+
+def streams(name: str) -> np.ndarray:
+    w = WORKLOADS[name]
+    assert w.kind == "bitstream"
+    return bitstream(w.n_seq, w.seed)

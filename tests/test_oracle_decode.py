@@ -1,0 +1,93 @@
+"""Pins for the oracle's bitstream decode and pack.
+
+The window formula is the page's decode (QTIP blog, "The trellis: a stateful
+codebook"): with the stream as one integer of nbits bits read most significant
+first, weight t is ``(bits >> (nbits - L - t*k)) & (2^L - 1)``.  Here it is
+evaluated with Python integers, a route independent of the oracle's numpy bit
+arrays.  A tail-biting stream (QTIP blog, "Tail-biting is worth its
+complexity") is exactly k*T bits and its windows wrap around; evaluating the
+same formula on the stream with its first L - k bits appended gives them.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _to_int(words):
+    v = 0
+    for w in words:
+        v = (v << 32) | int(w)
+    return v
+
+
+def _page_window(bits, nbits, t, L, k):
+    return (bits >> (nbits - L - t * k)) & ((1 << L) - 1)
+
+
+@pytest.mark.parametrize("L,T", [(8, 13), (12, 40), (16, 256)])
+def test_free_start_windows_match_page_formula(L, T):
+    k = 2
+    rng = np.random.default_rng(L + T)
+    nw = oracle.stream_words(L, k, T, oracle.FREE_START)
+    words = rng.integers(0, 2 ** 32, (3, nw), dtype=np.uint32)
+    win = oracle.windows(words, L, k, T, oracle.FREE_START)
+    nb = oracle.stream_nbits(L, k, T, oracle.FREE_START)
+    for i in range(3):
+        full = _to_int(words[i]) >> (32 * nw - nb)      # the nb-bit stream
+        for t in range(T):
+            assert win[i, t] == _page_window(full, nb, t, L, k)
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+def test_tailbiting_windows_wrap(L):
+    k, T = 2, 256
+    rng = np.random.default_rng(L)
+    words = rng.integers(0, 2 ** 32, (2, 16), dtype=np.uint32)
+    win = oracle.windows(words, L, k, T, oracle.TAILBITING)
+    for i in range(2):
+        stream = _to_int(words[i])                       # exactly k*T = 512 bits
+        ext = (stream << (L - k)) | (stream >> (k * T - (L - k)))
+        nb = k * T + L - k
+        for t in range(T):
+            assert win[i, t] == _page_window(ext, nb, t, L, k)
+
+
+def _random_walk(rng, n, T, L, k):
+    st = np.empty((n, T), dtype=np.int64)
+    st[:, 0] = rng.integers(0, 1 << L, n)
+    for t in range(1, T):
+        st[:, t] = ((st[:, t - 1] << k) | rng.integers(0, 1 << k, n)) & ((1 << L) - 1)
+    return st
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+def test_pack_then_decode_is_identity_free_start(L):
+    rng = np.random.default_rng(3 * L)
+    st = _random_walk(rng, 5, 256, L, 2)
+    words = oracle.pack(st, L, oracle.FREE_START)
+    assert words.shape[1] == oracle.stream_words(L, 2, 256, oracle.FREE_START)
+    assert np.array_equal(oracle.windows(words, L, 2, 256, oracle.FREE_START), st)
+    dec = oracle.decode(words, L, 256, oracle.FREE_START)
+    assert np.array_equal(dec.view(np.uint16), oracle.codebook_f16(L)[st].view(np.uint16))
+
+
+@pytest.mark.parametrize("L", [8, 16])
+def test_pack_then_decode_is_identity_tailbiting(L):
+    rng = np.random.default_rng(5 * L)
+    words = rng.integers(0, 2 ** 32, (4, 16), dtype=np.uint32)
+    st = oracle.windows(words, L, 2, 256, oracle.TAILBITING)     # a circular walk
+    assert np.array_equal(oracle.pack(st, L, oracle.TAILBITING), words)
+
+
+def test_tile_layout():
+    rng = np.random.default_rng(9)
+    words = rng.integers(0, 2 ** 32, (4 * 6, 16), dtype=np.uint32)
+    m = oracle.decode_tiles(words, 64, 96)
+    seqs = oracle.decode(words, 16, 256)
+    # sequence r*(cols/16)+c is the tile at (16r, 16c), row-major inside it
+    for r in range(4):
+        for c in range(6):
+            tile = m[16 * r:16 * r + 16, 16 * c:16 * c + 16]
+            assert np.array_equal(tile.reshape(-1).view(np.uint16),
+                                  seqs[r * 6 + c].view(np.uint16))

@@ -1,0 +1,102 @@
+"""Pins for the oracle's Viterbi (QTIP blog, "The trellis: a stateful codebook").
+
+* brute force over every walk (2^(L + k(T-1)) of them) gives the same minimum;
+* the returned walk is a bitshift walk and its cost, summed in order, is the
+  returned cost bit for bit (fp32) or to rounding (fp64);
+* fp32 and fp64 walks agree except at decisions closer than 1e-6 relative;
+* the free-start MSE by L printed on the page, and the monotone-code MSE;
+* the MSE stays above the rate-distortion bound D(R) = 2^(-2R).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+from scipy.stats import norm
+
+import oracle
+import tcq_workloads as W
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_figures.json")))
+
+
+def _is_walk(states, L, k):
+    st = np.asarray(states).astype(np.int64)
+    low = (1 << (L - k)) - 1
+    return bool(np.all((st[1:] >> k) == (st[:-1] & low)))
+
+
+@pytest.mark.parametrize("L,k,T", [(4, 2, 6), (6, 2, 5), (8, 2, 4), (4, 1, 10), (6, 3, 4)])
+def test_viterbi_matches_brute_force(L, k, T):
+    rng = np.random.default_rng(1000 + L * 10 + T)
+    for trial in range(4):
+        s = rng.standard_normal(T)
+        bf = oracle.bruteforce(s, L, 1.0, k=k)
+        st, mse, _ = oracle.viterbi_f64(s, L, k=k)
+        assert abs(mse[0] * T - bf["min_energy"]) <= 1e-12 * max(1.0, bf["min_energy"])
+        assert _is_walk(st[0], L, k)
+        c = oracle.codebook_f64(L)
+        path_cost = np.sum((c[st[0].astype(np.int64)] - s) ** 2)
+        assert abs(path_cost - bf["min_energy"]) <= 1e-12 * max(1.0, bf["min_energy"])
+
+
+@pytest.mark.parametrize("L", [4, 6, 8])
+def test_fp32_viterbi_walk_cost_is_sequential_sum(L):
+    s = W.gaussian(16, 7, seq_len=64)
+    st, mse = oracle.viterbi_f32(s, L)
+    c = oracle.codebook_f32(L)
+    for i in range(s.shape[0]):
+        assert _is_walk(st[i], L, 2)
+        acc = np.float32(0.0)
+        for t in range(s.shape[1]):
+            d = np.float32(c[st[i, t]] - s[i, t])
+            acc = np.float32(acc + np.float32(d * d))
+        assert np.float32(acc / np.float32(s.shape[1])) == mse[i]
+
+
+def test_fp32_viterbi_near_brute_force_optimum():
+    rng = np.random.default_rng(5)
+    for _ in range(6):
+        s = rng.standard_normal(5).astype(np.float32)
+        bf = oracle.bruteforce(s.astype(np.float64), 6, 1.0)
+        st, _ = oracle.viterbi_f32(s, 6)
+        c = oracle.codebook_f64(6)
+        cost = np.sum((c[st[0].astype(np.int64)] - s.astype(np.float64)) ** 2)
+        assert cost <= bf["min_energy"] * (1 + 1e-5) + 1e-12
+
+
+@pytest.mark.parametrize("L", [8, 12])
+def test_fp32_and_fp64_walks_agree_off_near_ties(L):
+    s = W.gaussian(24 if L == 8 else 6, 11)
+    st32, mse32 = oracle.viterbi_f32(s, L)
+    st64, mse64, margin = oracle.viterbi_f64(s, L)
+    for i in range(s.shape[0]):
+        if margin[i] >= 1e-6:
+            assert np.array_equal(st32[i], st64[i])
+        # fp32 accumulation of 256 terms stays within 256 * 2^-24 relative
+        assert abs(float(mse32[i]) - mse64[i]) <= 256 * 2.0 ** -24 * mse64[i] + 1e-7
+
+
+@pytest.mark.parametrize("L,n", [(8, 200), (12, 40), (16, 12)])
+def test_free_start_mse_matches_page(L, n):
+    g = GOLD["free_start_mse_by_L"]
+    s = W.gaussian(n, 2024 + L)
+    _, mse = oracle.viterbi_f32(s, L)
+    m = float(np.mean(mse))
+    # page: +-0.002 run to run; the sample mean over n sequences adds
+    # 3 * sd/sqrt(n) of sampling noise (per-sequence sd measured here).
+    tol = g["run_to_run"] + 3 * float(np.std(mse)) / np.sqrt(n)
+    assert abs(m - g[f"L{L}"]) <= tol, (m, g[f"L{L}"], tol)
+    assert m > GOLD["rate_distortion_bound_2bpw"]["value"]
+
+
+@pytest.mark.parametrize("L,n", [(8, 64), (12, 16)])
+def test_monotone_code_loses_to_scalar_rounding(L, n):
+    # Gaussian quantile of (j + 1/2) / 2^L: a codebook monotone in the state
+    g = GOLD["monotone_code_mse_by_L"]
+    code = norm.ppf((np.arange(1 << L) + 0.5) / (1 << L)).astype(np.float32)
+    s = W.gaussian(n, 99)
+    _, mse = oracle.viterbi_f32(s, L, code=code)
+    m = float(np.mean(mse))
+    assert abs(m - g[f"L{L}"]) <= 0.004 + 3 * float(np.std(mse)) / np.sqrt(n), m
+    assert m > 0.118    # worse than the 4-level Lloyd-Max scalar quantiser on the page
