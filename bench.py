@@ -1,0 +1,393 @@
+"""Throughput of the bitshift-trellis hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+for the default workload (L=12, 1024 x 256 i.i.d. N(0,1) weights) that is
+Viterbi encode (forward + traceback, per-sequence MSE), the BCJR soft codeword
+at temp 0.05 and the gradient of the sum of soft codewords w.r.t. the targets.
+The metric is weights per second (whole job, all ranks).  Under torchrun each
+rank encodes its own batch (weak scaling, no data-path collective); the step
+time is the maximum over ranks of the CUDA-event time.
+
+Inputs (1 MiB) are smaller than L2, so L2 is flushed (a 256 MiB write) before
+every timed step, outside the step's event pair.  `--impl reference` times the
+plain CPU oracle on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import tcq_workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "l12_gauss1024"
+METRIC = "weights quantized/sec (Viterbi + BCJR soft + BCJR gradient)"
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def _metric_for(w: W.Workload) -> str:
+    if w.ops == ("decode",):
+        return "decoded weights/sec (2-bit tail-biting stream -> fp16, 16x16 tiles)"
+    parts = []
+    if "viterbi" in w.ops:
+        parts.append("Viterbi")
+    if "bcjr" in w.ops:
+        parts.append("BCJR soft" + (f" x{len(w.temps)} temps" if len(w.temps) > 1 else ""))
+    if "bcjr_grad" in w.ops:
+        parts.append("BCJR gradient")
+    return "weights quantized/sec (" + " + ".join(parts) + ")"
+
+
+def _weights_per_step(w: W.Workload) -> int:
+    return w.n_seq * W.SEQ_LEN
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self) -> dict:
+        rows = [r.split(", ") for r in getattr(self, "out", "").strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            if len(r) < len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(r[0])); mx.append(float(r[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[4:8]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _oracle_step(w: W.Workload, s: np.ndarray) -> None:
+    import oracle
+    if "viterbi" in w.ops:
+        oracle.viterbi_f32(s, w.L)
+    for temp in w.temps:
+        if "bcjr_grad" in w.ops and temp == w.temps[0]:
+            oracle.bcjr_vjp(s, np.ones_like(s, dtype=np.float64), w.L, temp)  # also yields soft
+        elif "bcjr" in w.ops:
+            oracle.bcjr_soft(s, w.L, temp)
+
+
+def _oracle_decode_step(bits: np.ndarray, w: W.Workload) -> None:
+    import oracle
+    oracle.decode(bits, w.L, 256, oracle.TAILBITING)
+
+
+def cpu_baseline(w: W.Workload, budget_s: float = 12.0) -> dict:
+    """Time the oracle, as it stands, on a bounded sample of the workload."""
+    import oracle
+    oracle.build()
+    n_done, t0 = 0, time.perf_counter()
+    if w.ops == ("decode",):
+        bits = W.streams(w.name)
+        chunk = 1024
+        while time.perf_counter() - t0 < budget_s and n_done + chunk <= bits.shape[0]:
+            _oracle_decode_step(bits[n_done:n_done + chunk], w)
+            n_done += chunk
+    else:
+        s = W.sequences(w.name, n_limit=min(w.n_seq, 256))
+        while time.perf_counter() - t0 < budget_s and n_done < s.shape[0]:
+            _oracle_step(w, s[n_done:n_done + 1])
+            n_done += 1
+    dt = time.perf_counter() - t0
+    return {"value": n_done * W.SEQ_LEN / dt, "unit": "weights/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {n_done} of {w.n_seq} sequences of {w.name}, single-threaded, "
+                      f"{dt:.1f} s wall"}
+
+
+def run_reference(a) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = W.WORKLOADS[a.workload]
+    import oracle
+    oracle.build()
+    per_step = 4 if w.ops != ("decode",) else 1024        # sequences per bounded step
+    if w.ops == ("decode",):
+        data = W.streams(w.name)[: per_step * (a.steps + a.warmup)]
+    else:
+        data = W.sequences(w.name, n_limit=min(w.n_seq, per_step * (a.steps + a.warmup)))
+    pos = 0
+    times = []
+    for i in range(a.warmup + a.steps):
+        chunk = data[pos % data.shape[0]: pos % data.shape[0] + per_step]
+        pos += per_step
+        t0 = time.perf_counter()
+        if w.ops == ("decode",):
+            _oracle_decode_step(chunk, w)
+        else:
+            _oracle_step(w, chunk)
+        if i >= a.warmup:
+            times.append(time.perf_counter() - t0)
+    step_s = sum(times) / len(times)
+    value = per_step * W.SEQ_LEN / step_s
+    line = {
+        "impl": "reference", "metric": _metric_for(w), "value": value, "unit": "weights/s",
+        "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "L": w.L, "n_seq": w.n_seq,
+                                        "seq_len": W.SEQ_LEN, "temps": list(w.temps)},
+        "cpu_baseline": {"value": value, "unit": "weights/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} sequences per step of {w.name}, single-threaded"},
+        "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(a) -> None:
+    import torch
+    import trellis_coded_weight_bitshift_b200 as tcq
+    from trellis_coded_weight_bitshift_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    if rank == 0:
+        build()
+    if dist is not None:
+        dist.barrier()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = W.WORKLOADS[a.workload]
+
+    # ---- inputs (each rank its own batch: seed offset by rank) ----
+    if w.ops == ("decode",):
+        host = W.bitstream(w.n_seq, w.seed + 1000 * rank)
+        x = torch.from_numpy(host.view(np.int32)).to(dev).view(torch.uint32)
+        h2d_bytes = host.nbytes
+    else:
+        if rank == 0:
+            host = W.sequences(w.name)
+        else:
+            rng = np.random.default_rng(w.seed + 1000 * rank)
+            host = W.sequences(w.name) if w.kind != "gaussian" else \
+                rng.standard_normal((w.n_seq, W.SEQ_LEN)).astype(np.float32)
+        x = torch.from_numpy(host).to(dev)
+        h2d_bytes = host.nbytes
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    ws_v = ws_b = ws_g = None
+    if "viterbi" in w.ops:
+        ws_v = torch.empty(tcq.viterbi_workspace_size(w.L, 256, w.n_seq), dtype=torch.uint8, device=dev)
+    if "bcjr" in w.ops:
+        ws_b = torch.empty(tcq.bcjr_workspace_size(w.L, 256, w.n_seq), dtype=torch.uint8, device=dev)
+    if "bcjr_grad" in w.ops:
+        ws_g = torch.empty(tcq.bcjr_workspace_size(w.L, 256, w.n_seq, True), dtype=torch.uint8, device=dev)
+    ones = torch.ones((w.n_seq, W.SEQ_LEN), dtype=torch.float32, device=dev)
+
+    kern_ms: dict[str, list[float]] = {}
+    launches_per_step = 0
+
+    def step(inp, timed: bool):
+        nonlocal launches_per_step
+        outs = []
+        ev = []
+        n_launch = 0
+
+        def mark(name):
+            if timed:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(stream)
+                ev.append((name, e))
+
+        if w.ops == ("decode",):
+            mark("start")
+            out = tcq.decode(inp, w.L, 256, tcq.TAILBITING, tcq.OUT_TILE16, w.rows, w.cols)
+            mark("decode_tile16")
+            n_launch += 1
+            outs.append(out)
+        else:
+            mark("start")
+            if "viterbi" in w.ops:
+                st, mse = tcq.viterbi_encode(inp, w.L, ws_v)
+                mark("viterbi")
+                n_launch += 2
+                outs += [st, mse]
+            for i, temp in enumerate(w.temps):
+                soft, lz = tcq.bcjr_soft(inp, w.L, temp, ws_b)
+                mark(f"bcjr_soft_t{temp:g}")
+                n_launch += 1
+                outs += [soft, lz]
+                if "bcjr_grad" in w.ops and i == 0:
+                    g = tcq.bcjr_soft_backward(inp, w.L, temp, soft, ones, ws_g)
+                    mark(f"bcjr_vjp_t{temp:g}")
+                    n_launch += 1
+                    outs.append(g)
+        launches_per_step = n_launch
+        return outs, ev
+
+    for _ in range(a.warmup):
+        step(x, False)
+    torch.cuda.synchronize()
+
+    # ---- device-timed region ----
+    gpu_id = "0"
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[local] if world > 1 else "0"
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = []
+    with ClockSampler(gpu_id) as clk:
+        for _ in range(a.steps):
+            flush.fill_(1)                                   # evict L2 (outside the step's events)
+            _, ev = step(x, True)
+            torch.cuda.synchronize()
+            step_ms.append(ev[0][1].elapsed_time(ev[-1][1]))
+            for (n0, e0), (n1, e1) in zip(ev[:-1], ev[1:]):
+                kern_ms.setdefault(n1, []).append(e0.elapsed_time(e1))
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    mean_ms = sum(step_ms) / len(step_ms)
+    if dist is not None:
+        t = torch.tensor([mean_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mean_ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers ----
+    pinned = torch.from_numpy(host.view(np.int32) if w.ops == ("decode",) else host).pin_memory()
+    e2e_ms = []
+    d2h_bytes = 0
+    for i in range(a.warmup + a.steps):
+        flush.fill_(1)
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        inp = pinned.to(dev, non_blocking=True)
+        if w.ops == ("decode",):
+            inp = inp.view(torch.uint32)
+        outs, _ = step(inp, False)
+        host_outs = []
+        for o in outs:
+            h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+            h.copy_(o, non_blocking=True)
+            host_outs.append(h)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= a.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+        d2h_bytes = sum(o.numel() * o.element_size() for o in outs)
+    e2e_mean = sum(e2e_ms) / len(e2e_ms)
+    if dist is not None:
+        t = torch.tensor([e2e_mean], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_mean = float(t.item())
+
+    units = _weights_per_step(w) * world
+    clocks = clk.summary()
+
+    # ---- roofline of the dominant kernel ----
+    from trellis_coded_weight_bitshift_b200 import roofline as RL
+    kern_mean = {k: sum(v) / len(v) for k, v in kern_ms.items()}
+    dom = max(kern_mean, key=kern_mean.get)
+    peaks = RL.load_measured_peaks(ROOT)
+    roof = RL.roofline_entry(dom, w, kern_mean[dom], peaks)
+
+    line = {
+        "metric": _metric_for(w), "value": units / (mean_ms * 1e-3), "unit": "weights/s",
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": mean_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8" if w.ops == ("decode",) else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "L": w.L, "k": 2, "V": 1, "n_seq_per_gpu": w.n_seq,
+                   "seq_len": W.SEQ_LEN, "temps": list(w.temps), "ops": list(w.ops),
+                   "l2": "flushed (256 MiB write) before every timed step, outside its events",
+                   "parallelism": f"dp{world} (independent batches, no data-path collective)"},
+        "kernels_ms": {k: round(v, 4) for k, v in kern_mean.items()},
+        "roofline": roof,
+        "e2e": {"value": units / (e2e_mean * 1e-3), "unit": "weights/s",
+                "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes)},
+        "gpu_launches": launches_per_step * a.steps,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"]},
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

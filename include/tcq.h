@@ -1,0 +1,188 @@
+/*
+ * tcq.h -- C ABI of the bitshift-trellis coded quantisation library (libtcq.so).
+ *
+ * The library computes, on one NVIDIA B200 (sm_100a), the data-parallel hot
+ * path of trellis-coded weight quantisation on a bitshift trellis:
+ *   - hard Viterbi (min-plus) encoding of many independent weight sequences,
+ *   - the BCJR forward-backward relaxation at a temperature (soft codeword)
+ *     and its vector-Jacobian product,
+ *   - packing state walks into bitstreams and the sliding-window decode of
+ *     those streams to fp16 weights.
+ *
+ * Sources:
+ *   [QTIP]  blog post "QTIP: Trellis-Coded Quantization Puts 2-Bit LLM Weights
+ *           10% Above the Rate-Distortion Bound, and a Monotone Codebook Loses
+ *           to Scalar Rounding", sections "The trellis: a stateful codebook",
+ *           "The codebook is computed", "Tail-biting is worth its complexity",
+ *           "What it buys end to end".
+ *   [BCJR]  "BCJR-QAT: A Differentiable Relaxation of Trellis-Coded Weight
+ *           Quantization", abstract.
+ *
+ * Common conventions
+ *   - The trellis is (L, k, V) with V = 1: 2^L states, each step appends k
+ *     bits; state j may follow state i iff the top L-k bits of j equal the
+ *     bottom L-k bits of i [QTIP, trellis].  Supported: k = 2, V = 1,
+ *     L in {8, 12, 16}, 1 <= seq_len <= 256.  Anything else returns
+ *     TCQ_ERR_UNSUPPORTED.
+ *   - The codebook is 1MAD [QTIP, codebook]: code(j) = (bytesum(34038481 j +
+ *     76625530 mod 2^32) - 510) / 147.8.  Viterbi and BCJR use its fp32 value
+ *     (the fp64 value rounded once to fp32); decode writes its fp16 value
+ *     (round to nearest even).
+ *   - Every array pointer is a DEVICE pointer owned by the caller, contiguous,
+ *     row-major, 16-byte aligned.  The library never allocates, never frees
+ *     and never synchronises the host in these calls: work is enqueued on the
+ *     caller's stream (`stream` is a cudaStream_t passed as void*; NULL = the
+ *     legacy default stream) and outputs are valid once that stream reaches
+ *     the work.  Calls are re-entrant; two calls may share a workspace only if
+ *     they are ordered on the GPU.
+ *   - Arguments are validated on the host before anything is launched; on an
+ *     error no work is enqueued and outputs are untouched.  A failed launch
+ *     returns TCQ_ERR_CUDA (the CUDA error is left for the caller to query).
+ *   - Input values are not checked: non-finite targets give unspecified
+ *     outputs.
+ */
+#ifndef TCQ_H
+#define TCQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TCQ_API __attribute__((visibility("default")))
+#else
+#define TCQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tcq_trellis {
+    int32_t L;        /* state bits (8, 12 or 16) */
+    int32_t k;        /* bits per step (2) */
+    int32_t V;        /* weights per step (1) */
+    int32_t seq_len;  /* weights per sequence, T (1..256) */
+} tcq_trellis_t;
+
+typedef enum tcq_status {
+    TCQ_OK = 0,
+    TCQ_ERR_INVALID_ARG = -1,   /* null pointer, bad size, misalignment, bad enum */
+    TCQ_ERR_UNSUPPORTED = -2,   /* valid but not implemented (L, k, V, seq_len, layout) */
+    TCQ_ERR_WORKSPACE = -3,     /* workspace pointer missing or smaller than required */
+    TCQ_ERR_CUDA = -4           /* a CUDA call or kernel launch failed */
+} tcq_status_t;
+
+/* Bitstream layouts [QTIP, trellis; tail-biting].  Stream bit p of a sequence
+ * sits in 32-bit word p / 32 at bit 31 - p % 32 (read most significant first);
+ * weight t reads the window of bits [k t, k t + L).
+ *   TCQ_TAILBITING: exactly k*T bits, the windows wrap around (needs k*T a
+ *                   multiple of 32 and k*T >= L).
+ *   TCQ_FREE_START: k*T + L - k bits, padded with zeros to whole words. */
+enum { TCQ_TAILBITING = 0, TCQ_FREE_START = 1 };
+
+/* Decode output layouts.
+ *   TCQ_OUT_SEQ:    out[n_seq][seq_len].
+ *   TCQ_OUT_TILE16: out[rows][cols] with sequence r*(cols/16)+c filling the
+ *                   16x16 tile whose top-left element is (16r, 16c), row-major
+ *                   inside the tile [QTIP, "What it buys end to end": each
+ *                   16x16 tile is one 256-long sequence].  Needs seq_len = 256,
+ *                   rows, cols multiples of 16 and rows*cols = 256*n_seq. */
+enum { TCQ_OUT_SEQ = 0, TCQ_OUT_TILE16 = 1 };
+
+/* Library version (major*10000 + minor*100 + patch). */
+TCQ_API int tcq_version(void);
+
+/* Static description of a status code. */
+TCQ_API const char *tcq_status_string(tcq_status_t status);
+
+/* Number of 32-bit words in one sequence's stream for `layout`, or 0 if the
+ * trellis/layout is invalid. */
+TCQ_API size_t tcq_stream_words(const tcq_trellis_t *trellis, int layout);
+
+/* ------------------------------------------------------------------------
+ * Viterbi encode [QTIP, trellis: the min-MSE walk is a shortest path].
+ *   cost_0(j) = (code_j - s_0)^2,
+ *   cost_t(j) = min_a cost_{t-1}((j >> k) | (a << (L-k))) + (code_j - s_t)^2,
+ * free start, free end.  fp32 arithmetic with each operation rounded on its
+ * own (d = code - s, e = d*d, cost = best + e; no fused multiply-add); ties go
+ * to the lowest predecessor digit a, and the final argmin to the lowest state.
+ *
+ *   s          [n_seq][seq_len] fp32 targets (input).
+ *   states     [n_seq][seq_len] uint16: the chosen walk, state (L-bit window)
+ *              of every weight (output).
+ *   mse        [n_seq] fp32: minimum total cost / seq_len (output).
+ *   ws         device workspace of at least tcq_viterbi_workspace_size()
+ *              bytes, 256-byte aligned; it holds the 2-bit backpointers.
+ * Returns TCQ_OK, or an error as described above.
+ * ------------------------------------------------------------------------ */
+TCQ_API size_t tcq_viterbi_workspace_size(const tcq_trellis_t *trellis, int64_t n_seq);
+
+TCQ_API tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *trellis, const float *s, int64_t n_seq,
+                                uint16_t *states, float *mse, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* ------------------------------------------------------------------------
+ * BCJR soft codeword [BCJR: the argmax of Viterbi replaced by forward-backward
+ * sum-product at temperature temp; the soft codeword is the Boltzmann
+ * expectation over trellis walks].  A walk x has energy
+ *   E(x) = sum_t (code(x_t) - s_t)^2
+ * and probability exp(-E/temp)/Z over all walks (free start, free end):
+ *   soft[t] = E_p[code(x_t)],   log_z = log Z (natural log).
+ * fp32, log domain (base 2 inside), renormalised every step.
+ *
+ *   s        [n_seq][seq_len] fp32 (input); temp > 0 and finite.
+ *   soft     [n_seq][seq_len] fp32 (output).
+ *   log_z    [n_seq] fp32 (output, may be NULL).
+ *   ws       device workspace of at least tcq_bcjr_workspace_size(.., 0)
+ *            bytes (per-step forward messages of the sequences in flight).
+ * ------------------------------------------------------------------------ */
+TCQ_API size_t tcq_bcjr_workspace_size(const tcq_trellis_t *trellis, int64_t n_seq, int with_grad);
+
+TCQ_API tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *trellis, const float *s, int64_t n_seq,
+                           float temp, float *soft, float *log_z, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* ------------------------------------------------------------------------
+ * Vector-Jacobian product of the soft codeword [BCJR: the relaxed code is a
+ * smooth function of the targets]:
+ *   grad_s[u] = sum_t grad_soft[t] d soft[t] / d s[u]
+ *             = (2/temp) Cov_p( sum_t grad_soft[t] code(x_t), code(x_u) ).
+ *   soft       [n_seq][seq_len] the forward output of tcq_bcjr_soft for the
+ *              same s and temp (input; used to centre the covariance).
+ *   grad_soft  [n_seq][seq_len] fp32 (input), grad_s [n_seq][seq_len] (output).
+ *   ws         at least tcq_bcjr_workspace_size(.., 1) bytes.
+ * L = 16 returns TCQ_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------ */
+TCQ_API tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *trellis, const float *s,
+                                    int64_t n_seq, float temp, const float *soft,
+                                    const float *grad_soft, float *grad_s, void *ws,
+                                    size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Pack walks into bitstreams [QTIP, trellis: the state is a sliding L-bit
+ * window over the stream].  Stream bits [k t, k t + k) are the top k bits of
+ * state t; a free-start stream ends with the low L-k bits of the last state.
+ * For a valid walk (and, for TCQ_TAILBITING, a circular one) decode of the
+ * result returns code(states).
+ *   states [n_seq][seq_len] uint16 (input), bits [n_seq][tcq_stream_words()]
+ *   uint32 (output).
+ * ------------------------------------------------------------------------ */
+TCQ_API tcq_status_t tcq_pack_states(const tcq_trellis_t *trellis, const uint16_t *states,
+                             int64_t n_seq, int layout, uint32_t *bits, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Sliding-window decode [QTIP, trellis: weight t reads the L-bit window at
+ * stream bit k t, most significant first; every weight decodes on its own].
+ *   bits  [n_seq][tcq_stream_words()] uint32 (input).
+ *   out   fp16 bit patterns (uint16), layout per out_layout (output);
+ *         rows/cols are used by TCQ_OUT_TILE16 only (pass 0 otherwise).
+ * ------------------------------------------------------------------------ */
+TCQ_API tcq_status_t tcq_decode(const tcq_trellis_t *trellis, const uint32_t *bits, int64_t n_seq,
+                        int layout, int out_layout, int64_t rows, int64_t cols,
+                        uint16_t *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TCQ_H */

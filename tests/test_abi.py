@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point that ``include/tcq.h`` declares, and rejects bad arguments
+with the documented status codes before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_names():
+    src = open(os.path.join(ROOT, "include", "tcq.h")).read()
+    return sorted(set(re.findall(r"TCQ_API\s+[\w\s\*]+?\b(tcq_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from trellis_coded_weight_bitshift_b200 import _abi
+    from trellis_coded_weight_bitshift_b200.build import build
+    build()
+    return _abi.lib()
+
+
+def test_header_declares_the_abi():
+    names = _header_names()
+    from trellis_coded_weight_bitshift_b200._abi import EXPORTS
+    assert set(EXPORTS) == set(names), names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _header_names():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    from trellis_coded_weight_bitshift_b200 import _abi
+    for st in (0, -1, -2, -3, -4):
+        assert len(_abi.status_string(st)) > 0
+    assert L.tcq_version() >= 100
+
+
+def test_invalid_arguments_return_status_without_launch(L):
+    from trellis_coded_weight_bitshift_b200 import _abi
+    tr = _abi.trellis(10, 256)                     # unsupported L
+    bad = ctypes.c_void_p(16)                      # never dereferenced on these paths
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, 1, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_UNSUPPORTED
+    tr = _abi.trellis(12, 300)                     # seq_len above 256
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, 1, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_UNSUPPORTED
+    tr = _abi.trellis(12, 256, k=3)
+    assert L.tcq_decode(ctypes.byref(tr), bad, 1, 0, 0, 0, 0, bad, None) == _abi.TCQ_ERR_UNSUPPORTED
+    tr = _abi.trellis(12, 256)
+    # null pointers
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), None, 4, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
+    # misaligned pointer
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), ctypes.c_void_p(18), 4, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
+    # workspace too small / missing / misaligned
+    need = L.tcq_viterbi_workspace_size(ctypes.byref(tr), 4)
+    assert need >= 4 * 255 * 256
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, 4, bad, bad, ctypes.c_void_p(256), need - 1, None) == _abi.TCQ_ERR_WORKSPACE
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, 4, bad, bad, None, need, None) == _abi.TCQ_ERR_WORKSPACE
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, 4, bad, bad, ctypes.c_void_p(128), need, None) == _abi.TCQ_ERR_WORKSPACE
+    # nothing to do
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), None, 0, None, None, None, 0, None) == _abi.TCQ_OK
+    # temperature must be positive and finite
+    assert L.tcq_bcjr_soft(ctypes.byref(tr), bad, 4, ctypes.c_float(0.0), bad, None, bad, 1 << 30, None) == _abi.TCQ_ERR_INVALID_ARG
+    assert L.tcq_bcjr_soft(ctypes.byref(tr), bad, 4, ctypes.c_float(float("inf")), bad, None, bad, 1 << 30, None) == _abi.TCQ_ERR_INVALID_ARG
+    tr16 = _abi.trellis(16, 256)
+    assert L.tcq_bcjr_soft_backward(ctypes.byref(tr16), bad, 4, ctypes.c_float(0.1), bad, bad, bad, bad, 1 << 30, None) == _abi.TCQ_ERR_UNSUPPORTED
+    # decode: tile shape must cover exactly n_seq tiles
+    assert L.tcq_decode(ctypes.byref(tr16), bad, 4, 0, 1, 32, 48, bad, None) == _abi.TCQ_ERR_INVALID_ARG
+    assert L.tcq_decode(ctypes.byref(tr16), bad, 4, 0, 1, 32, 30, bad, None) == _abi.TCQ_ERR_INVALID_ARG
+    assert L.tcq_decode(ctypes.byref(tr16), bad, 4, 7, 0, 0, 0, bad, None) == _abi.TCQ_ERR_INVALID_ARG
+
+
+def test_stream_words(L):
+    from trellis_coded_weight_bitshift_b200 import _abi
+    for Lb in (8, 12, 16):
+        tr = _abi.trellis(Lb, 256)
+        assert L.tcq_stream_words(ctypes.byref(tr), _abi.TAILBITING) == 16
+        assert L.tcq_stream_words(ctypes.byref(tr), _abi.FREE_START) == (512 + Lb - 2 + 31) // 32
+    tr = _abi.trellis(16, 7)                       # 14 bits: too short to wrap a 16-bit window
+    assert L.tcq_stream_words(ctypes.byref(tr), _abi.TAILBITING) == 0
+    assert L.tcq_stream_words(ctypes.byref(tr), _abi.FREE_START) == 1

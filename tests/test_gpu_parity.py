@@ -1,0 +1,272 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Rules:
+  * decode, pack and Viterbi states: bit-exact (integer results).  Viterbi
+    runs in fp32 with every operation rounded on its own on both sides, so
+    the MSE is bit-exact too; against the fp64 oracle the walks agree except
+    on sequences with a decision closer than 1e-6 relative (counted, printed).
+  * BCJR soft codeword: within 1e-4 absolute of the fp64 oracle.
+  * VJP: within 1e-3 * max|g| of the fp64 oracle (fp32 accumulation of a
+    covariance; see the design notes).
+Full-size workloads run on the GPU in the launch configuration the benchmark
+uses; the oracle checks every output it can afford and a seeded sample of the
+rest, and cheap properties (valid walks, sequential MSE) are checked on all.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tcq_workloads as W
+
+pytestmark = pytest.mark.gpu
+
+SOFT_ATOL = 1e-4
+GRAD_RTOL_OF_MAX = 1e-3
+
+
+@pytest.fixture(scope="module")
+def tcq():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import trellis_coded_weight_bitshift_b200 as m
+    from trellis_coded_weight_bitshift_b200.build import build
+    build()
+    return m
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _is_walk(st, L):
+    st = st.astype(np.int64)
+    return np.all((st[:, 1:] >> 2) == (st[:, :-1] & ((1 << (L - 2)) - 1)), axis=1)
+
+
+def _seq_mse_f32(s, st, L):
+    """fp32 sequential sum of (code - s)^2 along each walk, / T."""
+    c = oracle.codebook_f32(L)[st.astype(np.int64)]
+    acc = np.zeros(s.shape[0], dtype=np.float32)
+    for t in range(s.shape[1]):
+        d = (c[:, t] - s[:, t]).astype(np.float32)
+        acc = (acc + (d * d).astype(np.float32)).astype(np.float32)
+    return (acc / np.float32(s.shape[1])).astype(np.float32)
+
+
+# ---------------------------------------------------------------- decode / pack
+def test_decode_tile16_full_8192_square(tcq):
+    bits = W.streams("l16_decode_8192sq")
+    out = tcq.decode(_dev(bits.view(np.int32)).view(torch.uint32), 16, 256, tcq.TAILBITING,
+                     tcq.OUT_TILE16, 8192, 8192)
+    got = out.cpu().numpy().view(np.uint16)
+    ref = oracle.decode_tiles(bits, 8192, 8192).view(np.uint16)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("T", [256, 48, 16, 7])
+def test_decode_seq_layouts(tcq, L, layout, T):
+    if layout == 0 and (2 * T) % 32:
+        pytest.skip("tail-biting needs k*T a multiple of 32")
+    nw = oracle.stream_words(L, 2, T, layout)
+    rng = np.random.default_rng(L * 1000 + T * 10 + layout)
+    bits = rng.integers(0, 2 ** 32, (37, nw), dtype=np.uint32)
+    if layout == 1:                                 # zero padding past the stream end
+        nb = oracle.stream_nbits(L, 2, T, layout)
+        pad = nw * 32 - nb
+        if pad:
+            bits[:, -1] &= np.uint32((0xFFFFFFFF << pad) & 0xFFFFFFFF)
+    out = tcq.decode(_dev(bits.view(np.int32)).view(torch.uint32), L, T, layout, tcq.OUT_SEQ)
+    ref = oracle.decode(bits, L, T, layout)
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), ref.view(np.uint16))
+
+
+def test_decode_tile16_free_start_small(tcq):
+    rng = np.random.default_rng(77)
+    st = np.empty((6 * 5, 256), dtype=np.int64)
+    st[:, 0] = rng.integers(0, 1 << 16, st.shape[0])
+    for t in range(1, 256):
+        st[:, t] = ((st[:, t - 1] << 2) | rng.integers(0, 4, st.shape[0])) & 0xFFFF
+    bits = oracle.pack(st, 16, oracle.FREE_START)
+    out = tcq.decode(_dev(bits.view(np.int32)).view(torch.uint32), 16, 256, tcq.FREE_START,
+                     tcq.OUT_TILE16, 96, 80)
+    ref = oracle.decode_tiles(bits, 96, 80, layout=oracle.FREE_START)
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_pack_matches_oracle_and_roundtrips(tcq, L, layout):
+    rng = np.random.default_rng(L + 31 * layout)
+    n, T = 41, 256
+    if layout == 0:
+        words = rng.integers(0, 2 ** 32, (n, 16), dtype=np.uint32)
+        st = oracle.windows(words, L, 2, T, 0)
+    else:
+        st = np.empty((n, T), dtype=np.int64)
+        st[:, 0] = rng.integers(0, 1 << L, n)
+        for t in range(1, T):
+            st[:, t] = ((st[:, t - 1] << 2) | rng.integers(0, 4, n)) & ((1 << L) - 1)
+    bits = tcq.pack_states(_dev(st.astype(np.uint16).view(np.int16)).view(torch.uint16), L, layout)
+    got = bits.cpu().view(torch.int32).numpy().view(np.uint32)
+    assert np.array_equal(got, oracle.pack(st, L, layout))
+    dec = tcq.decode(bits, L, T, layout, tcq.OUT_SEQ).cpu().numpy().view(np.uint16)
+    assert np.array_equal(dec, oracle.codebook_f16(L)[st].view(np.uint16))
+
+
+# ---------------------------------------------------------------- Viterbi
+def _viterbi_gpu(tcq, s, L):
+    st, mse = tcq.viterbi_encode(_dev(s), L)
+    torch.cuda.synchronize()
+    return st.cpu().view(torch.int16).numpy().view(np.uint16), mse.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["l8_gauss64", "l12_gauss1024"])
+def test_viterbi_full_workload_bit_exact(tcq, name):
+    w = W.WORKLOADS[name]
+    s = W.sequences(name)
+    st, mse = _viterbi_gpu(tcq, s, w.L)
+    rst, rmse = oracle.viterbi_f32(s, w.L)
+    assert np.array_equal(st, rst)
+    assert np.array_equal(mse.view(np.uint32), rmse.view(np.uint32))
+    # against fp64: walks equal off near-ties (reported), MSE within 2e-5 rel
+    n64 = min(s.shape[0], 128)
+    st64, mse64, margin = oracle.viterbi_f64(s[:n64], w.L)
+    near = margin < 1e-6
+    print(f"{name}: {int(near.sum())} near-tie sequences of {n64} (fp64 margin < 1e-6)")
+    assert np.array_equal(st[:n64][~near], st64[~near])
+    assert np.all(np.abs(mse[:n64] - mse64) <= 2e-5 * mse64)
+
+
+def test_viterbi_l16_rht_block(tcq):
+    w = W.WORKLOADS["l16_rht1024"]
+    s = W.sequences("l16_rht1024")
+    st, mse = _viterbi_gpu(tcq, s, 16)
+    assert st.shape == (4096, 256)
+    assert np.all(_is_walk(st, 16))
+    assert np.array_equal(_seq_mse_f32(s, st, 16).view(np.uint32), mse.view(np.uint32))
+    idx = np.random.default_rng(3).choice(4096, 12, replace=False)
+    idx = np.concatenate([[0, 4095], idx])
+    rst, rmse = oracle.viterbi_f32(s[idx], 16)
+    assert np.array_equal(st[idx], rst)
+    assert np.array_equal(mse[idx].view(np.uint32), rmse.view(np.uint32))
+    assert abs(float(mse.mean()) - 0.065) < 0.004       # page: free-start L=16 MSE
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+@pytest.mark.parametrize("T,n", [(1, 3), (2, 5), (3, 1), (17, 9), (100, 2)])
+def test_viterbi_edge_shapes(tcq, L, T, n):
+    s = W.gaussian(n, 500 + T, seq_len=T) * np.float32(1.5)
+    st, mse = _viterbi_gpu(tcq, s, L)
+    rst, rmse = oracle.viterbi_f32(s, L)
+    assert np.array_equal(st, rst)
+    assert np.array_equal(mse.view(np.uint32), rmse.view(np.uint32))
+
+
+def test_viterbi_ties_resolve_to_lowest_index(tcq):
+    # all-zero targets on a codebook with repeated values: many exact ties
+    s = np.zeros((9, 64), dtype=np.float32)
+    s[1] = 0.25
+    s[2, ::2] = -1.0
+    st, mse = _viterbi_gpu(tcq, s, 8)
+    rst, rmse = oracle.viterbi_f32(s, 8)
+    assert np.array_equal(st, rst)
+    assert np.array_equal(mse.view(np.uint32), rmse.view(np.uint32))
+
+
+# ---------------------------------------------------------------- BCJR
+def _bcjr_gpu(tcq, s, L, temp):
+    soft, lz = tcq.bcjr_soft(_dev(s), L, temp)
+    torch.cuda.synchronize()
+    return soft.cpu().numpy(), lz.cpu().numpy()
+
+
+@pytest.mark.parametrize("temp", [1.0, 0.1])
+def test_bcjr_l8_full_workload(tcq, temp):
+    s = W.sequences("l8_gauss64")
+    soft, lz = _bcjr_gpu(tcq, s, 8, temp)
+    rsoft, rlz = oracle.bcjr_soft(s, 8, temp)
+    err = np.abs(soft - rsoft).max()
+    print(f"L=8 temp={temp}: max |soft - oracle| = {err:.2e}")
+    assert err <= SOFT_ATOL
+    assert np.all(np.abs(lz - rlz) <= 1e-5 * np.abs(rlz) + 1e-4)
+
+
+def test_bcjr_l12_workload(tcq):
+    s = W.sequences("l12_gauss1024")
+    soft, lz = _bcjr_gpu(tcq, s, 12, 0.05)
+    idx = np.concatenate([[0, 1023], np.random.default_rng(12).choice(1024, 30, replace=False)])
+    rsoft, rlz = oracle.bcjr_soft(s[idx], 12, 0.05)
+    err = np.abs(soft[idx] - rsoft).max()
+    print(f"L=12 temp=0.05: max |soft - oracle| = {err:.2e} over {len(idx)} sequences")
+    assert err <= SOFT_ATOL
+    assert np.all(np.abs(lz[idx] - rlz) <= 1e-5 * np.abs(rlz) + 1e-3)
+    assert np.all(np.isfinite(soft))
+
+
+@pytest.mark.parametrize("temp", [1.0, 0.1, 0.01])
+def test_bcjr_l16_student_t(tcq, temp):
+    s = W.sequences("l16_studentt_2048x8192")
+    soft, lz = _bcjr_gpu(tcq, s, 16, temp)
+    assert np.all(np.isfinite(soft)) and np.all(np.isfinite(lz))
+    c = oracle.codebook_f64(16)
+    assert soft.min() >= c.min() - 1e-4 and soft.max() <= c.max() + 1e-4
+    idx = np.array([0, 65535, int(np.random.default_rng(int(temp * 100)).integers(1, 65535))])
+    rsoft, rlz = oracle.bcjr_soft(s[idx], 16, temp)
+    err = np.abs(soft[idx] - rsoft).max()
+    print(f"L=16 temp={temp}: max |soft - oracle| = {err:.2e}")
+    assert err <= SOFT_ATOL
+    assert np.all(np.abs(lz[idx] - rlz) <= 1e-5 * np.abs(rlz) + 1e-3)
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+@pytest.mark.parametrize("T,n", [(1, 2), (2, 3), (5, 9), (33, 1)])
+def test_bcjr_edge_shapes(tcq, L, T, n):
+    s = W.gaussian(n, 900 + T, seq_len=T)
+    soft, lz = _bcjr_gpu(tcq, s, L, 0.3)
+    rsoft, rlz = oracle.bcjr_soft(s, L, 0.3)
+    assert np.abs(soft - rsoft).max() <= SOFT_ATOL
+    assert np.all(np.abs(lz - rlz) <= 1e-5 * np.abs(rlz) + 1e-4)
+
+
+def test_bcjr_low_temperature_matches_viterbi_codeword(tcq):
+    s = W.sequences("l8_gauss64")[:16]
+    soft, _ = _bcjr_gpu(tcq, s, 8, 1e-4)
+    st, _, margin = oracle.viterbi_f64(s, 8)
+    hard = oracle.codebook_f64(8)[st.astype(np.int64)]
+    ok = margin > 1e-2
+    assert ok.sum() >= 4
+    assert np.abs(soft[ok] - hard[ok]).max() <= 1e-4
+
+
+# ---------------------------------------------------------------- VJP
+@pytest.mark.parametrize("name,temp,nsample", [("l12_gauss1024", 0.05, 12), ("l8_gauss64", 0.1, 64)])
+def test_vjp_matches_oracle(tcq, name, temp, nsample):
+    w = W.WORKLOADS[name]
+    s = W.sequences(name)
+    v = np.ones_like(s)                      # gradient of sum of soft codewords
+    sd = _dev(s)
+    soft, _ = tcq.bcjr_soft(sd, w.L, temp)
+    g = tcq.bcjr_soft_backward(sd, w.L, temp, soft, _dev(v))
+    torch.cuda.synchronize()
+    g = g.cpu().numpy()
+    assert np.all(np.isfinite(g))
+    idx = np.arange(s.shape[0]) if nsample >= s.shape[0] else \
+        np.random.default_rng(5).choice(s.shape[0], nsample, replace=False)
+    rg, _ = oracle.bcjr_vjp(s[idx], v[idx], w.L, temp)
+    for i, j in enumerate(idx):
+        tol = GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+        assert np.abs(g[j] - rg[i]).max() <= tol, (j, np.abs(g[j] - rg[i]).max(), tol)
+
+
+def test_vjp_random_cotangent_and_autograd(tcq):
+    s = W.gaussian(5, 61, seq_len=40)
+    v = W.gaussian(5, 62, seq_len=40)
+    sd = _dev(s).requires_grad_(True)
+    soft = tcq.BcjrSoft.apply(sd, 8, 0.2)
+    (soft * _dev(v)).sum().backward()
+    g = sd.grad.cpu().numpy()
+    rg, _ = oracle.bcjr_vjp(s, v, 8, 0.2)
+    for i in range(5):
+        assert np.abs(g[i] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()

@@ -1,0 +1,168 @@
+"""Bitshift-trellis coded quantisation on NVIDIA B200 (sm_100a).
+
+Thin PyTorch binding of ``libtcq.so`` (C ABI in ``include/tcq.h``).  Every
+step of the computation runs in the library's CUDA kernels; this module only
+checks tensor shapes, allocates outputs and workspaces with torch's caching
+allocator and passes device pointers and the current CUDA stream.  There is
+no CPU fallback: without the built library or a CUDA device every call raises.
+
+Functions (QTIP blog "The trellis: a stateful codebook" / "The codebook is
+computed" / "Tail-biting is worth its complexity"; BCJR-QAT abstract):
+  viterbi_encode(s, L)                   -> (states uint16 [n,T], mse f32 [n])
+  bcjr_soft(s, L, temp)                  -> (soft f32 [n,T], log_z f32 [n])
+  bcjr_soft_backward(s, L, temp, soft, g)-> grad_s f32 [n,T]
+  BcjrSoft.apply(s, L, temp)             -> soft (autograd through the VJP)
+  pack_states(states, L, layout)         -> bits uint32 [n, words]
+  decode(bits, L, T, layout, ...)        -> fp16 weights
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import (FREE_START, OUT_SEQ, OUT_TILE16, TAILBITING, TcqError, check, lib,
+                   status_string, trellis)
+
+__all__ = [
+    "viterbi_encode", "bcjr_soft", "bcjr_soft_backward", "BcjrSoft", "pack_states", "decode",
+    "stream_words", "viterbi_workspace_size", "bcjr_workspace_size", "TcqError",
+    "TAILBITING", "FREE_START", "OUT_SEQ", "OUT_TILE16", "lib", "status_string",
+]
+
+
+def _require_cuda(*tensors: torch.Tensor) -> None:
+    for t in tensors:
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors (no CPU fallback)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # 256-byte aligned: the caching allocator hands out 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def stream_words(L: int, seq_len: int, layout: int) -> int:
+    return int(lib().tcq_stream_words(ctypes.byref(trellis(L, seq_len)), int(layout)))
+
+
+def viterbi_workspace_size(L: int, seq_len: int, n_seq: int) -> int:
+    return int(lib().tcq_viterbi_workspace_size(ctypes.byref(trellis(L, seq_len)), int(n_seq)))
+
+
+def bcjr_workspace_size(L: int, seq_len: int, n_seq: int, with_grad: bool = False) -> int:
+    return int(lib().tcq_bcjr_workspace_size(ctypes.byref(trellis(L, seq_len)), int(n_seq),
+                                             int(bool(with_grad))))
+
+
+def viterbi_encode(s: torch.Tensor, L: int, workspace: torch.Tensor | None = None):
+    """Min-MSE walk of every row of ``s`` [n, T] (fp32) on the (L, 2, 1)
+    bitshift trellis with the 1MAD code; returns (states uint16, mse fp32)."""
+    _require_cuda(s)
+    if s.dtype != torch.float32 or s.dim() != 2:
+        raise ValueError("s must be a 2-D float32 tensor [n_seq, seq_len]")
+    n, T = s.shape
+    tr = trellis(L, T)
+    states = torch.empty((n, T), dtype=torch.uint16, device=s.device)
+    mse = torch.empty((n,), dtype=torch.float32, device=s.device)
+    need = int(lib().tcq_viterbi_workspace_size(ctypes.byref(tr), n))
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    check(lib().tcq_viterbi_encode(ctypes.byref(tr), _ptr(s), n, _ptr(states), _ptr(mse), _ptr(ws),
+                                   ws.numel(), _stream()), "tcq_viterbi_encode")
+    return states, mse
+
+
+def bcjr_soft(s: torch.Tensor, L: int, temp: float, workspace: torch.Tensor | None = None):
+    """Soft codeword (Boltzmann expectation of the code at temperature
+    ``temp``) of every row of ``s``; returns (soft fp32 [n,T], log_z fp32 [n])."""
+    _require_cuda(s)
+    if s.dtype != torch.float32 or s.dim() != 2:
+        raise ValueError("s must be a 2-D float32 tensor [n_seq, seq_len]")
+    n, T = s.shape
+    tr = trellis(L, T)
+    soft = torch.empty_like(s)
+    logz = torch.empty((n,), dtype=torch.float32, device=s.device)
+    need = int(lib().tcq_bcjr_workspace_size(ctypes.byref(tr), n, 0))
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    check(lib().tcq_bcjr_soft(ctypes.byref(tr), _ptr(s), n, float(temp), _ptr(soft), _ptr(logz),
+                              _ptr(ws), ws.numel(), _stream()), "tcq_bcjr_soft")
+    return soft, logz
+
+
+def bcjr_soft_backward(s: torch.Tensor, L: int, temp: float, soft: torch.Tensor,
+                       grad_soft: torch.Tensor, workspace: torch.Tensor | None = None):
+    """Vector-Jacobian product: grad_s[u] = sum_t grad_soft[t] d soft[t] / d s[u]."""
+    _require_cuda(s, soft, grad_soft)
+    if s.shape != soft.shape or s.shape != grad_soft.shape:
+        raise ValueError("s, soft and grad_soft must have the same shape")
+    n, T = s.shape
+    tr = trellis(L, T)
+    grad = torch.empty_like(s)
+    need = int(lib().tcq_bcjr_workspace_size(ctypes.byref(tr), n, 1))
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    check(lib().tcq_bcjr_soft_backward(ctypes.byref(tr), _ptr(s), n, float(temp), _ptr(soft),
+                                       _ptr(grad_soft), _ptr(grad), _ptr(ws), ws.numel(),
+                                       _stream()), "tcq_bcjr_soft_backward")
+    return grad
+
+
+class BcjrSoft(torch.autograd.Function):
+    """soft = BcjrSoft.apply(s, L, temp): differentiable soft codeword."""
+
+    @staticmethod
+    def forward(ctx, s, L, temp):
+        soft, _ = bcjr_soft(s, L, temp)
+        ctx.save_for_backward(s, soft)
+        ctx.L, ctx.temp = L, temp
+        return soft
+
+    @staticmethod
+    def backward(ctx, g):
+        s, soft = ctx.saved_tensors
+        return bcjr_soft_backward(s, ctx.L, ctx.temp, soft, g.contiguous()), None, None
+
+
+def pack_states(states: torch.Tensor, L: int, layout: int = FREE_START) -> torch.Tensor:
+    """Pack walks [n, T] (uint16) into MSB-first bitstreams [n, words] (uint32)."""
+    _require_cuda(states)
+    if states.dtype != torch.uint16 or states.dim() != 2:
+        raise ValueError("states must be a 2-D uint16 tensor")
+    n, T = states.shape
+    tr = trellis(L, T)
+    words = int(lib().tcq_stream_words(ctypes.byref(tr), int(layout)))
+    if words == 0:
+        raise TcqError(_abi.TCQ_ERR_UNSUPPORTED, "tcq_stream_words")
+    bits = torch.empty((n, words), dtype=torch.uint32, device=states.device)
+    check(lib().tcq_pack_states(ctypes.byref(tr), _ptr(states), n, int(layout), _ptr(bits),
+                                _stream()), "tcq_pack_states")
+    return bits
+
+
+def decode(bits: torch.Tensor, L: int, seq_len: int = 256, layout: int = TAILBITING,
+           out_layout: int = OUT_SEQ, rows: int = 0, cols: int = 0,
+           out: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode bitstreams [n, words] (uint32) into fp16 weights: [n, seq_len]
+    (OUT_SEQ) or a [rows, cols] matrix of 16x16 tiles (OUT_TILE16)."""
+    _require_cuda(bits)
+    if bits.dtype != torch.uint32 or bits.dim() != 2:
+        raise ValueError("bits must be a 2-D uint32 tensor")
+    n = bits.shape[0]
+    tr = trellis(L, seq_len)
+    if out is None:
+        shape = (rows, cols) if out_layout == OUT_TILE16 else (n, seq_len)
+        out = torch.empty(shape, dtype=torch.float16, device=bits.device)
+    _require_cuda(out)
+    check(lib().tcq_decode(ctypes.byref(tr), _ptr(bits), n, int(layout), int(out_layout), int(rows),
+                           int(cols), _ptr(out), _stream()), "tcq_decode")
+    return out

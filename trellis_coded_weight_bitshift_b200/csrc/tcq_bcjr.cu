@@ -1,0 +1,572 @@
+// BCJR forward-backward on the bitshift trellis at temperature temp, and the
+// vector-Jacobian product of the soft codeword.
+//
+// [BCJR-QAT abstract] the Viterbi argmax is replaced by the forward-backward
+// sum-product recursion at temperature temp; the soft codeword is the
+// Boltzmann expectation of the code over trellis walks and is exactly
+// differentiable.  With E(x) = sum_t (code(x_t) - s_t)^2 and p(x) ~ exp(-E/temp)
+// (free start, free end):
+//   alpha_0(j) = -e_0(j)/temp,  alpha_t(j) = LSE_a alpha_{t-1}(pred_a j) - e_t(j)/temp
+//   beta_{T-1} = 0,             beta_t(i)  = LSE_b [beta_{t+1}(succ_b i) - e_{t+1}(succ_b i)/temp]
+//   soft_t = sum_j softmax_j(alpha_t + beta_t) code_j
+// Everything here runs in base 2 (kappa = log2(e)/temp scales the energy) on
+// the MUFU ex2/lg2 units, fp32.
+//
+// Structure (k = 2, the same one as the Viterbi kernel):
+//   * forward: the four states j = 4q + b share one log-sum-exp over their
+//     predecessors, A_t(q) = LSE_a alpha_{t-1}(q | a << (L-2)), so the state
+//     vector carried between steps is A (2^(L-2) values) and
+//     alpha_t(p) = A_t(p >> 2) - kappa e_t(p) is rebuilt on the fly;
+//   * backward: beta_t(i) depends only on i's low L-2 bits,
+//     B_t(r) = LSE_b [B_{t+1}((4r + b) mod 2^(L-2)) - kappa e_{t+1}(4r + b)],
+//     and thread w evaluates exactly the groups r whose states 4r + b are its
+//     forward predecessor states, so the code values in its registers serve
+//     both passes (the backward reads G contiguous values, writes four runs:
+//     the mirror image of the forward step);
+//   * combine: alpha_{t+1}(4r+b) + beta_{t+1}(4r+b) = A_{t+1}(r) + y_b where
+//     y_b are the four inputs of the backward log-sum-exp for r, so the soft
+//     codeword reuses those four exponentials plus one for the group weight;
+//   * A_t is renormalised every step by the running maximum (a constant per
+//     step, global over the sequence), and so is B; the constants are tracked
+//     to place the combine's exponent reference K_t = log2 Z - (constants)
+//     near zero, and soft_t = num_t / den_t cancels K_t exactly;
+//   * the forward spills, per thread and per step, the A values it read to
+//     its private slice of the workspace, and the backward reads them back in
+//     reverse order (thread-private, so no inter-thread ordering is needed).
+//
+// Gradient (GRAD = true): d soft_t / d s_u = (2/temp) Cov(code(x_t), code(x_u)),
+// so grad_u = (2/temp) Cov(F, code(x_u)) with F = sum_t v_t (code(x_t) - soft_t)
+// (centred by the forward soft codeword).  E[F | x_u = j] splits by the Markov
+// property into a prefix part phi (forward expectation recursion, weights =
+// the forward softmax over predecessors) and a suffix part psi (backward
+// recursion, weights = the backward softmax over successors); both reuse the
+// exponentials of the log-sum-exps above.
+#include <algorithm>
+
+#include "tcq_device.cuh"
+
+namespace tcq {
+
+template <int L_, int G_, int SPC_, int AREG_, int NBUF_, bool GRAD_>
+struct BcjrCfg {
+  static constexpr int L = L_, G = G_, SPC = SPC_, AREG = AREG_, NBUF = NBUF_;
+  static constexpr bool GRAD = GRAD_;
+  static constexpr int NG = 1 << (L - 2);
+  static constexpr int TPS = NG / G;
+  static constexpr int NT = TPS * SPC;
+  static constexpr int GQ = G / 4;
+  static constexpr int ASM = 4 - AREG;
+  static constexpr int NPART = TPS >= 32 ? TPS / 32 : 1;       // partial records per sequence
+  static constexpr int PREC = 8;                                 // floats per partial record
+  static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
+  static constexpr int NV = GRAD ? 2 : 1;                        // carried vectors (A | A, Phi)
+  static constexpr int SPILL = NV * G;                           // floats spilled per thread-step
+  static constexpr size_t smem_floats() {
+    return (size_t)SPC * NBUF * NV * NG                            // state vectors
+           + (size_t)ASM * G * TPS                                  // smem code values
+           + (size_t)SPC * 256 * (GRAD ? 3 : 1)                     // s (+ v, soft)
+           + (size_t)SPC * 256                                       // CA_t prefix sums
+           + (size_t)2 * SPC * NPART * PREC;                        // partial records
+  }
+  static constexpr size_t smem_bytes() { return smem_floats() * sizeof(float); }
+  __host__ __device__ static constexpr size_t ws_floats_per_slot(int T) { return (size_t)T * NV * NG; }
+  static_assert(NG % G == 0 && G % 4 == 0, "bad split");
+  static_assert(SPILL % 4 == 0, "spill in float4 chunks");
+};
+
+template <class C>
+__device__ __forceinline__ float code_at(const float (&creg)[C::AREG > 0 ? C::AREG : 1][C::G],
+                                         const float *Csm, int a, int i, int w) {
+  if (a < C::AREG) return creg[a < C::AREG ? a : 0][i];
+  return Csm[((a - C::AREG) * C::GQ + (i >> 2)) * C::TPS * 4 + w * 4 + (i & 3)];
+}
+
+// Reduce within the TPS lanes of a sequence (TPS < 32) or the whole warp.
+template <int TPS, class Op>
+__device__ __forceinline__ float lane_reduce(float v, Op op) {
+  constexpr int WL = TPS < 32 ? TPS : 32;
+#pragma unroll
+  for (int off = WL / 2; off > 0; off >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+struct MaxOp { __device__ float operator()(float a, float b) const { return fmaxf(a, b); } };
+struct SumOp { __device__ float operator()(float a, float b) const { return a + b; } };
+
+// GQ contiguous state-vector values of run `base` (swizzled shared memory).
+template <class C>
+__device__ __forceinline__ void read_run(const float *vec, int base, float *dst) {
+  constexpr int GQ = C::GQ;
+  if constexpr (GQ == 1) {
+    dst[0] = vec[swz<C::SWZ>(base)];
+  } else if constexpr (GQ == 2) {
+    const float2 v = *reinterpret_cast<const float2 *>(vec + swz<C::SWZ>(base));
+    dst[0] = v.x; dst[1] = v.y;
+  } else {
+#pragma unroll
+    for (int q = 0; q < GQ / 4; ++q) {
+      const float4 v = *reinterpret_cast<const float4 *>(vec + swz<C::SWZ>(base + 4 * q));
+      dst[4 * q] = v.x; dst[4 * q + 1] = v.y; dst[4 * q + 2] = v.z; dst[4 * q + 3] = v.w;
+    }
+  }
+}
+
+template <class C>
+__device__ __forceinline__ void write_run(float *vec, int base, const float *src) {
+  constexpr int GQ = C::GQ;
+  if constexpr (GQ == 1) {
+    vec[swz<C::SWZ>(base)] = src[0];
+  } else if constexpr (GQ == 2) {
+    *reinterpret_cast<float2 *>(vec + swz<C::SWZ>(base)) = make_float2(src[0], src[1]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < GQ / 4; ++q)
+      *reinterpret_cast<float4 *>(vec + swz<C::SWZ>(base + 4 * q)) =
+          make_float4(src[4 * q], src[4 * q + 1], src[4 * q + 2], src[4 * q + 3]);
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::NT, 1)
+bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, float two_over_temp,
+            const float *__restrict__ vgrad, const float *__restrict__ soft_in,
+            float *__restrict__ soft_out, float *__restrict__ logz_out,
+            float *__restrict__ grad_out, float *__restrict__ ws) {
+  constexpr int NG = C::NG, G = C::G, GQ = C::GQ, TPS = C::TPS, NB = C::NBUF, NV = C::NV;
+  constexpr int NPART = C::NPART, SPC = C::SPC, PREC = C::PREC, NCH = C::SPILL / 4;
+  constexpr bool GRAD = C::GRAD;
+  extern __shared__ __align__(16) float smem[];
+  float *Vall = smem;                                      // [SPC][NB][NV][NG]
+  float *Csm = Vall + SPC * NB * NV * NG;                  // [ASM][GQ][TPS][4]
+  float *ssm = Csm + C::ASM * G * TPS;                     // [SPC][256]
+  float *vsm = ssm + SPC * 256;                            // GRAD: v, soft rows
+  float *fsm = vsm + (GRAD ? SPC * 256 : 0);
+  float *cah = fsm + (GRAD ? SPC * 256 : 0);               // [SPC][256] CA_t
+  float *part = cah + SPC * 256;                           // [2][SPC][NPART][PREC]
+
+  const int tid = threadIdx.x;
+  const int ls = tid / TPS, w = tid - ls * TPS;
+  const int lane = tid & 31;
+  const int pidx = TPS >= 32 ? (w >> 5) : 0;
+  const bool plead = TPS >= 32 ? (lane == 0) : (w == 0);
+
+  float creg[C::AREG > 0 ? C::AREG : 1][G];
+#pragma unroll
+  for (int a = 0; a < C::AREG; ++a)
+#pragma unroll
+    for (int i = 0; i < G; ++i) creg[a][i] = one_mad_f32((uint32_t)(a * NG + G * w + i));
+  if (ls == 0) {
+    for (int a = 0; a < C::ASM; ++a)
+      for (int i = 0; i < G; ++i)
+        Csm[(a * GQ + (i >> 2)) * TPS * 4 + w * 4 + (i & 3)] =
+            one_mad_f32((uint32_t)((a + C::AREG) * NG + G * w + i));
+  }
+
+  // thread-private spill: [T][NCH][TPS] float4; step t holds A_t (and Phi_t)
+  // at this thread's groups r = a*NG/4 + GQ*w + k, flattened as a*GQ + k.
+  float4 *spill = reinterpret_cast<float4 *>(ws + (size_t)(blockIdx.x * SPC + ls) *
+                                                      C::ws_floats_per_slot(T));
+  auto prec = [&](int parity) { return part + ((parity * SPC + ls) * NPART) * PREC; };
+
+  for (int64_t base = (int64_t)blockIdx.x * SPC; base < n_seq; base += (int64_t)gridDim.x * SPC) {
+    const int64_t seq = base + ls;
+    const bool active = seq < n_seq;
+    __syncthreads();                                       // previous sequence fully done
+    for (int x = tid; x < SPC * T; x += C::NT) {
+      const int l = x / T, t = x - l * T;
+      const int64_t sq = base + l;
+      const bool ok = sq < n_seq;
+      ssm[l * 256 + t] = ok ? s[sq * T + t] : 0.0f;
+      if (GRAD) {
+        vsm[l * 256 + t] = ok ? vgrad[sq * T + t] : 0.0f;
+        fsm[l * 256 + t] = ok ? soft_in[sq * T + t] : 0.0f;
+      }
+    }
+    float *V = Vall + ls * NB * NV * NG;
+    for (int x = w; x < NV * NG; x += TPS) V[x] = 0.0f;     // A_0 = 0 (and Phi_0 = 0)
+    for (int x = tid; x < 2 * SPC * NPART * PREC; x += C::NT) part[x] = 0.0f;
+    __syncthreads();
+
+    // ---------------- forward ----------------
+    // A_t is stored relative to CA_t = c_0 + ... + c_{t-1}, c_t = max of stored A_t.
+    float CA = 0.0f, cmax = 0.0f;
+    for (int t = 1; t <= T; ++t) {
+      const float *Ai = V + ((t - 1) % NB) * NV * NG;
+      float ain[4][GQ], fin[GRAD ? 4 : 1][GQ];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        read_run<C>(Ai, a * (NG / 4) + GQ * w, ain[a]);
+        if (GRAD) read_run<C>(Ai + NG, a * (NG / 4) + GQ * w, fin[a < (GRAD ? 4 : 1) ? a : 0]);
+      }
+      cmax = 0.0f;
+      if (t > 1) {
+        const float *pp = prec((t - 1) & 1);
+        cmax = pp[0];
+#pragma unroll
+        for (int x = 1; x < NPART; ++x) cmax = fmaxf(cmax, pp[x * PREC]);
+      }
+      {   // spill A_{t-1} (and Phi_{t-1}) at this thread's groups
+        float flat[C::SPILL];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int k = 0; k < GQ; ++k) {
+            flat[a * GQ + k] = ain[a][k];
+            if (GRAD) flat[G + a * GQ + k] = fin[a < (GRAD ? 4 : 1) ? a : 0][k];
+          }
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+          spill[((size_t)(t - 1) * NCH + c) * TPS + w] =
+              make_float4(flat[4 * c], flat[4 * c + 1], flat[4 * c + 2], flat[4 * c + 3]);
+      }
+      if (w == 0) cah[ls * 256 + t - 1] = CA;
+      if (t == T) break;
+      if (NB == 1) __syncthreads();
+      CA += cmax;
+      float *Ao = V + (t % NB) * NV * NG;
+      const float sv = ssm[ls * 256 + t - 1];
+      const float vv = GRAD ? vsm[ls * 256 + t - 1] : 0.0f;
+      const float fv = GRAD ? fsm[ls * 256 + t - 1] : 0.0f;
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < GQ; ++q) {
+        float outA[4], outF[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = 4 * q + r;
+          float x[4], c[4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            c[a] = code_at<C>(creg, Csm, a, i, w);
+            const float d = c[a] - sv;
+            x[a] = fmaf(-kappa * d, d, ain[a][q] - cmax);
+          }
+          const float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+          float u[4], S = 0.0f;
+#pragma unroll
+          for (int a = 0; a < 4; ++a) { u[a] = ex2(x[a] - mx); S += u[a]; }
+          outA[r] = mx + lg2(S);
+          tmax = fmaxf(tmax, outA[r]);
+          if (GRAD) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+              acc = fmaf(u[a], fin[a < (GRAD ? 4 : 1) ? a : 0][q] + vv * (c[a] - fv), acc);
+            outF[r] = acc * __frcp_rn(S);
+          }
+        }
+        *reinterpret_cast<float4 *>(Ao + swz<C::SWZ>(G * w + 4 * q)) =
+            make_float4(outA[0], outA[1], outA[2], outA[3]);
+        if (GRAD)
+          *reinterpret_cast<float4 *>(Ao + NG + swz<C::SWZ>(G * w + 4 * q)) =
+              make_float4(outF[0], outF[1], outF[2], outF[3]);
+      }
+      tmax = lane_reduce<TPS>(tmax, MaxOp());
+      if (plead) prec(t & 1)[pidx * PREC] = tmax;
+      __syncthreads();
+    }
+    // CA = CA_{T-1}; cmax = max of stored A_{T-1}; spill step T-1 holds A_{T-1}.
+
+    // ---------------- log2 Z = LSE over all states at T-1 ----------------
+    float log2Z;
+    {
+      const float sT = ssm[ls * 256 + T - 1];
+      float vals[4][GQ], vmax = -INFINITY;
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        float av[GQ];
+#pragma unroll
+        for (int q = 0; q < (GQ + 3) / 4; ++q) {
+          const int f = a * GQ + 4 * q;
+          const float4 v = spill[((size_t)(T - 1) * NCH + (f >> 2)) * TPS + w];
+          const float e4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) av[4 * q + k] = e4[(f & 3) + k];
+        }
+#pragma unroll
+        for (int k = 0; k < GQ; ++k) {
+          float y[4];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const float d = code_at<C>(creg, Csm, a, 4 * k + b, w) - sT;
+            y[b] = -kappa * d * d;
+          }
+          const float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+          const float S = ex2(y[0] - mx) + ex2(y[1] - mx) + ex2(y[2] - mx) + ex2(y[3] - mx);
+          vals[a][k] = (av[k] - cmax) + mx + lg2(S);
+          vmax = fmaxf(vmax, vals[a][k]);
+        }
+      }
+      vmax = lane_reduce<TPS>(vmax, MaxOp());
+      float *pp = prec(0);
+      if (plead) pp[pidx * PREC + 5] = vmax;
+      __syncthreads();
+      vmax = pp[5];
+#pragma unroll
+      for (int x = 1; x < NPART; ++x) vmax = fmaxf(vmax, pp[x * PREC + 5]);
+      float sum = 0.0f;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int k = 0; k < GQ; ++k) sum += ex2(vals[a][k] - vmax);
+      sum = lane_reduce<TPS>(sum, SumOp());
+      if (plead) pp[pidx * PREC + 6] = sum;
+      __syncthreads();
+      float tot = 0.0f;
+#pragma unroll
+      for (int x = 0; x < NPART; ++x) tot += pp[x * PREC + 6];
+      log2Z = vmax + lg2(tot) + cmax + CA;
+    }
+    if (w == 0 && active && logz_out) logz_out[seq] = log2Z * 0.69314718055994531f;
+
+    // ---------------- backward + combine ----------------
+    // B_t is stored relative to DB_t (sum of the maxima removed); the combine
+    // at step tc uses K = log2Z - CA_tc - DB_tc so that the group weights are
+    // the posteriors themselves (sum ~ 1).
+    float *Bv = V;
+    for (int x = w; x < NV * NG; x += TPS) Bv[((T - 1) % NB) * NV * NG + x] = 0.0f;
+    __syncthreads();
+    float DB = 0.0f;
+    for (int t = T - 2; t >= -1; --t) {
+      const int tc = t + 1;                                  // combine step
+      const float *Bi = Bv + (tc % NB) * NV * NG;
+      float bin[G], pin[GRAD ? G : 1];
+#pragma unroll
+      for (int q = 0; q < GQ; ++q) {
+        const float4 v = *reinterpret_cast<const float4 *>(Bi + swz<C::SWZ>(G * w + 4 * q));
+        bin[4 * q] = v.x; bin[4 * q + 1] = v.y; bin[4 * q + 2] = v.z; bin[4 * q + 3] = v.w;
+        if (GRAD) {
+          const float4 f = *reinterpret_cast<const float4 *>(Bi + NG + swz<C::SWZ>(G * w + 4 * q));
+          pin[4 * q] = f.x; pin[4 * q + 1] = f.y; pin[4 * q + 2] = f.z; pin[4 * q + 3] = f.w;
+        }
+      }
+      float dprev = 0.0f;                                    // max of stored B_tc
+      if (tc < T - 1) {
+        const float *pp = prec((tc + 1) & 1);
+        dprev = pp[0];
+#pragma unroll
+        for (int x = 1; x < NPART; ++x) dprev = fmaxf(dprev, pp[x * PREC]);
+        if (w == 0 && active) {                              // finish step tc + 1
+          float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f;
+#pragma unroll
+          for (int x = 0; x < NPART; ++x) {
+            num += pp[x * PREC + 1]; den += pp[x * PREC + 2];
+            if (GRAD) { n1 += pp[x * PREC + 3]; n2 += pp[x * PREC + 4]; }
+          }
+          const float inv = 1.0f / den;
+          if (soft_out) soft_out[seq * T + tc + 1] = num * inv;
+          if (GRAD) grad_out[seq * T + tc + 1] = two_over_temp * (n2 * inv - (num * inv) * (n1 * inv));
+        }
+      }
+      if (NB == 1) __syncthreads();
+      const float K = log2Z - cah[ls * 256 + tc] - DB;
+      DB += dprev;
+      const float sv = ssm[ls * 256 + tc];
+      const float vv = GRAD ? vsm[ls * 256 + tc] : 0.0f;
+      const float fv = GRAD ? fsm[ls * 256 + tc] : 0.0f;
+      float *Bo = Bv + ((t + NB) % NB) * NV * NG;
+      float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f, tmax = -INFINITY;
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        float av[GQ], fa[GRAD ? GQ : 1];
+#pragma unroll
+        for (int q = 0; q < (GQ + 3) / 4; ++q) {
+          const int f = a * GQ + 4 * q;
+          const float4 v = spill[((size_t)tc * NCH + (f >> 2)) * TPS + w];
+          const float e4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) av[4 * q + k] = e4[(f & 3) + k];
+          if (GRAD) {
+            const int g = G + a * GQ + 4 * q;
+            const float4 u = spill[((size_t)tc * NCH + (g >> 2)) * TPS + w];
+            const float g4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) fa[(4 * q + k) < (GRAD ? GQ : 1) ? 4 * q + k : 0] = g4[(g & 3) + k];
+          }
+        }
+        float outB[GQ], outP[GQ];
+#pragma unroll
+        for (int k = 0; k < GQ; ++k) {
+          float y[4], c[4], z[4];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            c[b] = code_at<C>(creg, Csm, a, 4 * k + b, w);
+            const float d = c[b] - sv;
+            y[b] = fmaf(-kappa * d, d, bin[4 * k + b]);
+            z[b] = GRAD ? pin[GRAD ? 4 * k + b : 0] + vv * (c[b] - fv) : 0.0f;
+          }
+          const float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+          float S = 0.0f, Sc = 0.0f, Sz = 0.0f, Scz = 0.0f;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const float u = ex2(y[b] - mx);
+            S += u;
+            Sc = fmaf(u, c[b], Sc);
+            if (GRAD) { Sz = fmaf(u, z[b], Sz); Scz = fmaf(u * c[b], z[b], Scz); }
+          }
+          outB[k] = mx + lg2(S) - dprev;
+          tmax = fmaxf(tmax, outB[k]);
+          const float wgt = ex2(av[k] + mx - K);
+          den = fmaf(wgt, S, den);
+          num = fmaf(wgt, Sc, num);
+          if (GRAD) {
+            const float fk = fa[GRAD ? k : 0];
+            outP[k] = Sz * __frcp_rn(S);
+            n1 = fmaf(wgt, fmaf(fk, S, Sz), n1);
+            n2 = fmaf(wgt, fmaf(fk, Sc, Scz), n2);
+          }
+        }
+        if (t >= 0) {
+          write_run<C>(Bo, a * (NG / 4) + GQ * w, outB);
+          if (GRAD) write_run<C>(Bo + NG, a * (NG / 4) + GQ * w, outP);
+        }
+      }
+      tmax = lane_reduce<TPS>(tmax, MaxOp());
+      num = lane_reduce<TPS>(num, SumOp());
+      den = lane_reduce<TPS>(den, SumOp());
+      if (GRAD) {
+        n1 = lane_reduce<TPS>(n1, SumOp());
+        n2 = lane_reduce<TPS>(n2, SumOp());
+      }
+      if (plead) {
+        float *pp = prec(tc & 1) + pidx * PREC;
+        pp[0] = tmax; pp[1] = num; pp[2] = den; pp[3] = n1; pp[4] = n2;
+      }
+      __syncthreads();
+    }
+    if (w == 0 && active) {                                  // finish step 0
+      const float *pp = prec(0);
+      float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f;
+#pragma unroll
+      for (int x = 0; x < NPART; ++x) {
+        num += pp[x * PREC + 1]; den += pp[x * PREC + 2];
+        if (GRAD) { n1 += pp[x * PREC + 3]; n2 += pp[x * PREC + 4]; }
+      }
+      const float inv = 1.0f / den;
+      if (soft_out) soft_out[seq * T] = num * inv;
+      if (GRAD) grad_out[seq * T] = two_over_temp * (n2 * inv - (num * inv) * (n1 * inv));
+    }
+  }
+}
+
+}  // namespace tcq
+
+using namespace tcq;
+using namespace tcq_host;
+
+namespace {
+
+using Soft8 = BcjrCfg<8, 4, 8, 4, 2, false>;
+using Soft12 = BcjrCfg<12, 4, 1, 4, 2, false>;
+using Soft16 = BcjrCfg<16, 32, 1, 2, 1, false>;
+using Grad8 = BcjrCfg<8, 4, 8, 4, 2, true>;
+using Grad12 = BcjrCfg<12, 4, 1, 4, 2, true>;
+
+template <class C>
+int grid_for(int64_t n_seq) {
+  int dev = 0, per_sm = 0;
+  cudaGetDevice(&dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bcjr_kernel<C>, C::NT,
+                                                    C::smem_bytes()) != cudaSuccess ||
+      per_sm <= 0)
+    per_sm = 1;
+  const int64_t want = (n_seq + C::SPC - 1) / C::SPC;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)per_sm * sm_count()));
+}
+
+template <class C>
+bool set_smem() {
+  const size_t smem = C::smem_bytes();
+  if (smem <= 48 * 1024) return true;
+  return cudaFuncSetAttribute(bcjr_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)smem) == cudaSuccess;
+}
+
+template <class C>
+size_t ws_bytes_for(int64_t n_seq, int T) {
+  if (!set_smem<C>()) return 0;
+  const int grid = grid_for<C>(n_seq);
+  return (size_t)grid * C::SPC * C::ws_floats_per_slot(T) * sizeof(float) + 256;
+}
+
+template <class C>
+tcq_status_t launch(const float *s, int64_t n_seq, int T, float kappa, float two_over_temp,
+                    const float *v,
+                    const float *soft_in, float *soft, float *logz, float *grad, void *ws,
+                    size_t ws_bytes, cudaStream_t stream) {
+  if (!set_smem<C>()) return TCQ_ERR_CUDA;
+  const int grid = grid_for<C>(n_seq);
+  const size_t need = (size_t)grid * C::SPC * C::ws_floats_per_slot(T) * sizeof(float);
+  if (ws_bytes < need) return TCQ_ERR_WORKSPACE;
+  bcjr_kernel<C><<<grid, C::NT, C::smem_bytes(), stream>>>(s, n_seq, T, kappa, two_over_temp, v,
+                                                           soft_in, soft, logz, grad,
+                                                           static_cast<float *>(ws));
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" size_t tcq_bcjr_workspace_size(const tcq_trellis_t *tr, int64_t n_seq, int with_grad) {
+  if (check_trellis(tr) != TCQ_OK || n_seq <= 0) return 256;
+  const int T = tr->seq_len;
+  if (with_grad) {
+    switch (tr->L) {
+      case 8: return ws_bytes_for<Grad8>(n_seq, T);
+      case 12: return ws_bytes_for<Grad12>(n_seq, T);
+      default: return 0;
+    }
+  }
+  switch (tr->L) {
+    case 8: return ws_bytes_for<Soft8>(n_seq, T);
+    case 12: return ws_bytes_for<Soft12>(n_seq, T);
+    default: return ws_bytes_for<Soft16>(n_seq, T);
+  }
+}
+
+static bool temp_ok(float temp) { return temp > 0.0f && temp < INFINITY; }
+
+extern "C" tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *tr, const float *s, int64_t n_seq,
+                                      float temp, float *soft, float *log_z, void *ws,
+                                      size_t ws_bytes, void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if (!temp_ok(temp)) return TCQ_ERR_INVALID_ARG;
+  if (n_seq < 0 || n_seq > (int64_t)INT32_MAX) return TCQ_ERR_INVALID_ARG;
+  if (n_seq == 0) return TCQ_OK;
+  if (!s || !soft || !aligned16(s) || !aligned16(soft) || (log_z && !aligned16(log_z)))
+    return TCQ_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
+  const float kappa = (float)(1.4426950408889634 / (double)temp);
+  const float tot = (float)(2.0 / (double)temp);
+  cudaStream_t strm = (cudaStream_t)stream;
+  const int T = tr->seq_len;
+  switch (tr->L) {
+    case 8: return launch<Soft8>(s, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
+    case 12: return launch<Soft12>(s, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
+    default: return launch<Soft16>(s, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
+  }
+}
+
+extern "C" tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *tr, const float *s,
+                                               int64_t n_seq, float temp, const float *soft,
+                                               const float *grad_soft, float *grad_s, void *ws,
+                                               size_t ws_bytes, void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if (tr->L == 16) return TCQ_ERR_UNSUPPORTED;
+  if (!temp_ok(temp)) return TCQ_ERR_INVALID_ARG;
+  if (n_seq < 0 || n_seq > (int64_t)INT32_MAX) return TCQ_ERR_INVALID_ARG;
+  if (n_seq == 0) return TCQ_OK;
+  if (!s || !soft || !grad_soft || !grad_s || !aligned16(s) || !aligned16(soft) ||
+      !aligned16(grad_soft) || !aligned16(grad_s))
+    return TCQ_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
+  const float kappa = (float)(1.4426950408889634 / (double)temp);
+  const float tot = (float)(2.0 / (double)temp);
+  cudaStream_t strm = (cudaStream_t)stream;
+  const int T = tr->seq_len;
+  switch (tr->L) {
+    case 8: return launch<Grad8>(s, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
+    default: return launch<Grad12>(s, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
+  }
+}

@@ -1,0 +1,220 @@
+// Sliding-window decode and state packing.
+//
+// [QTIP blog, "The trellis: a stateful codebook"] the state of weight t is the
+// L-bit window of the bitstream starting at bit k*t (most significant first),
+// so every weight decodes on its own: a funnel shift, the 1MAD hash and a
+// conversion to fp16.  [QTIP blog, "Tail-biting is worth its complexity"] a
+// tail-biting stream is exactly k*T bits and its windows wrap around.
+// [QTIP blog, "What it buys end to end"] each 16x16 tile of a weight matrix is
+// one 256-weight sequence.
+//
+// The decode is bound by HBM traffic (2 bits in, 16 bits out per weight): the
+// tile kernel keeps a sequence's 64-byte stream in registers and writes each
+// tile row with one 16-byte store per thread, a warp covering 512 contiguous
+// bytes of the output matrix.
+#include <algorithm>
+
+#include "tcq_device.cuh"
+
+namespace tcq {
+
+// Window of L bits starting at bit offset o (0..31) of the 64-bit word pair
+// (hi:lo), most significant bit first.
+template <int L>
+__device__ __forceinline__ uint32_t window_at(uint32_t hi, uint32_t lo, uint32_t o) {
+  return __funnelshift_l(lo, hi, o) >> (32 - L);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// TILE16 decode of 256-weight sequences (k = 2, so a sequence's stream is 16
+// words tail-biting, 16 + ceil((L-2)/32) words free-start).  One thread owns
+// one half (8 columns) of one tile and walks its 16 rows.
+template <int L, int LAYOUT>
+__global__ void __launch_bounds__(256) decode_tile16_kernel(const uint32_t *__restrict__ bits,
+                                                            int n_tiles_c, int64_t n_items,
+                                                            int words_per_seq, int cols,
+                                                            uint16_t *__restrict__ out) {
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_items;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t tr = g / (2 * n_tiles_c);
+    const int rem = (int)(g - tr * 2 * n_tiles_c);
+    const int tc = rem >> 1, h = rem & 1;
+    const int64_t seq = tr * n_tiles_c + tc;
+    const uint32_t *src = bits + seq * words_per_seq;
+    uint32_t w[17];
+    if (LAYOUT == TCQ_TAILBITING) {
+      const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 v = __ldg(s4 + q);
+        w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+      }
+      w[16] = w[0];
+    } else {
+#pragma unroll
+      for (int q = 0; q < 16; ++q) w[q] = __ldg(src + q);
+      w[16] = __ldg(src + 16);
+    }
+    uint16_t *dst = out + (tr * 16) * (int64_t)cols + tc * 16 + h * 8;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      // weights t = 16 r + 8 h + j, stream bit 2t = 32 r + 16 h + 2 j
+      float c[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        c[j] = one_mad_decode_f32(window_at<L>(w[r], w[r + 1], 16 * h + 2 * j));
+      uint4 o;
+      o.x = pack_half2(c[0], c[1]);
+      o.y = pack_half2(c[2], c[3]);
+      o.z = pack_half2(c[4], c[5]);
+      o.w = pack_half2(c[6], c[7]);
+      *reinterpret_cast<uint4 *>(dst + (int64_t)r * cols) = o;
+    }
+  }
+}
+
+// Generic decode, one thread per weight, output in sequence order.
+template <int L>
+__global__ void __launch_bounds__(256) decode_seq_kernel(const uint32_t *__restrict__ bits,
+                                                         int64_t n_weights, int T, int layout,
+                                                         int words_per_seq, int nbits,
+                                                         uint16_t *__restrict__ out) {
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_weights;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t seq = g / T;
+    const int t = (int)(g - seq * T);
+    const uint32_t *src = bits + seq * words_per_seq;
+    const int p = 2 * t;              // k = 2
+    const int i = p >> 5, o = p & 31;
+    const uint32_t hi = __ldg(src + i);
+    int i1 = i + 1;
+    uint32_t lo = 0;
+    if (layout == TCQ_TAILBITING) {
+      if (i1 == words_per_seq) i1 = 0;
+      lo = __ldg(src + i1);
+    } else if (i1 < words_per_seq) {
+      lo = __ldg(src + i1);
+    }
+    (void)nbits;
+    const float c = one_mad_decode_f32(window_at<L>(hi, lo, (uint32_t)o));
+    out[g] = __half_as_ushort(__float2half_rn(c));
+  }
+}
+
+// Pack walks into streams: one thread per output word.
+__global__ void __launch_bounds__(256) pack_states_kernel(const uint16_t *__restrict__ states,
+                                                          int64_t n_words_total, int T, int L,
+                                                          int layout, int words_per_seq,
+                                                          uint32_t *__restrict__ bits) {
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_words_total;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t seq = g / words_per_seq;
+    const int wi = (int)(g - seq * words_per_seq);
+    const uint16_t *st = states + seq * T;
+    const int kT = 2 * T;
+    const int nbits = layout == TCQ_TAILBITING ? kT : kT + L - 2;
+    uint32_t word = 0;
+    for (int b = 0; b < 32; ++b) {
+      const int p = 32 * wi + b;
+      uint32_t bit = 0;
+      if (p < kT) {
+        const int t = p >> 1, i = p & 1;          // top bits of state t
+        bit = (st[t] >> (L - 1 - i)) & 1u;
+      } else if (p < nbits) {
+        const int i = p - 2 * (T - 1);            // tail of the last state
+        bit = (st[T - 1] >> (L - 1 - i)) & 1u;
+      }
+      word |= bit << (31 - b);
+    }
+    bits[g] = word;
+  }
+}
+
+}  // namespace tcq
+
+using namespace tcq;
+using namespace tcq_host;
+
+extern "C" size_t tcq_stream_words(const tcq_trellis_t *tr, int layout) {
+  if (check_trellis(tr) != TCQ_OK) return 0;
+  const int64_t kT = (int64_t)tr->k * tr->seq_len;
+  if (layout == TCQ_TAILBITING) {
+    if (kT % 32 != 0 || kT < tr->L) return 0;
+    return (size_t)(kT / 32);
+  }
+  if (layout == TCQ_FREE_START) return (size_t)((kT + tr->L - tr->k + 31) / 32);
+  return 0;
+}
+
+extern "C" tcq_status_t tcq_pack_states(const tcq_trellis_t *tr, const uint16_t *states,
+                                        int64_t n_seq, int layout, uint32_t *bits,
+                                        void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if (layout != TCQ_TAILBITING && layout != TCQ_FREE_START) return TCQ_ERR_INVALID_ARG;
+  if (n_seq < 0) return TCQ_ERR_INVALID_ARG;
+  const size_t wps = tcq_stream_words(tr, layout);
+  if (wps == 0) return TCQ_ERR_UNSUPPORTED;
+  if (n_seq == 0) return TCQ_OK;
+  if (!states || !bits || !aligned16(states) || !aligned16(bits)) return TCQ_ERR_INVALID_ARG;
+  const int64_t total = n_seq * (int64_t)wps;
+  const int64_t blocks = std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 16);
+  pack_states_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
+      states, total, tr->seq_len, tr->L, layout, (int)wps, bits);
+  return launch_status();
+}
+
+template <int L>
+static tcq_status_t decode_launch(const tcq_trellis_t *tr, const uint32_t *bits, int64_t n_seq,
+                                  int layout, int out_layout, int64_t rows, int64_t cols,
+                                  uint16_t *out, cudaStream_t stream, int wps) {
+  if (out_layout == TCQ_OUT_TILE16) {
+    const int64_t ntc = cols / 16;
+    const int64_t items = n_seq * 2;
+    const int64_t blocks = std::min<int64_t>((items + 255) / 256, (int64_t)sm_count() * 8);
+    if (layout == TCQ_TAILBITING)
+      decode_tile16_kernel<L, TCQ_TAILBITING><<<(unsigned)blocks, 256, 0, stream>>>(
+          bits, (int)ntc, items, wps, (int)cols, out);
+    else
+      decode_tile16_kernel<L, TCQ_FREE_START><<<(unsigned)blocks, 256, 0, stream>>>(
+          bits, (int)ntc, items, wps, (int)cols, out);
+  } else {
+    const int64_t nw = n_seq * tr->seq_len;
+    const int64_t blocks = std::min<int64_t>((nw + 255) / 256, (int64_t)sm_count() * 16);
+    decode_seq_kernel<L><<<(unsigned)blocks, 256, 0, stream>>>(
+        bits, nw, tr->seq_len, layout, wps, 0, out);
+  }
+  (void)rows;
+  return launch_status();
+}
+
+extern "C" tcq_status_t tcq_decode(const tcq_trellis_t *tr, const uint32_t *bits, int64_t n_seq,
+                                   int layout, int out_layout, int64_t rows, int64_t cols,
+                                   uint16_t *out, void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if (layout != TCQ_TAILBITING && layout != TCQ_FREE_START) return TCQ_ERR_INVALID_ARG;
+  if (out_layout != TCQ_OUT_SEQ && out_layout != TCQ_OUT_TILE16) return TCQ_ERR_INVALID_ARG;
+  if (n_seq < 0) return TCQ_ERR_INVALID_ARG;
+  const size_t wps = tcq_stream_words(tr, layout);
+  if (wps == 0) return TCQ_ERR_UNSUPPORTED;
+  if (out_layout == TCQ_OUT_TILE16) {
+    if (tr->seq_len != 256) return TCQ_ERR_UNSUPPORTED;
+    if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return TCQ_ERR_INVALID_ARG;
+    if ((rows / 16) * (cols / 16) != n_seq) return TCQ_ERR_INVALID_ARG;
+    if (cols > (int64_t)INT32_MAX / 2 || rows / 16 > (int64_t)INT32_MAX) return TCQ_ERR_UNSUPPORTED;
+  }
+  if (n_seq == 0) return TCQ_OK;
+  if (!bits || !out || !aligned16(bits) || !aligned16(out)) return TCQ_ERR_INVALID_ARG;
+  if (out_layout == TCQ_OUT_TILE16 && layout == TCQ_FREE_START && wps > 17) return TCQ_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (tr->L) {
+    case 8: return decode_launch<8>(tr, bits, n_seq, layout, out_layout, rows, cols, out, s, (int)wps);
+    case 12: return decode_launch<12>(tr, bits, n_seq, layout, out_layout, rows, cols, out, s, (int)wps);
+    default: return decode_launch<16>(tr, bits, n_seq, layout, out_layout, rows, cols, out, s, (int)wps);
+  }
+}

@@ -1,0 +1,95 @@
+// Device-side building blocks shared by the trellis kernels (sm_100a).
+//
+//   * the 1MAD computed code [QTIP blog, "The codebook is computed"]: a 32-bit
+//     LCG step, the byte sum of its output (one VABSDIFF4 against zero), the
+//     centring by 510 and the scale 1/147.8;
+//   * base-2 exponent/logarithm on the MUFU unit (PTX ex2/lg2.approx);
+//   * the shared-memory swizzle used by every state-vector exchange;
+//   * small launch/validation helpers for the C ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "tcq.h"
+
+namespace tcq {
+
+constexpr uint32_t kLcgMul = 34038481u;
+constexpr uint32_t kLcgAdd = 76625530u;
+
+// Byte sum of the LCG output for state x (Irwin-Hall with n = 4).
+__device__ __forceinline__ uint32_t one_mad_bytesum(uint32_t x) {
+  return __vsadu4(x * kLcgMul + kLcgAdd, 0u);
+}
+
+// fp32 code value: the fp64 value (bytesum - 510) / 147.8 rounded once to
+// fp32.  Used once per state at kernel start, so the exact fp64 division is
+// affordable and the table is identical to the definition.
+__device__ __forceinline__ float one_mad_f32(uint32_t x) {
+  const double v = (double)((int)one_mad_bytesum(x) - 510) / 147.8;
+  return __double2float_rn(v);
+}
+
+// fp32 value on the streaming decode path: (bytesum - 510) * RN(1/147.8).
+// bytesum - 510 is formed exactly with the 2^23 magic-number trick; after the
+// final round-to-nearest-even to fp16 this equals the fp16 rounding of the
+// fp64 definition for all 1,021 byte sums (checked exhaustively by the tests).
+__device__ __forceinline__ float one_mad_decode_f32(uint32_t x) {
+  const uint32_t bs = one_mad_bytesum(x);
+  const float centred = __fsub_rn(__uint_as_float(0x4B000000u | bs), 8389118.0f);
+  return __fmul_rn(centred, 0x1.bb68f6p-8f);  // RN32(1/147.8)
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Shared-memory swizzle of a state-vector index (float granularity).  Works on
+// 16-byte units: unit u goes to u ^ ((u >> 3) & MASK).  It is a bijection, so
+// any consistent use is correct; MASK = G/4 - 1 makes both the strided vector
+// reads and the contiguous vector writes of a trellis step bank-conflict free.
+template <int MASK>
+__device__ __forceinline__ int swz(int idx) {
+  const int u = idx >> 2;
+  return (((u ^ ((u >> 3) & MASK))) << 2) | (idx & 3);
+}
+
+}  // namespace tcq
+
+// Host-side helpers used by the C ABI translation units.
+namespace tcq_host {
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline tcq_status_t check_trellis(const tcq_trellis_t *tr) {
+  if (!tr) return TCQ_ERR_INVALID_ARG;
+  if (tr->L <= 0 || tr->k <= 0 || tr->V <= 0 || tr->seq_len <= 0) return TCQ_ERR_INVALID_ARG;
+  if (tr->k != 2 || tr->V != 1) return TCQ_ERR_UNSUPPORTED;
+  if (tr->L != 8 && tr->L != 12 && tr->L != 16) return TCQ_ERR_UNSUPPORTED;
+  if (tr->seq_len > 256) return TCQ_ERR_UNSUPPORTED;
+  return TCQ_OK;
+}
+
+inline tcq_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
+inline int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+}  // namespace tcq_host

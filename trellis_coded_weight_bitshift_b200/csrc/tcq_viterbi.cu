@@ -1,0 +1,317 @@
+// Viterbi (min-plus) encode on the bitshift trellis, fp32, state-parallel.
+//
+// [QTIP blog, "The trellis: a stateful codebook"] Viterbi keeps, per step,
+// the cheapest walk into each of the 2^L states; the predecessors of state j
+// are computed with shifts, pred_a(j) = (j >> k) | (a << (L-k)):
+//   cost_0(j) = (code_j - s_0)^2
+//   cost_t(j) = min_a cost_{t-1}(pred_a j) + (code_j - s_t)^2
+// and the walk is read back from the final argmin with stored backpointers.
+//
+// Layout used here (k = 2).  The four states j = 4q + b (b = 0..3) share the
+// same predecessor set {q | a << (L-2)}, so the minimum over a, and its
+// argmin, is taken once per group q: the kernel carries
+//   M_t(q) = min_a cost_{t-1}(q | a << (L-2)),   M_0 = 0,
+// (2^(L-2) values, a quarter of the cost vector) and recomputes
+//   cost_t(p) = M_t(p >> 2) + (code_p - s_t)^2
+// on the fly.  Every fp32 operation is the same correctly rounded operation
+// as in the definition (sub, mul, add; no FMA contraction), so costs, paths
+// and the MSE are bit-identical to a plain fp32 evaluation, and the
+// backpointer needs 2 bits per GROUP per step, not per state.
+//
+// Work split: a sequence's 2^(L-2) groups are spread over TPS threads, G
+// consecutive groups per thread.  The thread's 4G predecessor states
+// p = a*2^(L-2) + G*w + i never change, so their code values are computed
+// once (1MAD in registers; for L = 16, half of them in shared memory because
+// 2^16 fp32 values are the whole register file) and the state vector M lives
+// in shared memory.  Step t reads M_{t-1} at a*2^(L-4) + (G/4)*w + (0..G/4-1)
+// (four short runs), writes M_t at G*w + (0..G-1) (one run) and stores the
+// thread's 2G backpointer bits with one coalesced store.
+#include <algorithm>
+
+#include "tcq_device.cuh"
+
+namespace tcq {
+
+template <int L_, int G_, int SPC_, int AREG_, int NBUF_>
+struct VitCfg {
+  static constexpr int L = L_, G = G_, SPC = SPC_, AREG = AREG_, NBUF = NBUF_;
+  static constexpr int NG = 1 << (L - 2);      // groups (states / 4)
+  static constexpr int TPS = NG / G;           // threads per sequence
+  static constexpr int NT = TPS * SPC;         // threads per CTA
+  static constexpr int GQ = G / 4;             // M values read per predecessor digit
+  static constexpr int ASM = 4 - AREG;         // predecessor digits whose codes sit in smem
+  static constexpr int BPB = G / 4;            // backpointer bytes per thread per step
+  static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
+  static constexpr size_t smem_bytes() {
+    return sizeof(float) * ((size_t)SPC * NBUF * NG + (size_t)ASM * G * TPS + (size_t)SPC * 256) +
+           sizeof(unsigned long long) * NT;
+  }
+  static_assert(NG % G == 0 && G % 4 == 0, "bad group split");
+};
+
+template <int N>
+__device__ __forceinline__ void load_run(const float *base, int idx, float *dst) {
+  // N contiguous floats starting at idx (N in {1,2,4,8}; idx aligned to min(N,4))
+  if constexpr (N == 1) {
+    dst[0] = base[idx];
+  } else if constexpr (N == 2) {
+    const float2 v = *reinterpret_cast<const float2 *>(base + idx);
+    dst[0] = v.x; dst[1] = v.y;
+  } else {
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q) {
+      const float4 v = *reinterpret_cast<const float4 *>(base + idx + 4 * q);
+      dst[4 * q] = v.x; dst[4 * q + 1] = v.y; dst[4 * q + 2] = v.z; dst[4 * q + 3] = v.w;
+    }
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::NT, 1)
+viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
+                   uint8_t *__restrict__ bp, uint16_t *__restrict__ states,
+                   float *__restrict__ mse) {
+  constexpr int NG = C::NG, G = C::G, GQ = C::GQ, TPS = C::TPS, AREG = C::AREG, ASM = C::ASM;
+  constexpr int NB = C::NBUF;
+  extern __shared__ __align__(16) float smem[];
+  float *Mall = smem;                                              // [SPC][NB][NG]
+  float *Csm = Mall + C::SPC * NB * NG;                            // [ASM][G/4][TPS] float4
+  float *ssm = Csm + ASM * G * TPS;                                // [SPC][256]
+  unsigned long long *red = reinterpret_cast<unsigned long long *>(ssm + C::SPC * 256);
+
+  const int tid = threadIdx.x;
+  const int ls = tid / TPS, w = tid - ls * TPS;
+  const int64_t seq = (int64_t)blockIdx.x * C::SPC + ls;
+  const bool active = seq < n_seq;
+
+  // Code values of this thread's predecessor states p = a*NG + G*w + i.
+  float creg[AREG > 0 ? AREG : 1][G];
+#pragma unroll
+  for (int a = 0; a < AREG; ++a)
+#pragma unroll
+    for (int i = 0; i < G; ++i) creg[a][i] = one_mad_f32((uint32_t)(a * NG + G * w + i));
+  if (ls == 0) {
+#pragma unroll
+    for (int a = 0; a < ASM; ++a)
+#pragma unroll
+      for (int q = 0; q < GQ; ++q) {
+        const uint32_t p = (uint32_t)((a + AREG) * NG + G * w + 4 * q);
+        float4 v = make_float4(one_mad_f32(p), one_mad_f32(p + 1), one_mad_f32(p + 2),
+                               one_mad_f32(p + 3));
+        reinterpret_cast<float4 *>(Csm)[(a * GQ + q) * TPS + w] = v;
+      }
+  }
+  for (int x = tid; x < C::SPC * T; x += C::NT) {
+    const int l = x / T, t = x - l * T;
+    const int64_t sq = (int64_t)blockIdx.x * C::SPC + l;
+    ssm[l * 256 + t] = sq < n_seq ? s[sq * T + t] : 0.0f;
+  }
+  float *M = Mall + ls * NB * NG;
+  for (int x = w; x < NG; x += TPS) M[x] = 0.0f;                 // M_0 = 0
+  __syncthreads();
+
+  uint8_t *bps = bp + (active ? seq : 0) * (int64_t)(T - 1) * (NG / 4);
+  float min_in[4][GQ];
+
+  for (int t = 1; t <= T; ++t) {
+    // t < T: step computing M_t from M_{t-1}; t == T: final argmin over cost_{T-1}
+    const float *Mi = M + ((t - 1) % NB) * NG;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int base = a * (NG / 4) + GQ * w;
+      if constexpr (GQ <= 4) {
+        float tmp[GQ];
+        load_run<GQ>(Mi, swz<C::SWZ>(base), tmp);
+#pragma unroll
+        for (int k = 0; k < GQ; ++k) min_in[a][k] = tmp[k];
+      } else {
+#pragma unroll
+        for (int q = 0; q < GQ / 4; ++q) {
+          float tmp[4];
+          load_run<4>(Mi, swz<C::SWZ>(base + 4 * q), tmp);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) min_in[a][4 * q + k] = tmp[k];
+        }
+      }
+    }
+    const float sv = ssm[ls * 256 + t - 1];
+    if (t == T) break;
+    if (NB == 1) __syncthreads();                                 // all reads of M_{t-1} done
+    float *Mo = M + (t % NB) * NG;
+    uint32_t bits[(2 * G + 31) / 32];
+#pragma unroll
+    for (int b = 0; b < (2 * G + 31) / 32; ++b) bits[b] = 0;
+#pragma unroll
+    for (int q = 0; q < GQ; ++q) {
+      float4 csm[ASM > 0 ? ASM : 1];
+#pragma unroll
+      for (int a = 0; a < ASM; ++a) csm[a] = reinterpret_cast<const float4 *>(Csm)[(a * GQ + q) * TPS + w];
+      float outv[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = 4 * q + r;
+        float cst[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          float c;
+          if (a < AREG) c = creg[a < AREG ? a : 0][i];
+          else {
+            const float4 v = csm[a >= AREG ? a - AREG : 0];
+            c = r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
+          }
+          const float d = __fsub_rn(c, sv);
+          cst[a] = __fadd_rn(min_in[a][q], __fmul_rn(d, d));
+        }
+        // first minimum (lowest a) of the four candidates
+        const bool p1 = cst[1] < cst[0];
+        const float m01 = p1 ? cst[1] : cst[0];
+        const bool p2 = cst[3] < cst[2];
+        const float m23 = p2 ? cst[3] : cst[2];
+        const bool p3 = m23 < m01;
+        outv[r] = p3 ? m23 : m01;
+        const uint32_t idx = p3 ? (2u | (uint32_t)p2) : (uint32_t)p1;
+        bits[i >> 4] |= idx << (2 * (i & 15));
+      }
+      *reinterpret_cast<float4 *>(Mo + swz<C::SWZ>(G * w + 4 * q)) =
+          make_float4(outv[0], outv[1], outv[2], outv[3]);
+    }
+    if (active) {
+      uint8_t *dst = bps + (int64_t)(t - 1) * (NG / 4) + w * C::BPB;
+      if constexpr (C::BPB == 1) *dst = (uint8_t)bits[0];
+      else if constexpr (C::BPB == 2) *reinterpret_cast<uint16_t *>(dst) = (uint16_t)bits[0];
+      else if constexpr (C::BPB == 4) *reinterpret_cast<uint32_t *>(dst) = bits[0];
+      else *reinterpret_cast<uint2 *>(dst) = make_uint2(bits[0], bits[1]);
+    }
+    __syncthreads();
+  }
+
+  // Final decision: cost_{T-1}(p) = M_{T-1}(p >> 2) + e_{T-1}(p); lowest p wins ties.
+  {
+    const float sv = ssm[ls * 256 + T - 1];
+    unsigned long long best = ~0ull;
+#pragma unroll
+    for (int q = 0; q < GQ; ++q) {
+      float4 csm[ASM > 0 ? ASM : 1];
+#pragma unroll
+      for (int a = 0; a < ASM; ++a) csm[a] = reinterpret_cast<const float4 *>(Csm)[(a * GQ + q) * TPS + w];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = 4 * q + r;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          float c;
+          if (a < AREG) c = creg[a < AREG ? a : 0][i];
+          else {
+            const float4 v = csm[a >= AREG ? a - AREG : 0];
+            c = r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
+          }
+          const float d = __fsub_rn(c, sv);
+          const float cost = __fadd_rn(min_in[a][q], __fmul_rn(d, d));
+          const unsigned long long key =
+              ((unsigned long long)__float_as_uint(cost) << 32) | (uint32_t)(a * NG + G * w + i);
+          best = key < best ? key : best;
+        }
+      }
+    }
+    // reduce over the sequence's TPS threads
+    constexpr int WL = TPS < 32 ? TPS : 32;
+#pragma unroll
+    for (int off = WL / 2; off > 0; off >>= 1) {
+      const unsigned long long o = __shfl_xor_sync(0xffffffffu, best, off);
+      best = o < best ? o : best;
+    }
+    red[tid] = best;
+    __syncthreads();
+    if (w == 0 && active) {
+      for (int x = WL; x < TPS; x += WL) {
+        const unsigned long long o = red[tid + x];
+        best = o < best ? o : best;
+      }
+      const float cost = __uint_as_float((uint32_t)(best >> 32));
+      states[seq * T + T - 1] = (uint16_t)(best & 0xffffffffu);
+      mse[seq] = __fdiv_rn(cost, (float)T);
+    }
+  }
+}
+
+// Traceback: one thread per sequence, st[t-1] = (st[t] >> 2) | (bp_t(st[t] >> 2) << (L-2)).
+template <int L>
+__global__ void __launch_bounds__(128) viterbi_traceback_kernel(const uint8_t *__restrict__ bp,
+                                                                int64_t n_seq, int T,
+                                                                uint16_t *__restrict__ states) {
+  constexpr int NG = 1 << (L - 2);
+  const int64_t seq = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (seq >= n_seq) return;
+  const uint8_t *b = bp + seq * (int64_t)(T - 1) * (NG / 4);
+  uint16_t *st = states + seq * T;
+  uint32_t cur = st[T - 1];
+  for (int t = T - 1; t > 0; --t) {
+    const uint32_t q = cur >> 2;
+    const uint32_t a = (__ldg(b + (int64_t)(t - 1) * (NG / 4) + (q >> 2)) >> (2 * (q & 3))) & 3u;
+    cur = q | (a << (L - 2));
+    st[t - 1] = (uint16_t)cur;
+  }
+}
+
+}  // namespace tcq
+
+using namespace tcq;
+using namespace tcq_host;
+
+namespace {
+
+using Vit8 = VitCfg<8, 4, 8, 4, 2>;      // 16 threads / sequence, 8 sequences / CTA
+using Vit12 = VitCfg<12, 4, 1, 4, 2>;    // 256 threads / sequence
+using Vit16 = VitCfg<16, 32, 1, 2, 1>;   // 512 threads / sequence, half the codes in smem
+
+size_t bp_bytes_per_seq(int L, int T) { return (size_t)(T - 1) * ((size_t)1 << (L - 4)); }
+
+template <class C>
+tcq_status_t launch_fwd(const float *s, int64_t n_seq, int T, uint8_t *bp, uint16_t *states,
+                        float *mse, cudaStream_t stream) {
+  const size_t smem = C::smem_bytes();
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(viterbi_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return TCQ_ERR_CUDA;
+  }
+  const int64_t blocks = (n_seq + C::SPC - 1) / C::SPC;
+  viterbi_fwd_kernel<C><<<(unsigned)blocks, C::NT, smem, stream>>>(s, n_seq, T, bp, states, mse);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" size_t tcq_viterbi_workspace_size(const tcq_trellis_t *tr, int64_t n_seq) {
+  if (check_trellis(tr) != TCQ_OK || n_seq < 0) return 0;
+  return ((bp_bytes_per_seq(tr->L, tr->seq_len) * (size_t)n_seq + 255) / 256) * 256 + 256;
+}
+
+extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float *s, int64_t n_seq,
+                                           uint16_t *states, float *mse, void *ws,
+                                           size_t ws_bytes, void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if (n_seq < 0 || n_seq > (int64_t)INT32_MAX * 8) return TCQ_ERR_INVALID_ARG;
+  if (n_seq == 0) return TCQ_OK;
+  if (!s || !states || !mse || !aligned16(s) || !aligned16(states) || !aligned16(mse))
+    return TCQ_ERR_INVALID_ARG;
+  const size_t need = tcq_viterbi_workspace_size(tr, n_seq);
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
+  const int T = tr->seq_len;
+  uint8_t *bp = static_cast<uint8_t *>(ws);
+  cudaStream_t strm = (cudaStream_t)stream;
+  switch (tr->L) {
+    case 8: st = launch_fwd<Vit8>(s, n_seq, T, bp, states, mse, strm); break;
+    case 12: st = launch_fwd<Vit12>(s, n_seq, T, bp, states, mse, strm); break;
+    default: st = launch_fwd<Vit16>(s, n_seq, T, bp, states, mse, strm); break;
+  }
+  if (st != TCQ_OK || T == 1) return st;
+  const unsigned tb_blocks = (unsigned)((n_seq + 127) / 128);
+  switch (tr->L) {
+    case 8: viterbi_traceback_kernel<8><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
+    case 12: viterbi_traceback_kernel<12><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
+    default: viterbi_traceback_kernel<16><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
+  }
+  return launch_status();
+}

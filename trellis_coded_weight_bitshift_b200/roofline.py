@@ -1,0 +1,80 @@
+"""Roofline bookkeeping for the benchmark: algorithmic work per kernel and the
+peak it is measured against.
+
+Units of work (per sequence of T = 256 weights on a 2^L-state trellis):
+
+  decode (HBM):  64 B of 2-bit stream read + 512 B of fp16 written, i.e.
+                 2.25 bytes per weight.  Peak: the measured HBM copy bandwidth.
+  viterbi (ALU): per state and step, the emission (code - s)^2 (sub, mul), the
+                 accumulate (add), and a quarter of the shared 4-way min and
+                 argmin of its predecessor group (3 min + 3 compare per group):
+                 4.5 lane operations per state-step, T * 2^L state-steps.
+                 Peak: 128 lane-instructions per clock per SM (4 schedulers x
+                 32 lanes, also the fp32 FMA rate) x SMs x max SM clock.
+  bcjr  (MUFU):  per group of 4 states and step, the forward log-sum-exp over
+                 4 predecessors (4 ex2 + 1 lg2) and the backward one over 4
+                 successors (4 ex2 + 1 lg2) plus the group's posterior weight
+                 (1 ex2): 11 / 4 special-function ops per state-step; the
+                 gradient pass adds a reciprocal in each direction (13 / 4).
+                 Peak: 16 special-function results per clock per SM x SMs x
+                 max SM clock.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+SEQ_LEN = 256
+B200_SMS = 148
+ISSUE_LANES_PER_SM = 128       # 4 schedulers x 32 lanes per clock
+MUFU_PER_SM = 16               # special-function results per clock per SM
+
+
+def load_measured_peaks(root: str) -> dict:
+    path = os.path.join(root, "MEASURED_PEAKS.json")
+    out = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        out.update({"hbm_gbs": float(d.get("hbm_gbs", out["hbm_gbs"])),
+                    "sm_max_mhz": float(d.get("sm_max_mhz", out["sm_max_mhz"])),
+                    "source": "measured"})
+    return out
+
+
+def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str, float, str]:
+    """(bound, algorithmic work per launch, unit of work) for a benchmark kernel."""
+    states = float(1 << L)
+    if kernel.startswith("decode"):
+        return "hbm", n_seq * (T * 2 / 8 + T * 2), "bytes"
+    if kernel.startswith("viterbi"):
+        return "alu", n_seq * T * states * 4.5, "lane-ops"
+    if kernel.startswith("bcjr_vjp"):
+        return "alu", n_seq * T * states * 13 / 4, "mufu-ops"
+    if kernel.startswith("bcjr"):
+        return "alu", n_seq * T * states * 11 / 4, "mufu-ops"
+    raise KeyError(kernel)
+
+
+def roofline_entry(kernel: str, workload, ms: float, peaks: dict, traffic=None) -> dict:
+    bound, work, unit = kernel_work(kernel, workload.L, workload.n_seq)
+    sec = ms * 1e-3
+    clk = peaks["sm_max_mhz"] * 1e6
+    if bound == "hbm":
+        achieved = work / sec / 1e9
+        peak = peaks["hbm_gbs"]
+        u = "GB/s"
+        src = f"{peaks['source']} HBM copy bandwidth"
+    elif unit == "lane-ops":
+        achieved = work / sec / 1e9
+        peak = ISSUE_LANES_PER_SM * B200_SMS * clk / 1e9
+        u = "Glane-op/s"
+        src = f"derived: {ISSUE_LANES_PER_SM} lanes/clk/SM x {B200_SMS} SMs x {peaks['sm_max_mhz']:.0f} MHz"
+    else:
+        achieved = work / sec / 1e9
+        peak = MUFU_PER_SM * B200_SMS * clk / 1e9
+        u = "Gmufu-op/s"
+        src = f"derived: {MUFU_PER_SM} MUFU/clk/SM x {B200_SMS} SMs x {peaks['sm_max_mhz']:.0f} MHz"
+    return {"kernel": kernel, "bound": bound, "achieved": achieved, "peak": peak, "unit": u,
+            "frac": achieved / peak, "traffic": traffic, "peak_source": src,
+            "work_per_launch": work, "work_unit": unit, "launch_ms": ms}
