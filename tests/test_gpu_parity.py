@@ -231,13 +231,16 @@ def test_bcjr_edge_shapes(tcq, L, T, n):
 
 
 def test_bcjr_low_temperature_matches_viterbi_codeword(tcq):
-    s = W.sequences("l8_gauss64")[:16]
+    # temp -> 0 recovers the hard code: on sequences whose closest Viterbi
+    # decision is at least 1e-3 relative apart, temp 1e-4 leaves the runner-up
+    # walks a weight below 2^-50
+    s = W.gaussian(16, 47, seq_len=64)
     soft, _ = _bcjr_gpu(tcq, s, 8, 1e-4)
     st, _, margin = oracle.viterbi_f64(s, 8)
     hard = oracle.codebook_f64(8)[st.astype(np.int64)]
-    ok = margin > 1e-2
-    assert ok.sum() >= 4
-    assert np.abs(soft[ok] - hard[ok]).max() <= 1e-4
+    ok = margin > 1e-3
+    assert ok.sum() >= 2
+    assert np.abs(soft[ok] - hard[ok]).max() <= SOFT_ATOL
 
 
 # ---------------------------------------------------------------- VJP
