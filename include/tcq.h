@@ -122,6 +122,33 @@ TCQ_API tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *trellis, const floa
                                 void *stream);
 
 /* ------------------------------------------------------------------------
+ * Allocation-free Viterbi encode (the pages have no counterpart: this is a
+ * deployment convenience of this library).
+ *
+ * For callers that may not allocate device memory at call time -- a plugin
+ * whose host owns all device memory and passes it only inputs and outputs, or
+ * a deployment whose memory budget is fixed at start-up and that forbids
+ * cudaMalloc afterwards.  Same computation and outputs as
+ * tcq_viterbi_encode, but the backpointers live in a 32 MiB buffer that is
+ * part of the library image on every GPU that loads it (held until the
+ * process exits) instead of a caller workspace; nothing is allocated or freed.
+ *
+ *   Limit: n_seq * (seq_len - 1) * 2^(L-4) bytes <= 32 MiB (for seq_len 256:
+ *   8,224 sequences at L = 8, 514 at L = 12, 32 at L = 16); larger requests
+ *   return TCQ_ERR_WORKSPACE without launching.
+ *   The first call on each device looks up the buffer's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ *   All calls share the one buffer per device: calls whose work overlaps on
+ *   the GPU (different streams without ordering) race and give wrong walks.
+ *   The buffer keeps the last call's contents; every byte a call reads is
+ *   written earlier by the same call, so nothing is cleared.
+ * ------------------------------------------------------------------------ */
+TCQ_API tcq_status_t tcq_viterbi_encode_noalloc(const tcq_trellis_t *trellis, const float *s,
+                                                int64_t n_seq, uint16_t *states, float *mse,
+                                                void *stream);
+
+/* ------------------------------------------------------------------------
  * BCJR soft codeword [BCJR: the argmax of Viterbi replaced by forward-backward
  * sum-product at temperature temp; the soft codeword is the Boltzmann
  * expectation over trellis walks].  A walk x has energy

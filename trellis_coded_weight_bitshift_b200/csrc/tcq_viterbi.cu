@@ -32,9 +32,10 @@
 
 namespace tcq {
 
-template <int L_, int G_, int SPC_, int AREG_, int NBUF_>
+template <int L_, int G_, int SPC_, int AREG_, int NBUF_, int MINB_ = 1>
 struct VitCfg {
   static constexpr int L = L_, G = G_, SPC = SPC_, AREG = AREG_, NBUF = NBUF_;
+  static constexpr int MINB = MINB_;                // CTAs per SM the registers must allow
   static constexpr int NG = 1 << (L - 2);      // groups (states / 4)
   static constexpr int TPS = NG / G;           // threads per sequence
   static constexpr int NT = TPS * SPC;         // threads per CTA
@@ -67,7 +68,7 @@ __device__ __forceinline__ void load_run(const float *base, int idx, float *dst)
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::NT, 1)
+__global__ void __launch_bounds__(C::NT, C::MINB)
 viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
                    uint8_t *__restrict__ bp, uint16_t *__restrict__ states,
                    float *__restrict__ mse) {
@@ -300,6 +301,86 @@ extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float 
   if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
   const int T = tr->seq_len;
   uint8_t *bp = static_cast<uint8_t *>(ws);
+  cudaStream_t strm = (cudaStream_t)stream;
+  switch (tr->L) {
+    case 8: st = launch_fwd<Vit8>(s, n_seq, T, bp, states, mse, strm); break;
+    case 12: st = launch_fwd<Vit12>(s, n_seq, T, bp, states, mse, strm); break;
+    default: st = launch_fwd<Vit16>(s, n_seq, T, bp, states, mse, strm); break;
+  }
+  if (st != TCQ_OK || T == 1) return st;
+  const unsigned tb_blocks = (unsigned)((n_seq + 127) / 128);
+  switch (tr->L) {
+    case 8: viterbi_traceback_kernel<8><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
+    case 12: viterbi_traceback_kernel<12><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
+    default: viterbi_traceback_kernel<16><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
+  }
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free Viterbi encode.
+//
+// Some callers may not allocate device memory when they call us: a plugin
+// whose host owns all device memory and hands it only the inputs and outputs,
+// or a deployment whose memory budget is fixed at start-up and that forbids
+// cudaMalloc afterwards.  This entry point keeps the backpointers in a fixed
+// buffer that is part of the library image instead of a caller workspace.
+//
+// The buffer below is a host-side symbol as far as host code is concerned:
+// its address on the device must be fetched with cudaGetSymbolAddress, with
+// the device current, before it can be passed to a kernel.  That is done once
+// per device, by the first call on that device, and cached.
+#include <atomic>
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB per device
+constexpr int kNoAllocMaxDevices = 64;
+
+std::atomic<uint8_t *> g_noalloc_scratch_ptr[kNoAllocMaxDevices];
+std::mutex g_noalloc_mutex;
+
+}  // namespace
+
+static __device__ __align__(256) uint8_t tcq_noalloc_scratch[kNoAllocScratchBytes];
+
+static tcq_status_t noalloc_scratch_for_current_device(uint8_t **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TCQ_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return TCQ_ERR_UNSUPPORTED;
+  uint8_t *p = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    p = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+      void *addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, tcq_noalloc_scratch) != cudaSuccess || addr == nullptr)
+        return TCQ_ERR_CUDA;
+      p = static_cast<uint8_t *>(addr);
+      g_noalloc_scratch_ptr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return TCQ_OK;
+}
+
+extern "C" tcq_status_t tcq_viterbi_encode_noalloc(const tcq_trellis_t *tr, const float *s,
+                                                   int64_t n_seq, uint16_t *states, float *mse,
+                                                   void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if (n_seq < 0 || n_seq > (int64_t)INT32_MAX * 8) return TCQ_ERR_INVALID_ARG;
+  if (n_seq == 0) return TCQ_OK;
+  if (!s || !states || !mse || !aligned16(s) || !aligned16(states) || !aligned16(mse))
+    return TCQ_ERR_INVALID_ARG;
+  const int T = tr->seq_len;
+  // every backpointer byte a call reads is written earlier in the same call,
+  // so the buffer needs no clearing between calls
+  if (bp_bytes_per_seq(tr->L, T) * (size_t)n_seq > kNoAllocScratchBytes) return TCQ_ERR_WORKSPACE;
+  uint8_t *bp = nullptr;
+  st = noalloc_scratch_for_current_device(&bp);
+  if (st != TCQ_OK) return st;
   cudaStream_t strm = (cudaStream_t)stream;
   switch (tr->L) {
     case 8: st = launch_fwd<Vit8>(s, n_seq, T, bp, states, mse, strm); break;
