@@ -47,9 +47,58 @@
 
 namespace tcq {
 
-template <int L_, int G_, int SPC_, int AREG_, int NBUF_, bool GRAD_>
+// Packed fp32 pairs (sm_100a f32x2 arithmetic, round-to-nearest per lane).
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t f2(float lo, float hi) {
+  f2_t r;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f2lo(f2_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+__device__ __forceinline__ float f2hi(f2_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
+}
+__device__ __forceinline__ f2_t f2sub(f2_t a, f2_t b) {
+  f2_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2mul(f2_t a, f2_t b) {
+  f2_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2add(f2_t a, f2_t b) {
+  f2_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2fma(f2_t a, f2_t b, f2_t c) {
+  f2_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// log2(2^x0 + 2^x1 + 2^x2 + 2^x3) with three ex2: after a min/max network
+// the largest term is exactly 1.
+__device__ __forceinline__ float lse4_base2(float x0, float x1, float x2, float x3) {
+  const float hi01 = fmaxf(x0, x1), lo01 = fminf(x0, x1);
+  const float hi23 = fmaxf(x2, x3), lo23 = fminf(x2, x3);
+  const float mx = fmaxf(hi01, hi23), mo = fminf(hi01, hi23);
+  const float S = (1.0f + ex2(lo01 - mx)) + (ex2(lo23 - mx) + ex2(mo - mx));
+  return mx + lg2(S);
+}
+
+template <int L_, int G_, int SPC_, int AREG_, int NBUF_, bool GRAD_, int MINB_ = 1>
 struct BcjrCfg {
   static constexpr int L = L_, G = G_, SPC = SPC_, AREG = AREG_, NBUF = NBUF_;
+  static constexpr int MINB = MINB_;                // CTAs per SM the registers must allow
   static constexpr bool GRAD = GRAD_;
   static constexpr int NG = 1 << (L - 2);
   static constexpr int TPS = NG / G;
@@ -79,6 +128,16 @@ __device__ __forceinline__ float code_at(const float (&creg)[C::AREG > 0 ? C::AR
                                          const float *Csm, int a, int i, int w) {
   if (a < C::AREG) return creg[a < C::AREG ? a : 0][i];
   return Csm[((a - C::AREG) * C::GQ + (i >> 2)) * C::TPS * 4 + w * 4 + (i & 3)];
+}
+
+// Code values of predecessor states (a, i) and (a, i+1) as a packed pair (i even).
+template <class C>
+__device__ __forceinline__ f2_t code_pair(const float (&creg)[C::AREG > 0 ? C::AREG : 1][C::G],
+                                         const float *Csm, int a, int i, int w) {
+  if (a < C::AREG) return f2(creg[a < C::AREG ? a : 0][i], creg[a < C::AREG ? a : 0][i + 1]);
+  const float2 v = *reinterpret_cast<const float2 *>(
+      &Csm[((a - C::AREG) * C::GQ + (i >> 2)) * C::TPS * 4 + w * 4 + (i & 3)]);
+  return f2(v.x, v.y);
 }
 
 // Reduce within the TPS lanes of a sequence (TPS < 32) or the whole warp.
@@ -127,7 +186,7 @@ __device__ __forceinline__ void write_run(float *vec, int base, const float *src
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::NT, 1)
+__global__ void __launch_bounds__(C::NT, C::MINB)
 bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, float two_over_temp,
             const float *__restrict__ vgrad, const float *__restrict__ soft_in,
             float *__restrict__ soft_out, float *__restrict__ logz_out,
@@ -228,38 +287,73 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
       const float vv = GRAD ? vsm[ls * 256 + t - 1] : 0.0f;
       const float fv = GRAD ? fsm[ls * 256 + t - 1] : 0.0f;
       float tmax = -INFINITY;
+      if constexpr (!GRAD) {
+        const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa);
 #pragma unroll
-      for (int q = 0; q < GQ; ++q) {
-        float outA[4], outF[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = 4 * q + r;
-          float x[4], c[4];
+        for (int q = 0; q < GQ; ++q) {
+          // x[a][r]: input of group 4q + r from predecessor digit a
+          float x[4][4];
 #pragma unroll
           for (int a = 0; a < 4; ++a) {
-            c[a] = code_at<C>(creg, Csm, a, i, w);
-            const float d = c[a] - sv;
-            x[a] = fmaf(-kappa * d, d, ain[a][q] - cmax);
-          }
-          const float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-          float u[4], S = 0.0f;
+            const float am = ain[a][q] - cmax;
+            const f2_t am2 = f2(am, am);
 #pragma unroll
-          for (int a = 0; a < 4; ++a) { u[a] = ex2(x[a] - mx); S += u[a]; }
-          outA[r] = mx + lg2(S);
-          tmax = fmaxf(tmax, outA[r]);
-          if (GRAD) {
-            float acc = 0.0f;
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-              acc = fmaf(u[a], fin[a < (GRAD ? 4 : 1) ? a : 0][q] + vv * (c[a] - fv), acc);
-            outF[r] = acc * __frcp_rn(S);
+            for (int h = 0; h < 2; ++h) {
+              const f2_t d = f2sub(code_pair<C>(creg, Csm, a, 4 * q + 2 * h, w), sv2);
+              const f2_t xv = f2fma(f2mul(d, nk2), d, am2);
+              x[a][2 * h] = f2lo(xv);
+              x[a][2 * h + 1] = f2hi(xv);
+            }
           }
+          float outA[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            outA[r] = lse4_base2(x[0][r], x[1][r], x[2][r], x[3][r]);
+            tmax = fmaxf(tmax, outA[r]);
+          }
+          *reinterpret_cast<float4 *>(Ao + swz<C::SWZ>(G * w + 4 * q)) =
+              make_float4(outA[0], outA[1], outA[2], outA[3]);
         }
-        *reinterpret_cast<float4 *>(Ao + swz<C::SWZ>(G * w + 4 * q)) =
-            make_float4(outA[0], outA[1], outA[2], outA[3]);
-        if (GRAD)
+      } else {
+        const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa), vv2 = f2(vv, vv);
+#pragma unroll
+        for (int q = 0; q < GQ; ++q) {
+          float x[4][4], z[4][4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const float am = ain[a][q] - cmax;
+            const float ph = fin[a < (GRAD ? 4 : 1) ? a : 0][q] - vv * fv;
+            const f2_t am2 = f2(am, am), ph2 = f2(ph, ph);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const f2_t cp = code_pair<C>(creg, Csm, a, 4 * q + 2 * h, w);
+              const f2_t d = f2sub(cp, sv2);
+              const f2_t xv = f2fma(f2mul(d, nk2), d, am2);
+              const f2_t zv = f2fma(vv2, cp, ph2);        // phi_{t-1}(p) = Phi + v (c - soft)
+              x[a][2 * h] = f2lo(xv); x[a][2 * h + 1] = f2hi(xv);
+              z[a][2 * h] = f2lo(zv); z[a][2 * h + 1] = f2hi(zv);
+            }
+          }
+          float outA[4], outF[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const float mx = fmaxf(fmaxf(x[0][r], x[1][r]), fmaxf(x[2][r], x[3][r]));
+            const f2_t e01 = f2sub(f2(x[0][r], x[1][r]), f2(mx, mx));
+            const f2_t e23 = f2sub(f2(x[2][r], x[3][r]), f2(mx, mx));
+            const f2_t u01 = f2(ex2(f2lo(e01)), ex2(f2hi(e01)));
+            const f2_t u23 = f2(ex2(f2lo(e23)), ex2(f2hi(e23)));
+            const f2_t su = f2add(u01, u23);
+            const f2_t sz = f2fma(u23, f2(z[2][r], z[3][r]), f2mul(u01, f2(z[0][r], z[1][r])));
+            const float S = f2lo(su) + f2hi(su);
+            outA[r] = mx + lg2(S);
+            tmax = fmaxf(tmax, outA[r]);
+            outF[r] = (f2lo(sz) + f2hi(sz)) * __frcp_rn(S);
+          }
+          *reinterpret_cast<float4 *>(Ao + swz<C::SWZ>(G * w + 4 * q)) =
+              make_float4(outA[0], outA[1], outA[2], outA[3]);
           *reinterpret_cast<float4 *>(Ao + NG + swz<C::SWZ>(G * w + 4 * q)) =
               make_float4(outF[0], outF[1], outF[2], outF[3]);
+        }
       }
       tmax = lane_reduce<TPS>(tmax, MaxOp());
       if (plead) prec(t & 1)[pidx * PREC] = tmax;
@@ -329,6 +423,14 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
     float DB = 0.0f;
     for (int t = T - 2; t >= -1; --t) {
       const int tc = t + 1;                                  // combine step
+      // this thread's spilled A_tc values (issued first: they come from HBM)
+      // (the gradient pass carries twice the values and would spill registers)
+      constexpr bool PREFETCH = !GRAD && G <= 16;
+      float4 avq[PREFETCH ? NCH : 1];
+      if constexpr (PREFETCH) {
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) avq[c] = spill[((size_t)tc * NCH + c) * TPS + w];
+      }
       const float *Bi = Bv + (tc % NB) * NV * NG;
       float bin[G], pin[GRAD ? G : 1];
 #pragma unroll
@@ -366,59 +468,100 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
       const float fv = GRAD ? fsm[ls * 256 + tc] : 0.0f;
       float *Bo = Bv + ((t + NB) % NB) * NV * NG;
       float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f, tmax = -INFINITY;
+      if constexpr (!GRAD) {
+        const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa);
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        float av[GQ], fa[GRAD ? GQ : 1];
+        for (int a = 0; a < 4; ++a) {
+          float av[GQ];
 #pragma unroll
-        for (int q = 0; q < (GQ + 3) / 4; ++q) {
-          const int f = a * GQ + 4 * q;
-          const float4 v = spill[((size_t)tc * NCH + (f >> 2)) * TPS + w];
-          const float e4[4] = {v.x, v.y, v.z, v.w};
+          for (int q = 0; q < (GQ + 3) / 4; ++q) {
+            const int f = a * GQ + 4 * q;
+            float4 v;
+            if constexpr (PREFETCH) v = avq[PREFETCH ? (f >> 2) : 0];
+            else v = spill[((size_t)tc * NCH + (f >> 2)) * TPS + w];
+            const float e4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) av[4 * q + k] = e4[(f & 3) + k];
-          if (GRAD) {
-            const int g = G + a * GQ + 4 * q;
+            for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) av[4 * q + k] = e4[(f & 3) + k];
+          }
+          float outB[GQ];
+#pragma unroll
+          for (int k = 0; k < GQ; ++k) {
+            const f2_t c01 = code_pair<C>(creg, Csm, a, 4 * k, w);
+            const f2_t c23 = code_pair<C>(creg, Csm, a, 4 * k + 2, w);
+            const f2_t d01 = f2sub(c01, sv2), d23 = f2sub(c23, sv2);
+            const f2_t y01 = f2fma(f2mul(d01, nk2), d01, f2(bin[4 * k], bin[4 * k + 1]));
+            const f2_t y23 = f2fma(f2mul(d23, nk2), d23, f2(bin[4 * k + 2], bin[4 * k + 3]));
+            const float mx = fmaxf(fmaxf(f2lo(y01), f2hi(y01)), fmaxf(f2lo(y23), f2hi(y23)));
+            const f2_t mx2 = f2(mx, mx);
+            const f2_t e01 = f2sub(y01, mx2), e23 = f2sub(y23, mx2);
+            const f2_t u01 = f2(ex2(f2lo(e01)), ex2(f2hi(e01)));
+            const f2_t u23 = f2(ex2(f2lo(e23)), ex2(f2hi(e23)));
+            const f2_t su = f2add(u01, u23);
+            const f2_t sc = f2fma(u23, c23, f2mul(u01, c01));
+            const float S = f2lo(su) + f2hi(su), Sc = f2lo(sc) + f2hi(sc);
+            outB[k] = (mx - dprev) + lg2(S);
+            tmax = fmaxf(tmax, outB[k]);
+            const float wgt = ex2((av[k] - K) + mx);
+            den = fmaf(wgt, S, den);
+            num = fmaf(wgt, Sc, num);
+          }
+          if (t >= 0) write_run<C>(Bo, a * (NG / 4) + GQ * w, outB);
+        }
+      } else {
+        const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa), vv2 = f2(vv, vv);
+        const float nvf = -vv * fv;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          float av[GQ], fa[GQ];
+#pragma unroll
+          for (int q = 0; q < (GQ + 3) / 4; ++q) {
+            const int f = a * GQ + 4 * q, g = G + a * GQ + 4 * q;
+            const float4 v = spill[((size_t)tc * NCH + (f >> 2)) * TPS + w];
             const float4 u = spill[((size_t)tc * NCH + (g >> 2)) * TPS + w];
+            const float e4[4] = {v.x, v.y, v.z, v.w};
             const float g4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) fa[(4 * q + k) < (GRAD ? GQ : 1) ? 4 * q + k : 0] = g4[(g & 3) + k];
+            for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) {
+              av[4 * q + k] = e4[(f & 3) + k];
+              fa[4 * q + k] = g4[(g & 3) + k];
+            }
           }
-        }
-        float outB[GQ], outP[GQ];
+          float outB[GQ], outP[GQ];
 #pragma unroll
-        for (int k = 0; k < GQ; ++k) {
-          float y[4], c[4], z[4];
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            c[b] = code_at<C>(creg, Csm, a, 4 * k + b, w);
-            const float d = c[b] - sv;
-            y[b] = fmaf(-kappa * d, d, bin[4 * k + b]);
-            z[b] = GRAD ? pin[GRAD ? 4 * k + b : 0] + vv * (c[b] - fv) : 0.0f;
-          }
-          const float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
-          float S = 0.0f, Sc = 0.0f, Sz = 0.0f, Scz = 0.0f;
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const float u = ex2(y[b] - mx);
-            S += u;
-            Sc = fmaf(u, c[b], Sc);
-            if (GRAD) { Sz = fmaf(u, z[b], Sz); Scz = fmaf(u * c[b], z[b], Scz); }
-          }
-          outB[k] = mx + lg2(S) - dprev;
-          tmax = fmaxf(tmax, outB[k]);
-          const float wgt = ex2(av[k] + mx - K);
-          den = fmaf(wgt, S, den);
-          num = fmaf(wgt, Sc, num);
-          if (GRAD) {
-            const float fk = fa[GRAD ? k : 0];
+          for (int k = 0; k < GQ; ++k) {
+            const f2_t c01 = code_pair<C>(creg, Csm, a, 4 * k, w);
+            const f2_t c23 = code_pair<C>(creg, Csm, a, 4 * k + 2, w);
+            const f2_t d01 = f2sub(c01, sv2), d23 = f2sub(c23, sv2);
+            const f2_t y01 = f2fma(f2mul(d01, nk2), d01, f2(bin[4 * k], bin[4 * k + 1]));
+            const f2_t y23 = f2fma(f2mul(d23, nk2), d23, f2(bin[4 * k + 2], bin[4 * k + 3]));
+            // z_b = psi_{tc}(succ) + v_tc (c_b - soft_tc)
+            const f2_t z01 = f2fma(vv2, c01, f2add(f2(pin[4 * k], pin[4 * k + 1]), f2(nvf, nvf)));
+            const f2_t z23 = f2fma(vv2, c23, f2add(f2(pin[4 * k + 2], pin[4 * k + 3]), f2(nvf, nvf)));
+            const float mx = fmaxf(fmaxf(f2lo(y01), f2hi(y01)), fmaxf(f2lo(y23), f2hi(y23)));
+            const f2_t mx2 = f2(mx, mx);
+            const f2_t e01 = f2sub(y01, mx2), e23 = f2sub(y23, mx2);
+            const f2_t u01 = f2(ex2(f2lo(e01)), ex2(f2hi(e01)));
+            const f2_t u23 = f2(ex2(f2lo(e23)), ex2(f2hi(e23)));
+            const f2_t uc01 = f2mul(u01, c01), uc23 = f2mul(u23, c23);
+            const f2_t su = f2add(u01, u23);
+            const f2_t sc = f2add(uc01, uc23);
+            const f2_t sz = f2fma(u23, z23, f2mul(u01, z01));
+            const f2_t scz = f2fma(uc23, z23, f2mul(uc01, z01));
+            const float S = f2lo(su) + f2hi(su), Sc = f2lo(sc) + f2hi(sc);
+            const float Sz = f2lo(sz) + f2hi(sz), Scz = f2lo(scz) + f2hi(scz);
+            outB[k] = (mx - dprev) + lg2(S);
+            tmax = fmaxf(tmax, outB[k]);
             outP[k] = Sz * __frcp_rn(S);
-            n1 = fmaf(wgt, fmaf(fk, S, Sz), n1);
-            n2 = fmaf(wgt, fmaf(fk, Sc, Scz), n2);
+            const float wgt = ex2((av[k] - K) + mx);
+            den = fmaf(wgt, S, den);
+            num = fmaf(wgt, Sc, num);
+            n1 = fmaf(wgt, fmaf(fa[k], S, Sz), n1);
+            n2 = fmaf(wgt, fmaf(fa[k], Sc, Scz), n2);
           }
-        }
-        if (t >= 0) {
-          write_run<C>(Bo, a * (NG / 4) + GQ * w, outB);
-          if (GRAD) write_run<C>(Bo + NG, a * (NG / 4) + GQ * w, outP);
+          if (t >= 0) {
+            write_run<C>(Bo, a * (NG / 4) + GQ * w, outB);
+            write_run<C>(Bo + NG, a * (NG / 4) + GQ * w, outP);
+          }
         }
       }
       tmax = lane_reduce<TPS>(tmax, MaxOp());
@@ -457,10 +600,10 @@ using namespace tcq_host;
 namespace {
 
 using Soft8 = BcjrCfg<8, 4, 8, 4, 2, false>;
-using Soft12 = BcjrCfg<12, 4, 1, 4, 2, false>;
+using Soft12 = BcjrCfg<12, 16, 1, 4, 2, false, 7>;   // 64 threads / sequence, 7 per SM: one wave of 1,036
 using Soft16 = BcjrCfg<16, 32, 1, 2, 1, false>;
 using Grad8 = BcjrCfg<8, 4, 8, 4, 2, true>;
-using Grad12 = BcjrCfg<12, 4, 1, 4, 2, true>;
+using Grad12 = BcjrCfg<12, 16, 1, 4, 2, true, 8>;    // 64 threads / sequence, 8 per SM
 
 template <class C>
 int grid_for(int64_t n_seq) {

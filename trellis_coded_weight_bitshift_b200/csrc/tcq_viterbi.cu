@@ -235,6 +235,36 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
   }
 }
 
+// Traceback with the sequence's backpointers staged in shared memory (L <= 12:
+// at most 64 KiB per sequence): the CTA copies them with 16-byte loads, then
+// one thread walks st[t-1] = (st[t] >> 2) | (bp_t(st[t] >> 2) << (L-2)) from
+// shared memory and the CTA writes the walk out coalesced.
+template <int L>
+__global__ void __launch_bounds__(256) viterbi_traceback_staged_kernel(const uint8_t *__restrict__ bp,
+                                                                       int64_t n_seq, int T,
+                                                                       uint16_t *__restrict__ states) {
+  constexpr int ROW = 1 << (L - 4);                       // backpointer bytes per step
+  extern __shared__ __align__(16) uint8_t sbp[];          // [T-1][ROW], then [256] uint16 walk
+  uint16_t *swalk = reinterpret_cast<uint16_t *>(sbp + (size_t)(T - 1) * ROW);
+  const int64_t seq = blockIdx.x;
+  const uint4 *src = reinterpret_cast<const uint4 *>(bp + seq * (int64_t)(T - 1) * ROW);
+  const int n16 = (T - 1) * ROW / 16;
+  for (int x = threadIdx.x; x < n16; x += blockDim.x) reinterpret_cast<uint4 *>(sbp)[x] = __ldg(src + x);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t cur = states[seq * T + T - 1];
+    swalk[T - 1] = (uint16_t)cur;
+    for (int t = T - 1; t > 0; --t) {
+      const uint32_t q = cur >> 2;
+      const uint32_t a = (sbp[(t - 1) * ROW + (q >> 2)] >> (2 * (q & 3))) & 3u;
+      cur = q | (a << (L - 2));
+      swalk[t - 1] = (uint16_t)cur;
+    }
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < T - 1; t += blockDim.x) states[seq * T + t] = swalk[t];
+}
+
 // Traceback: one thread per sequence, st[t-1] = (st[t] >> 2) | (bp_t(st[t] >> 2) << (L-2)).
 template <int L>
 __global__ void __launch_bounds__(128) viterbi_traceback_kernel(const uint8_t *__restrict__ bp,
@@ -281,6 +311,30 @@ tcq_status_t launch_fwd(const float *s, int64_t n_seq, int T, uint8_t *bp, uint1
   return launch_status();
 }
 
+template <int L>
+tcq_status_t launch_traceback_staged(const uint8_t *bp, int64_t n_seq, int T, uint16_t *states,
+                                     cudaStream_t stream) {
+  const size_t smem = (size_t)(T - 1) * ((size_t)1 << (L - 4)) + 256 * sizeof(uint16_t);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(viterbi_traceback_staged_kernel<L>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return TCQ_ERR_CUDA;
+  viterbi_traceback_staged_kernel<L><<<(unsigned)n_seq, 256, smem, stream>>>(bp, n_seq, T, states);
+  return launch_status();
+}
+
+tcq_status_t launch_traceback(int L, const uint8_t *bp, int64_t n_seq, int T, uint16_t *states,
+                              cudaStream_t stream) {
+  switch (L) {
+    case 8: return launch_traceback_staged<8>(bp, n_seq, T, states, stream);
+    case 12: return launch_traceback_staged<12>(bp, n_seq, T, states, stream);
+    default:
+      viterbi_traceback_kernel<16><<<(unsigned)((n_seq + 127) / 128), 128, 0, stream>>>(bp, n_seq, T,
+                                                                                        states);
+      return launch_status();
+  }
+}
+
 }  // namespace
 
 extern "C" size_t tcq_viterbi_workspace_size(const tcq_trellis_t *tr, int64_t n_seq) {
@@ -308,13 +362,7 @@ extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float 
     default: st = launch_fwd<Vit16>(s, n_seq, T, bp, states, mse, strm); break;
   }
   if (st != TCQ_OK || T == 1) return st;
-  const unsigned tb_blocks = (unsigned)((n_seq + 127) / 128);
-  switch (tr->L) {
-    case 8: viterbi_traceback_kernel<8><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
-    case 12: viterbi_traceback_kernel<12><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
-    default: viterbi_traceback_kernel<16><<<tb_blocks, 128, 0, strm>>>(bp, n_seq, T, states); break;
-  }
-  return launch_status();
+  return launch_traceback(tr->L, bp, n_seq, T, states, strm);
 }
 
 // ---------------------------------------------------------------------------
