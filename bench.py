@@ -20,7 +20,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -44,6 +43,8 @@ def _args():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--n-seq", type=int, default=0,
+                   help="encode only the first N sequences of the workload (profiling runs)")
     return p.parse_args()
 
 
@@ -66,52 +67,66 @@ def _weights_per_step(w: W.Workload) -> int:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
-              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
-              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the clock-event reasons (read-only NVML queries)
+    from a background thread while the timed region runs, plus once on entry
+    and once on exit so that even a sub-millisecond region gets samples."""
 
-    def __init__(self, gpu_id: str):
-        self.proc = None
-        self.gpu_id = gpu_id
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown"}
+
+    def __init__(self, gpu_uuid: str):
+        self.gpu_uuid = gpu_uuid
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+
+    def _sample(self):
+        import pynvml
+        sm = pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        try:
+            rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            rs = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append((sm, rs))
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._sample()
+        except Exception:
+            self.h = None
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.wait(0.01):
+                try:
+                    self._sample()
+                except Exception:
+                    return
+        self._t = threading.Thread(target=loop, daemon=True)
+        self._t.start()
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._stop is not None:
+            self._stop.set()
+            self._t.join(timeout=2)
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self._sample()
+            except Exception:
+                pass
 
     def summary(self) -> dict:
-        rows = [r.split(", ") for r in getattr(self, "out", "").strip().splitlines() if r.strip()]
-        sm, mx, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for r in rows:
-            if len(r) < len(self.FIELDS):
-                continue
-            try:
-                sm.append(float(r[0])); mx.append(float(r[1]))
-            except ValueError:
-                continue
-            for name, val in zip(names, r[4:8]):
-                if val.strip().lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        reasons = sorted({name for _, rs in self.samples for bit, name in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -217,6 +232,9 @@ def run_ours(a) -> None:
         dist.barrier()
     dev = torch.device("cuda", torch.cuda.current_device())
     w = W.WORKLOADS[a.workload]
+    if a.n_seq and a.n_seq < w.n_seq:
+        import dataclasses
+        w = dataclasses.replace(w, n_seq=a.n_seq, rows=0, cols=0)
 
     # ---- inputs (each rank its own batch: seed offset by rank) ----
     if w.ops == ("decode",):
@@ -225,10 +243,10 @@ def run_ours(a) -> None:
         h2d_bytes = host.nbytes
     else:
         if rank == 0:
-            host = W.sequences(w.name)
+            host = W.sequences(w.name, n_limit=w.n_seq)
         else:
             rng = np.random.default_rng(w.seed + 1000 * rank)
-            host = W.sequences(w.name) if w.kind != "gaussian" else \
+            host = W.sequences(w.name, n_limit=w.n_seq) if w.kind != "gaussian" else \
                 rng.standard_normal((w.n_seq, W.SEQ_LEN)).astype(np.float32)
         x = torch.from_numpy(host).to(dev)
         h2d_bytes = host.nbytes
@@ -290,12 +308,8 @@ def run_ours(a) -> None:
     torch.cuda.synchronize()
 
     # ---- device-timed region ----
-    gpu_id = "0"
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-    except Exception:
-        gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[local] if world > 1 else "0"
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -370,7 +384,7 @@ def run_ours(a) -> None:
                 "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes)},
         "gpu_launches": launches_per_step * a.steps,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                   "reasons": clocks["reasons"]},
+                   "reasons": clocks["reasons"], "samples": clocks["samples"]},
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)

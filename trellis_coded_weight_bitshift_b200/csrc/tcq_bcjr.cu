@@ -47,44 +47,6 @@
 
 namespace tcq {
 
-// Packed fp32 pairs (sm_100a f32x2 arithmetic, round-to-nearest per lane).
-typedef unsigned long long f2_t;
-__device__ __forceinline__ f2_t f2(float lo, float hi) {
-  f2_t r;
-  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float f2lo(f2_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
-}
-__device__ __forceinline__ float f2hi(f2_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
-}
-__device__ __forceinline__ f2_t f2sub(f2_t a, f2_t b) {
-  f2_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f2_t f2mul(f2_t a, f2_t b) {
-  f2_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f2_t f2add(f2_t a, f2_t b) {
-  f2_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f2_t f2fma(f2_t a, f2_t b, f2_t c) {
-  f2_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-
 // log2(2^x0 + 2^x1 + 2^x2 + 2^x3) with three ex2: after a min/max network
 // the largest term is exactly 1.
 __device__ __forceinline__ float lse4_base2(float x0, float x1, float x2, float x3) {
@@ -510,20 +472,33 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
       } else {
         const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa), vv2 = f2(vv, vv);
         const float nvf = -vv * fv;
+        // spilled (A, Phi) values of digit a, loaded one digit ahead
+        constexpr int QN = (GQ + 3) / 4;
+        float4 nv[QN], nu[QN];
+#pragma unroll
+        for (int q = 0; q < QN; ++q) {
+          nv[q] = spill[((size_t)tc * NCH + ((0 * GQ + 4 * q) >> 2)) * TPS + w];
+          nu[q] = spill[((size_t)tc * NCH + ((G + 0 * GQ + 4 * q) >> 2)) * TPS + w];
+        }
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           float av[GQ], fa[GQ];
 #pragma unroll
-          for (int q = 0; q < (GQ + 3) / 4; ++q) {
+          for (int q = 0; q < QN; ++q) {
             const int f = a * GQ + 4 * q, g = G + a * GQ + 4 * q;
-            const float4 v = spill[((size_t)tc * NCH + (f >> 2)) * TPS + w];
-            const float4 u = spill[((size_t)tc * NCH + (g >> 2)) * TPS + w];
-            const float e4[4] = {v.x, v.y, v.z, v.w};
-            const float g4[4] = {u.x, u.y, u.z, u.w};
+            const float e4[4] = {nv[q].x, nv[q].y, nv[q].z, nv[q].w};
+            const float g4[4] = {nu[q].x, nu[q].y, nu[q].z, nu[q].w};
 #pragma unroll
             for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) {
               av[4 * q + k] = e4[(f & 3) + k];
               fa[4 * q + k] = g4[(g & 3) + k];
+            }
+          }
+          if (a < 3) {
+#pragma unroll
+            for (int q = 0; q < QN; ++q) {
+              nv[q] = spill[((size_t)tc * NCH + (((a + 1) * GQ + 4 * q) >> 2)) * TPS + w];
+              nu[q] = spill[((size_t)tc * NCH + ((G + (a + 1) * GQ + 4 * q) >> 2)) * TPS + w];
             }
           }
           float outB[GQ], outP[GQ];
@@ -600,10 +575,10 @@ using namespace tcq_host;
 namespace {
 
 using Soft8 = BcjrCfg<8, 4, 8, 4, 2, false>;
-using Soft12 = BcjrCfg<12, 16, 1, 4, 2, false, 7>;   // 64 threads / sequence, 7 per SM: one wave of 1,036
+using Soft12 = BcjrCfg<12, 8, 1, 4, 2, false, 7>;    // 128 threads / sequence, 7 per SM: one wave of 1,036
 using Soft16 = BcjrCfg<16, 32, 1, 2, 1, false>;
 using Grad8 = BcjrCfg<8, 4, 8, 4, 2, true>;
-using Grad12 = BcjrCfg<12, 16, 1, 4, 2, true, 8>;    // 64 threads / sequence, 8 per SM
+using Grad12 = BcjrCfg<12, 8, 1, 4, 2, true, 7>;     // 128 threads / sequence, 7 per SM
 
 template <class C>
 int grid_for(int64_t n_seq) {

@@ -63,15 +63,16 @@ __global__ void __launch_bounds__(256) decode_tile16_kernel(const uint32_t *__re
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
       // weights t = 16 r + 8 h + j, stream bit 2t = 32 r + 16 h + 2 j
-      float c[8];
+      uint32_t hv[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        c[j] = one_mad_decode_f32(window_at<L>(w[r], w[r + 1], 16 * h + 2 * j));
+      for (int j = 0; j < 4; ++j) {
+        const unsigned long long c2 =
+            one_mad_decode_f32x2(window_at<L>(w[r], w[r + 1], 16 * h + 4 * j),
+                                 window_at<L>(w[r], w[r + 1], 16 * h + 4 * j + 2));
+        hv[j] = pack_half2(__uint_as_float((uint32_t)c2), __uint_as_float((uint32_t)(c2 >> 32)));
+      }
       uint4 o;
-      o.x = pack_half2(c[0], c[1]);
-      o.y = pack_half2(c[2], c[3]);
-      o.z = pack_half2(c[4], c[5]);
-      o.w = pack_half2(c[6], c[7]);
+      o.x = hv[0]; o.y = hv[1]; o.z = hv[2]; o.w = hv[3];
       *reinterpret_cast<uint4 *>(dst + (int64_t)r * cols) = o;
     }
   }

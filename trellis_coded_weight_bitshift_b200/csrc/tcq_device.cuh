@@ -42,6 +42,65 @@ __device__ __forceinline__ float one_mad_decode_f32(uint32_t x) {
   return __fmul_rn(centred, 0x1.bb68f6p-8f);  // RN32(1/147.8)
 }
 
+// The same value for two states at once, arranged for throughput: the byte sum
+// is a dot product with 0x01010101 whose accumulator carries the 2^23 exponent
+// bits (IDP4A, integer multiply-add pipe), and the centring and scaling run as
+// one packed fp32 pair (sub then mul, each correctly rounded per lane).
+__device__ __forceinline__ unsigned long long one_mad_decode_f32x2(uint32_t x0, uint32_t x1) {
+  const uint32_t m0 = __dp4a(x0 * kLcgMul + kLcgAdd, 0x01010101u, 0x4B000000u);
+  const uint32_t m1 = __dp4a(x1 * kLcgMul + kLcgAdd, 0x01010101u, 0x4B000000u);
+  unsigned long long v, c, r;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(v) : "r"(m0), "r"(m1));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(c) : "f"(8389118.0f));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(v), "l"(c));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(c) : "f"(0x1.bb68f6p-8f));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(r), "l"(c));
+  return r;
+}
+
+// Packed fp32 pairs (sm_100a f32x2 arithmetic, round-to-nearest per lane).
+// Each lane of sub/mul/add/fma.rn.f32x2 is the correctly rounded scalar
+// operation.  Note: ptxas may fuse a packed mul whose only use is a packed add
+// into one fma; code that needs the separately rounded product writes the
+// square as fma(d, d, +0), which rounds exactly like d * d for d * d >= 0 and
+// cannot be fused further.
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t f2(float lo, float hi) {
+  f2_t r;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f2lo(f2_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+__device__ __forceinline__ float f2hi(f2_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
+}
+__device__ __forceinline__ f2_t f2sub(f2_t a, f2_t b) {
+  f2_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2mul(f2_t a, f2_t b) {
+  f2_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2add(f2_t a, f2_t b) {
+  f2_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t f2fma(f2_t a, f2_t b, f2_t c) {
+  f2_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

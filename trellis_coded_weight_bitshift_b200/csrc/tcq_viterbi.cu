@@ -85,12 +85,15 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
   const int64_t seq = (int64_t)blockIdx.x * C::SPC + ls;
   const bool active = seq < n_seq;
 
-  // Code values of this thread's predecessor states p = a*NG + G*w + i.
-  float creg[AREG > 0 ? AREG : 1][G];
+  // Code values of this thread's predecessor states p = a*NG + G*w + i, as
+  // packed pairs (i, i+1).
+  f2_t creg[AREG > 0 ? AREG : 1][G / 2];
 #pragma unroll
   for (int a = 0; a < AREG; ++a)
 #pragma unroll
-    for (int i = 0; i < G; ++i) creg[a][i] = one_mad_f32((uint32_t)(a * NG + G * w + i));
+    for (int i = 0; i < G; i += 2)
+      creg[a][i / 2] = f2(one_mad_f32((uint32_t)(a * NG + G * w + i)),
+                          one_mad_f32((uint32_t)(a * NG + G * w + i + 1)));
   if (ls == 0) {
 #pragma unroll
     for (int a = 0; a < ASM; ++a)
@@ -142,6 +145,11 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
     uint32_t bits[(2 * G + 31) / 32];
 #pragma unroll
     for (int b = 0; b < (2 * G + 31) / 32; ++b) bits[b] = 0;
+    // Two neighbouring groups i, i+1 with the same predecessor digit a share
+    // the input M(q), so their candidate costs are computed as a packed pair:
+    // d = c - s, e = d*d (written fma(d, d, +0)), cost = M + e, each lane
+    // rounded exactly like the scalar operation.
+    const f2_t sv2 = f2(sv, sv);
 #pragma unroll
     for (int q = 0; q < GQ; ++q) {
       float4 csm[ASM > 0 ? ASM : 1];
@@ -149,29 +157,37 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
       for (int a = 0; a < ASM; ++a) csm[a] = reinterpret_cast<const float4 *>(Csm)[(a * GQ + q) * TPS + w];
       float outv[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = 4 * q + r;
-        float cst[4];
+      for (int h = 0; h < 2; ++h) {
+        float clo[4], chi[4];
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
-          float c;
-          if (a < AREG) c = creg[a < AREG ? a : 0][i];
+          f2_t cp;
+          if (a < AREG) cp = creg[a < AREG ? a : 0][2 * q + h];
           else {
             const float4 v = csm[a >= AREG ? a - AREG : 0];
-            c = r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
+            cp = h == 0 ? f2(v.x, v.y) : f2(v.z, v.w);
           }
-          const float d = __fsub_rn(c, sv);
-          cst[a] = __fadd_rn(min_in[a][q], __fmul_rn(d, d));
+          const f2_t d = f2sub(cp, sv2);
+          const f2_t cost = f2add(f2(min_in[a][q], min_in[a][q]), f2fma(d, d, 0ull));
+          clo[a] = f2lo(cost);
+          chi[a] = f2hi(cost);
         }
-        // first minimum (lowest a) of the four candidates
-        const bool p1 = cst[1] < cst[0];
-        const float m01 = p1 ? cst[1] : cst[0];
-        const bool p2 = cst[3] < cst[2];
-        const float m23 = p2 ? cst[3] : cst[2];
-        const bool p3 = m23 < m01;
-        outv[r] = p3 ? m23 : m01;
-        const uint32_t idx = p3 ? (2u | (uint32_t)p2) : (uint32_t)p1;
-        bits[i >> 4] |= idx << (2 * (i & 15));
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float *cst = u == 0 ? clo : chi;
+          const int r = 2 * h + u, i = 4 * q + r;
+          // First minimum (lowest a) of the four candidates with the DPX
+          // min-with-predicate: costs are sums of squares (>= +0), so their bit
+          // patterns order like their values, and (x <= y) keeps the lower
+          // index on ties.
+          bool q1, q2, q3;
+          const int m01 = __vibmin_s32(__float_as_int(cst[0]), __float_as_int(cst[1]), &q1);
+          const int m23 = __vibmin_s32(__float_as_int(cst[2]), __float_as_int(cst[3]), &q2);
+          const int m = __vibmin_s32(m01, m23, &q3);
+          outv[r] = __int_as_float(m);
+          const uint32_t idx = q3 ? (q1 ? 0u : 1u) : (q2 ? 2u : 3u);
+          bits[i >> 4] |= idx << (2 * (i & 15));
+        }
       }
       *reinterpret_cast<float4 *>(Mo + swz<C::SWZ>(G * w + 4 * q)) =
           make_float4(outv[0], outv[1], outv[2], outv[3]);
@@ -201,8 +217,10 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           float c;
-          if (a < AREG) c = creg[a < AREG ? a : 0][i];
-          else {
+          if (a < AREG) {
+            const f2_t cp = creg[a < AREG ? a : 0][i >> 1];
+            c = (i & 1) ? f2hi(cp) : f2lo(cp);
+          } else {
             const float4 v = csm[a >= AREG ? a - AREG : 0];
             c = r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
           }
@@ -292,7 +310,7 @@ using namespace tcq_host;
 namespace {
 
 using Vit8 = VitCfg<8, 4, 8, 4, 2>;      // 16 threads / sequence, 8 sequences / CTA
-using Vit12 = VitCfg<12, 4, 1, 4, 2>;    // 256 threads / sequence
+using Vit12 = VitCfg<12, 8, 1, 4, 2, 8>;  // 128 threads / sequence, 8 per SM: one wave
 using Vit16 = VitCfg<16, 32, 1, 2, 1>;   // 512 threads / sequence, half the codes in smem
 
 size_t bp_bytes_per_seq(int L, int T) { return (size_t)(T - 1) * ((size_t)1 << (L - 4)); }

@@ -12,10 +12,11 @@ Units of work (per sequence of T = 256 weights on a 2^L-state trellis):
                  Peak: 128 lane-instructions per clock per SM (4 schedulers x
                  32 lanes, also the fp32 FMA rate) x SMs x max SM clock.
   bcjr  (MUFU):  per group of 4 states and step, the forward log-sum-exp over
-                 4 predecessors (4 ex2 + 1 lg2) and the backward one over 4
-                 successors (4 ex2 + 1 lg2) plus the group's posterior weight
-                 (1 ex2): 11 / 4 special-function ops per state-step; the
-                 gradient pass adds a reciprocal in each direction (13 / 4).
+                 4 predecessors and the backward one over 4 successors, each
+                 3 ex2 + 1 lg2 once the largest term (exactly 1) is known, plus
+                 the group's posterior weight (1 ex2): 9 / 4 special-function
+                 ops per state-step; the gradient pass adds a reciprocal in
+                 each direction (11 / 4).
                  Peak: 16 special-function results per clock per SM x SMs x
                  max SM clock.
 """
@@ -50,9 +51,9 @@ def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str,
     if kernel.startswith("viterbi"):
         return "alu", n_seq * T * states * 4.5, "lane-ops"
     if kernel.startswith("bcjr_vjp"):
-        return "alu", n_seq * T * states * 13 / 4, "mufu-ops"
-    if kernel.startswith("bcjr"):
         return "alu", n_seq * T * states * 11 / 4, "mufu-ops"
+    if kernel.startswith("bcjr"):
+        return "alu", n_seq * T * states * 9 / 4, "mufu-ops"
     raise KeyError(kernel)
 
 
