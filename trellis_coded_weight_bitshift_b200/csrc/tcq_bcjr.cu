@@ -47,6 +47,17 @@
 
 namespace tcq {
 
+// Cache prefetch of a global address (no register result).
+template <int LEVEL>
+__device__ __forceinline__ void prefetch_global(const void *p) {
+  if constexpr (LEVEL == 1) asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+  else if constexpr (LEVEL == 2) asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+#ifndef TCQ_SPILL_PREFETCH_LEVEL
+#define TCQ_SPILL_PREFETCH_LEVEL 2
+#endif
+
 // log2(2^x0 + 2^x1 + 2^x2 + 2^x3) with three ex2: after a min/max network
 // the largest term is exactly 1.
 __device__ __forceinline__ float lse4_base2(float x0, float x1, float x2, float x3) {
@@ -392,6 +403,15 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
       if constexpr (PREFETCH) {
 #pragma unroll
         for (int c = 0; c < NCH; ++c) avq[c] = spill[((size_t)tc * NCH + c) * TPS + w];
+      }
+      // the next step's spilled chunks are read a whole step from now: start
+      // bringing them on chip (register prefetch covers the small soft case)
+      if constexpr (!PREFETCH) {
+        if (tc > 0) {
+#pragma unroll
+          for (int c = 0; c < NCH; ++c)
+            prefetch_global<TCQ_SPILL_PREFETCH_LEVEL>(&spill[((size_t)(tc - 1) * NCH + c) * TPS + w]);
+        }
       }
       const float *Bi = Bv + (tc % NB) * NV * NG;
       float bin[G], pin[GRAD ? G : 1];

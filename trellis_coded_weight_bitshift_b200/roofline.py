@@ -22,6 +22,7 @@ Units of work (per sequence of T = 256 weights on a 2^L-state trellis):
 """
 from __future__ import annotations
 
+import hashlib
 import json
 import os
 
@@ -29,6 +30,41 @@ SEQ_LEN = 256
 B200_SMS = 148
 ISSUE_LANES_PER_SM = 128       # 4 schedulers x 32 lanes per clock
 MUFU_PER_SM = 16               # special-function results per clock per SM
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from
+# ncu captures, with the sha1 of the kernel sources they were taken on: once a
+# source changes, the figure no longer describes the kernel and is reported as
+# null.  (kernel prefix, workload): (bytes, sequences in the capture, sources)
+_CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
+MEASURED_TRAFFIC = {
+    ("bcjr_vjp", "l12_gauss1024"): (2.142159e9 + 2.176458e9, 1024, {
+        "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
+        "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
+    ("bcjr_soft", "l12_gauss1024"): (1.020003e9 + 1.082902e9, 1024, {
+        "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
+        "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
+    # captured on the first 64 sequences; traffic scales with the sequences
+    ("bcjr_soft", "l16_studentt_2048x8192"): (0.99031168e9 + 1.080753e9, 64, {
+        "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
+        "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
+}
+
+
+def _sha1(name: str) -> str:
+    with open(os.path.join(_CSRC, name), "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+def measured_traffic(kernel: str, workload) -> float | None:
+    """Bytes per launch for this kernel and workload, or None if never
+    captured or if the kernel's sources changed since the capture."""
+    for (prefix, wl), (nbytes, n_cap, srcs) in MEASURED_TRAFFIC.items():
+        if kernel.startswith(prefix) and workload.name == wl:
+            if any(_sha1(f) != h for f, h in srcs.items()):
+                return None
+            return nbytes * workload.n_seq / n_cap
+    return None
 
 
 def load_measured_peaks(root: str) -> dict:
@@ -57,8 +93,9 @@ def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str,
     raise KeyError(kernel)
 
 
-def roofline_entry(kernel: str, workload, ms: float, peaks: dict, traffic=None) -> dict:
+def roofline_entry(kernel: str, workload, ms: float, peaks: dict) -> dict:
     bound, work, unit = kernel_work(kernel, workload.L, workload.n_seq)
+    traffic = measured_traffic(kernel, workload)
     sec = ms * 1e-3
     clk = peaks["sm_max_mhz"] * 1e6
     if bound == "hbm":
