@@ -208,6 +208,29 @@ def run_reference(a) -> None:
     print(json.dumps(line))
 
 
+# ------------------------------------------------------------------ ranks
+def rank_batch(w: W.Workload, rank: int) -> np.ndarray:
+    """The batch rank `rank` encodes (weak scaling: every rank a batch of the
+    workload's size, no data exchanged).  Rank 0 gets the workload itself;
+    other ranks get draws of the same distribution from seed + 1000 * rank."""
+    if w.ops == ("decode",):
+        return W.bitstream(w.n_seq, w.seed + 1000 * rank)
+    if rank == 0 or w.kind != "gaussian":
+        return W.sequences(w.name, n_limit=w.n_seq)
+    rng = np.random.default_rng(w.seed + 1000 * rank)
+    return rng.standard_normal((w.n_seq, W.SEQ_LEN)).astype(np.float32)
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Step time of the job = the slowest rank's (a timing collective only)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_ours(a) -> None:
     import torch
@@ -236,20 +259,13 @@ def run_ours(a) -> None:
         import dataclasses
         w = dataclasses.replace(w, n_seq=a.n_seq, rows=0, cols=0)
 
-    # ---- inputs (each rank its own batch: seed offset by rank) ----
+    # ---- inputs (each rank its own batch) ----
+    host = rank_batch(w, rank)
     if w.ops == ("decode",):
-        host = W.bitstream(w.n_seq, w.seed + 1000 * rank)
         x = torch.from_numpy(host.view(np.int32)).to(dev).view(torch.uint32)
-        h2d_bytes = host.nbytes
     else:
-        if rank == 0:
-            host = W.sequences(w.name, n_limit=w.n_seq)
-        else:
-            rng = np.random.default_rng(w.seed + 1000 * rank)
-            host = W.sequences(w.name, n_limit=w.n_seq) if w.kind != "gaussian" else \
-                rng.standard_normal((w.n_seq, W.SEQ_LEN)).astype(np.float32)
         x = torch.from_numpy(host).to(dev)
-        h2d_bytes = host.nbytes
+    h2d_bytes = host.nbytes
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
@@ -325,11 +341,7 @@ def run_ours(a) -> None:
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    mean_ms = sum(step_ms) / len(step_ms)
-    if dist is not None:
-        t = torch.tensor([mean_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_ms = float(t.item())
+    mean_ms = max_over_ranks(sum(step_ms) / len(step_ms), dist, dev)
 
     # ---- end to end through the public API with host buffers ----
     pinned = torch.from_numpy(host.view(np.int32) if w.ops == ("decode",) else host).pin_memory()
@@ -353,11 +365,7 @@ def run_ours(a) -> None:
         if i >= a.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
         d2h_bytes = sum(o.numel() * o.element_size() for o in outs)
-    e2e_mean = sum(e2e_ms) / len(e2e_ms)
-    if dist is not None:
-        t = torch.tensor([e2e_mean], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_mean = float(t.item())
+    e2e_mean = max_over_ranks(sum(e2e_ms) / len(e2e_ms), dist, dev)
 
     units = _weights_per_step(w) * world
     clocks = clk.summary()
