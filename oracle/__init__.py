@@ -69,21 +69,33 @@ def _lib():
     lib.orc_1mad_f32.restype = ctypes.c_float
     lib.orc_codebook_1mad_f64.argtypes = [I, P]
     lib.orc_codebook_1mad_f32.argtypes = [I, P]
-    lib.orc_viterbi_f32.argtypes = [I, I, I, P, P, P]
+    lib.orc_viterbi_f32.argtypes = [I, I, I, P, P, P, P]
     lib.orc_viterbi_f32.restype = ctypes.c_float
-    lib.orc_viterbi_f64.argtypes = [I, I, I, P, P, P, P]
+    lib.orc_viterbi_f64.argtypes = [I, I, I, P, P, P, P, P]
     lib.orc_viterbi_f64.restype = D
-    lib.orc_bcjr_f64.argtypes = [I, I, I, D, P, P, P, P, P, P]
+    lib.orc_bcjr_f64.argtypes = [I, I, I, D, P, P, P, P, P, P, P]
     lib.orc_bcjr_f64.restype = I
-    lib.orc_bcjr_vjp_f64.argtypes = [I, I, I, D, P, P, P, P, P]
+    lib.orc_bcjr_vjp_f64.argtypes = [I, I, I, D, P, P, P, P, P, P]
     lib.orc_bcjr_vjp_f64.restype = I
-    lib.orc_bruteforce_f64.argtypes = [I, I, I, D, P, P, P, P, P, P]
+    lib.orc_bruteforce_f64.argtypes = [I, I, I, D, P, P, P, P, P, P, P]
     lib.orc_bruteforce_f64.restype = ctypes.c_int64
     return lib
 
 
 def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _rows(D, n, T, dtype):
+    """Per-row curvature weights [n, T] (or None = all ones)."""
+    if D is None:
+        return None
+    D = np.ascontiguousarray(np.broadcast_to(np.asarray(D), (n, T)), dtype=dtype)
+    return D
+
+
+def _row_ptr(D, i):
+    return None if D is None else _ptr(D[i])
 
 
 # --------------------------------------------------------------------------
@@ -117,8 +129,9 @@ def codebook_f16(L: int) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Viterbi
 # --------------------------------------------------------------------------
-def viterbi_f32(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None):
-    """fp32-canonical Viterbi on each row of ``s`` [n, T].
+def viterbi_f32(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None, D=None):
+    """fp32-canonical Viterbi on each row of ``s`` [n, T] (optional per-weight
+    curvature ``D`` [n, T], step cost D_t (code - s_t)^2).
 
     Returns (states uint16 [n, T], mse float32 [n]) with mse = min cost / T
     computed in fp32."""
@@ -126,6 +139,7 @@ def viterbi_f32(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = Non
     if s.ndim == 1:
         s = s[None]
     n, T = s.shape
+    D = _rows(D, n, T, np.float32)
     code = codebook_f32(L) if code is None else np.ascontiguousarray(code, dtype=np.float32)
     states = np.empty((n, T), dtype=np.uint16)
     mse = np.empty(n, dtype=np.float32)
@@ -133,17 +147,18 @@ def viterbi_f32(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = Non
     for i in range(n):
         row = s[i]
         st = states[i]
-        cost = lib.orc_viterbi_f32(L, k, T, _ptr(row), _ptr(code), _ptr(st))
+        cost = lib.orc_viterbi_f32(L, k, T, _ptr(row), _row_ptr(D, i), _ptr(code), _ptr(st))
         mse[i] = np.float32(cost) / np.float32(T)
     return states, mse
 
 
-def viterbi_f64(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None):
+def viterbi_f64(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None, D=None):
     """fp64 Viterbi; returns (states [n, T], mse float64 [n], min_margin [n])."""
     s = np.ascontiguousarray(s, dtype=np.float64)
     if s.ndim == 1:
         s = s[None]
     n, T = s.shape
+    D = _rows(D, n, T, np.float64)
     code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
     states = np.empty((n, T), dtype=np.uint16)
     mse = np.empty(n, dtype=np.float64)
@@ -151,7 +166,8 @@ def viterbi_f64(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = Non
     lib = _lib()
     m = ctypes.c_double()
     for i in range(n):
-        cost = lib.orc_viterbi_f64(L, k, T, _ptr(s[i]), _ptr(code), _ptr(states[i]), ctypes.byref(m))
+        cost = lib.orc_viterbi_f64(L, k, T, _ptr(s[i]), _row_ptr(D, i), _ptr(code), _ptr(states[i]),
+                                   ctypes.byref(m))
         mse[i] = cost / T
         margin[i] = m.value
     return states, mse, margin
@@ -161,12 +177,13 @@ def viterbi_f64(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = Non
 # BCJR soft codeword and its vector-Jacobian product
 # --------------------------------------------------------------------------
 def bcjr_soft(s: np.ndarray, L: int, temp: float, k: int = 2, code: np.ndarray | None = None,
-              return_tables: bool = False):
+              return_tables: bool = False, D=None):
     """Soft codeword E_p[code(x_t)] and log Z per row of ``s`` (fp64)."""
     s = np.ascontiguousarray(s, dtype=np.float64)
     if s.ndim == 1:
         s = s[None]
     n, T = s.shape
+    D = _rows(D, n, T, np.float64)
     code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
     soft = np.empty((n, T), dtype=np.float64)
     logz = np.empty(n, dtype=np.float64)
@@ -179,8 +196,8 @@ def bcjr_soft(s: np.ndarray, L: int, temp: float, k: int = 2, code: np.ndarray |
             pa, pb = _ptr(al), _ptr(be)
         else:
             pa = pb = None
-        rc = lib.orc_bcjr_f64(L, k, T, float(temp), _ptr(s[i]), _ptr(code), _ptr(soft[i]),
-                              ctypes.byref(lz), pa, pb)
+        rc = lib.orc_bcjr_f64(L, k, T, float(temp), _ptr(s[i]), _row_ptr(D, i), _ptr(code),
+                              _ptr(soft[i]), ctypes.byref(lz), pa, pb)
         assert rc == 0
         logz[i] = lz.value
         if return_tables:
@@ -191,24 +208,26 @@ def bcjr_soft(s: np.ndarray, L: int, temp: float, k: int = 2, code: np.ndarray |
 
 
 def bcjr_vjp(s: np.ndarray, v: np.ndarray, L: int, temp: float, k: int = 2,
-             code: np.ndarray | None = None):
+             code: np.ndarray | None = None, D=None):
     """grad[u] = d/ds_u sum_t v_t soft_t per row (fp64); also returns soft."""
     s = np.ascontiguousarray(s, dtype=np.float64)
     v = np.ascontiguousarray(v, dtype=np.float64)
     if s.ndim == 1:
         s = s[None]; v = v[None]
     n, T = s.shape
+    D = _rows(D, n, T, np.float64)
     code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
     grad = np.empty((n, T)); soft = np.empty((n, T))
     lib = _lib()
     for i in range(n):
-        rc = lib.orc_bcjr_vjp_f64(L, k, T, float(temp), _ptr(s[i]), _ptr(code), _ptr(v[i]),
-                                  _ptr(grad[i]), _ptr(soft[i]))
+        rc = lib.orc_bcjr_vjp_f64(L, k, T, float(temp), _ptr(s[i]), _row_ptr(D, i), _ptr(code),
+                                  _ptr(v[i]), _ptr(grad[i]), _ptr(soft[i]))
         assert rc == 0
     return grad, soft
 
 
-def bruteforce(s: np.ndarray, L: int, temp: float, k: int = 2, code: np.ndarray | None = None):
+def bruteforce(s: np.ndarray, L: int, temp: float, k: int = 2, code: np.ndarray | None = None,
+               D=None):
     """Enumerate every walk of one sequence ``s`` [T] (tiny cases only).
 
     Returns dict(min_energy, log_z, soft [T], second [T, T], walks)."""
@@ -217,8 +236,10 @@ def bruteforce(s: np.ndarray, L: int, temp: float, k: int = 2, code: np.ndarray 
     code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
     soft = np.empty(T); second = np.empty((T, T))
     emin = ctypes.c_double(); lz = ctypes.c_double()
-    W = _lib().orc_bruteforce_f64(L, k, T, float(temp), _ptr(s), _ptr(code), ctypes.byref(emin),
-                                  ctypes.byref(lz), _ptr(soft), _ptr(second))
+    Dr = None if D is None else np.ascontiguousarray(np.broadcast_to(np.asarray(D), (T,)), dtype=np.float64)
+    W = _lib().orc_bruteforce_f64(L, k, T, float(temp), _ptr(s), None if Dr is None else _ptr(Dr),
+                                  _ptr(code), ctypes.byref(emin), ctypes.byref(lz), _ptr(soft),
+                                  _ptr(second))
     if W < 0:
         raise ValueError("too many walks for brute force")
     return dict(min_energy=emin.value, log_z=lz.value, soft=soft, second=second, walks=W)

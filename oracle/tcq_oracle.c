@@ -22,6 +22,10 @@
  *   pred_a(j) = (j >> k) | (a << (L-k)),  a in [0, 2^k)     [QTIP-blog, trellis]
  *   succ_b(i) = ((i << k) | b) & (2^L - 1), b in [0, 2^k)
  *   Free start: every state may begin a walk with cost (code - s_0)^2.
+ *   D      optional per-weight curvature (NULL = all ones).  [XOR-Trellis
+ *          explainer, "Cliff edges": the search multiplies each step's squared
+ *          error by that weight's D; states and decoder are unchanged.]  The
+ *          step cost becomes D_t (code - s_t)^2.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off (no fast-math), so
  * every float/double operation below is one IEEE-754 operation, correctly
@@ -69,12 +73,13 @@ void orc_codebook_1mad_f32(int L, float *out)
 /* Viterbi, fp32 canonical arithmetic   [QTIP-blog, trellis section]         */
 /*   cost_0(j) = (code_j - s_0)^2                                            */
 /*   cost_t(j) = min_a cost_{t-1}(pred_a(j)) + (code_j - s_t)^2              */
-/* Each fp32 step is d = code - s, e = d * d, cost = best + e, every one     */
-/* rounded to fp32 (no fused multiply-add).  The argmin over a keeps the     */
+/* Each fp32 step is d = code - s, e = d * d (then e = e * D_t when weights */
+/* are given), cost = best + e, every one rounded to fp32 (no fused          */
+/* multiply-add).  The argmin over a keeps the     */
 /* first (lowest a) minimum, like numpy's argmin; the final argmin keeps the */
 /* lowest state.  Returns the minimum total cost; states[0..T-1] the walk.   */
 /* ------------------------------------------------------------------------ */
-float orc_viterbi_f32(int L, int k, int T, const float *s, const float *code,
+float orc_viterbi_f32(int L, int k, int T, const float *s, const float *D, const float *code,
                       uint16_t *states)
 {
     const int N = 1 << L, A = 1 << k;
@@ -84,7 +89,8 @@ float orc_viterbi_f32(int L, int k, int T, const float *s, const float *code,
 
     for (int j = 0; j < N; ++j) {
         float d = code[j] - s[0];
-        cost[j] = d * d;
+        float e = d * d;
+        cost[j] = D ? e * D[0] : e;
     }
     for (int t = 1; t < T; ++t) {
         for (int j = 0; j < N; ++j) {
@@ -96,6 +102,7 @@ float orc_viterbi_f32(int L, int k, int T, const float *s, const float *code,
             }
             float d = code[j] - s[t];
             float e = d * d;
+            if (D) e = e * D[t];
             next[j] = best + e;
             back[(size_t)t * N + j] = bestp;
         }
@@ -130,7 +137,7 @@ static double rel_gap(double best, double second)
     return (second - best) / den;
 }
 
-double orc_viterbi_f64(int L, int k, int T, const double *s, const double *code,
+double orc_viterbi_f64(int L, int k, int T, const double *s, const double *D, const double *code,
                        uint16_t *states, double *min_margin)
 {
     const int N = 1 << L, A = 1 << k;
@@ -139,7 +146,7 @@ double orc_viterbi_f64(int L, int k, int T, const double *s, const double *code,
 
     for (int j = 0; j < N; ++j) {
         double d = code[j] - s[0];
-        cost[j] = d * d;
+        cost[j] = (D ? D[0] : 1.0) * d * d;
     }
     for (int t = 1; t < T; ++t) {
         const double *prev = cost + (size_t)(t - 1) * N;
@@ -152,7 +159,7 @@ double orc_viterbi_f64(int L, int k, int T, const double *s, const double *code,
                 if (bestp < 0 || prev[p] < best) { best = prev[p]; bestp = p; }
             }
             double d = code[j] - s[t];
-            cur[j] = best + d * d;
+            cur[j] = best + (D ? D[t] : 1.0) * d * d;
             back[(size_t)t * N + j] = bestp;
         }
     }
@@ -211,43 +218,44 @@ static double lse_array(const double *v, int n)
     return m + log(acc);
 }
 
-static double emis(const double *code, const double *s, int t, int j)
+static double emis(const double *code, const double *s, const double *D, int t, int j)
 {
     double d = code[j] - s[t];
-    return d * d;
+    return (D ? D[t] : 1.0) * d * d;
 }
 
-static void bcjr_tables(int L, int k, int T, double temp, const double *s,
+static void bcjr_tables(int L, int k, int T, double temp, const double *s, const double *D,
                         const double *code, double *alpha, double *beta)
 {
     const int N = 1 << L, A = 1 << k;
     double tmp[64];
-    for (int j = 0; j < N; ++j) alpha[j] = -emis(code, s, 0, j) / temp;
+    for (int j = 0; j < N; ++j) alpha[j] = -emis(code, s, D, 0, j) / temp;
     for (int t = 1; t < T; ++t)
         for (int j = 0; j < N; ++j) {
             for (int a = 0; a < A; ++a)
                 tmp[a] = alpha[(size_t)(t - 1) * N + ((j >> k) | (a << (L - k)))];
-            alpha[(size_t)t * N + j] = lse_array(tmp, A) - emis(code, s, t, j) / temp;
+            alpha[(size_t)t * N + j] = lse_array(tmp, A) - emis(code, s, D, t, j) / temp;
         }
     for (int i = 0; i < N; ++i) beta[(size_t)(T - 1) * N + i] = 0.0;
     for (int t = T - 2; t >= 0; --t)
         for (int i = 0; i < N; ++i) {
             for (int b = 0; b < A; ++b) {
                 int nx = ((i << k) | b) & (N - 1);
-                tmp[b] = beta[(size_t)(t + 1) * N + nx] - emis(code, s, t + 1, nx) / temp;
+                tmp[b] = beta[(size_t)(t + 1) * N + nx] - emis(code, s, D, t + 1, nx) / temp;
             }
             beta[(size_t)t * N + i] = lse_array(tmp, A);
         }
 }
 
-int orc_bcjr_f64(int L, int k, int T, double temp, const double *s, const double *code,
-                 double *soft, double *log_z, double *alpha_out, double *beta_out)
+int orc_bcjr_f64(int L, int k, int T, double temp, const double *s, const double *D,
+                 const double *code, double *soft, double *log_z, double *alpha_out,
+                 double *beta_out)
 {
     const int N = 1 << L;
     if (k > 6) return -1;
     double *alpha = alpha_out ? alpha_out : (double *)malloc(sizeof(double) * (size_t)T * N);
     double *beta = beta_out ? beta_out : (double *)malloc(sizeof(double) * (size_t)T * N);
-    bcjr_tables(L, k, T, temp, s, code, alpha, beta);
+    bcjr_tables(L, k, T, temp, s, D, code, alpha, beta);
     double lz = lse_array(alpha + (size_t)(T - 1) * N, N);
     for (int t = 0; t < T; ++t) {
         double acc = 0.0;
@@ -265,8 +273,8 @@ int orc_bcjr_f64(int L, int k, int T, double temp, const double *s, const double
 /* Vector-Jacobian product of the soft codeword, fp64.                      */
 /* grad[u] = d/ds_u sum_t v_t soft_t.  Differentiating the Boltzmann         */
 /* expectation (E is a sum of squares, so dE/ds_u = -2(code[x_u] - s_u)):   */
-/*   d soft_t / d s_u = (2/temp) Cov_p(code[x_t], code[x_u]),               */
-/*   grad[u] = (2/temp) (E_p[F code[x_u]] - E_p[F] soft_u),                 */
+/*   d soft_t / d s_u = (2 D_u/temp) Cov_p(code[x_t], code[x_u]),           */
+/*   grad[u] = (2 D_u/temp) (E_p[F code[x_u]] - E_p[F] soft_u),             */
 /*   F = sum_t v_t code[x_t].                                               */
 /* E_p[F | x_u = j] is split by the Markov property into the prefix part    */
 /* phi_u(j) (which includes v_u code_j) and the suffix part psi_u(j):       */
@@ -279,8 +287,8 @@ int orc_bcjr_f64(int L, int k, int T, double temp, const double *s, const double
 /*   E_p[F code[x_u]] = sum_j gamma_u(j) code_j (phi_u(j) + psi_u(j)).      */
 /* soft_out (nullable) receives the soft codeword as a by-product.          */
 /* ------------------------------------------------------------------------ */
-int orc_bcjr_vjp_f64(int L, int k, int T, double temp, const double *s, const double *code,
-                     const double *v, double *grad, double *soft_out)
+int orc_bcjr_vjp_f64(int L, int k, int T, double temp, const double *s, const double *D,
+                     const double *code, const double *v, double *grad, double *soft_out)
 {
     const int N = 1 << L, A = 1 << k;
     if (k > 6) return -1;
@@ -290,7 +298,7 @@ int orc_bcjr_vjp_f64(int L, int k, int T, double temp, const double *s, const do
     double *psi = (double *)malloc(sizeof(double) * (size_t)T * N);
     double *soft = (double *)malloc(sizeof(double) * (size_t)T);
     double tmp[64];
-    bcjr_tables(L, k, T, temp, s, code, alpha, beta);
+    bcjr_tables(L, k, T, temp, s, D, code, alpha, beta);
     double lz = lse_array(alpha + (size_t)(T - 1) * N, N);
 
     for (int j = 0; j < N; ++j) phi[j] = v[0] * code[j];
@@ -308,7 +316,7 @@ int orc_bcjr_vjp_f64(int L, int k, int T, double temp, const double *s, const do
         for (int i = 0; i < N; ++i) {
             for (int b = 0; b < A; ++b) {
                 int nx = ((i << k) | b) & (N - 1);
-                tmp[b] = beta[(size_t)(t + 1) * N + nx] - emis(code, s, t + 1, nx) / temp;
+                tmp[b] = beta[(size_t)(t + 1) * N + nx] - emis(code, s, D, t + 1, nx) / temp;
             }
             double m = lse_array(tmp, A), acc = 0.0;
             for (int b = 0; b < A; ++b) {
@@ -331,7 +339,7 @@ int orc_bcjr_vjp_f64(int L, int k, int T, double temp, const double *s, const do
             double g = exp(alpha[(size_t)u * N + j] + beta[(size_t)u * N + j] - lz);
             acc += g * code[j] * (phi[(size_t)u * N + j] + psi[(size_t)u * N + j]);
         }
-        grad[u] = (2.0 / temp) * (acc - ef * soft[u]);
+        grad[u] = (2.0 * (D ? D[u] : 1.0) / temp) * (acc - ef * soft[u]);
     }
     if (soft_out) memcpy(soft_out, soft, sizeof(double) * (size_t)T);
     free(alpha); free(beta); free(phi); free(psi); free(soft);
@@ -347,7 +355,7 @@ int orc_bcjr_vjp_f64(int L, int k, int T, double temp, const double *s, const do
 /* second[t*T+u] = E[code[x_t] code[x_u]].  Returns the walk count, or -1   */
 /* if it would exceed 2^24.                                                 */
 /* ------------------------------------------------------------------------ */
-int64_t orc_bruteforce_f64(int L, int k, int T, double temp, const double *s,
+int64_t orc_bruteforce_f64(int L, int k, int T, double temp, const double *s, const double *D,
                            const double *code, double *min_energy, double *log_z,
                            double *soft, double *second)
 {
@@ -376,7 +384,7 @@ int64_t orc_bruteforce_f64(int L, int k, int T, double temp, const double *s,
                 }
                 xs[t] = (int)x;
                 double d = code[x] - s[t];
-                E += d * d;
+                E += (D ? D[t] : 1.0) * d * d;
             }
             if (pass == 0) {
                 if (E < emin) emin = E;

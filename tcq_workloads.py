@@ -16,6 +16,8 @@ Workloads (the pages' shapes and distributions):
   * student_t:  2048x8192 Student-t (nu = 5) rescaled to unit variance, tiled
   * bitstream:  uniform random 32-bit words, 16 per sequence = a tail-biting
                 2-bit stream of 256 weights (QTIP blog, "Tail-biting")
+  * curvature:  per-weight positive weights D, log-uniform on [0.1, 10], for the
+                curvature-weighted search (XOR-Trellis explainer, "Cliff edges")
 """
 from __future__ import annotations
 
@@ -90,6 +92,14 @@ def rht_block(seed: int, n: int = 1024) -> np.ndarray:
 def student_t_block(seed: int, rows: int = 2048, cols: int = 8192, nu: float = 5.0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     return (rng.standard_t(nu, (rows, cols)) * np.sqrt((nu - 2.0) / nu)).astype(np.float32)
+
+
+def curvature(n_seq: int, seed: int, seq_len: int = SEQ_LEN, lo: float = 0.1,
+              hi: float = 10.0) -> np.ndarray:
+    """Synthetic per-weight curvature D > 0, log-uniform on [lo, hi] (stands in
+    for the LDL diagonal of a layer Hessian, which needs a model and data)."""
+    rng = np.random.default_rng(seed)
+    return np.exp(rng.uniform(np.log(lo), np.log(hi), (n_seq, seq_len))).astype(np.float32)
 
 
 def bitstream(n_seq: int, seed: int, words: int = 16) -> np.ndarray:
