@@ -58,7 +58,8 @@ def _metric_for(w: W.Workload) -> str:
         parts.append("BCJR soft" + (f" x{len(w.temps)} temps" if len(w.temps) > 1 else ""))
     if "bcjr_grad" in w.ops:
         parts.append("BCJR gradient")
-    return "weights quantized/sec (" + " + ".join(parts) + ")"
+    tail = ", curvature-weighted" if w.curv_seed else ""
+    return "weights quantized/sec (" + " + ".join(parts) + tail + ")"
 
 
 def _weights_per_step(w: W.Workload) -> int:
@@ -130,15 +131,15 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle
-def _oracle_step(w: W.Workload, s: np.ndarray) -> None:
+def _oracle_step(w: W.Workload, s: np.ndarray, D=None) -> None:
     import oracle
     if "viterbi" in w.ops:
-        oracle.viterbi_f32(s, w.L)
+        oracle.viterbi_f32(s, w.L, D=D)
     for temp in w.temps:
         if "bcjr_grad" in w.ops and temp == w.temps[0]:
-            oracle.bcjr_vjp(s, np.ones_like(s, dtype=np.float64), w.L, temp)  # also yields soft
+            oracle.bcjr_vjp(s, np.ones_like(s, dtype=np.float64), w.L, temp, D=D)  # also yields soft
         elif "bcjr" in w.ops:
-            oracle.bcjr_soft(s, w.L, temp)
+            oracle.bcjr_soft(s, w.L, temp, D=D)
 
 
 def _oracle_decode_step(bits: np.ndarray, w: W.Workload) -> None:
@@ -159,8 +160,9 @@ def cpu_baseline(w: W.Workload, budget_s: float = 12.0) -> dict:
             n_done += chunk
     else:
         s = W.sequences(w.name, n_limit=min(w.n_seq, 256))
+        D = W.weights(w.name, n_limit=min(w.n_seq, 256))
         while time.perf_counter() - t0 < budget_s and n_done < s.shape[0]:
-            _oracle_step(w, s[n_done:n_done + 1])
+            _oracle_step(w, s[n_done:n_done + 1], None if D is None else D[n_done:n_done + 1])
             n_done += 1
     dt = time.perf_counter() - t0
     return {"value": n_done * W.SEQ_LEN / dt, "unit": "weights/s", "cores": 1, "kind": "oracle",
@@ -176,20 +178,23 @@ def run_reference(a) -> None:
     import oracle
     oracle.build()
     per_step = 4 if w.ops != ("decode",) else 1024        # sequences per bounded step
+    wts = None
     if w.ops == ("decode",):
         data = W.streams(w.name)[: per_step * (a.steps + a.warmup)]
     else:
         data = W.sequences(w.name, n_limit=min(w.n_seq, per_step * (a.steps + a.warmup)))
+        wts = W.weights(w.name, n_limit=min(w.n_seq, per_step * (a.steps + a.warmup)))
     pos = 0
     times = []
     for i in range(a.warmup + a.steps):
-        chunk = data[pos % data.shape[0]: pos % data.shape[0] + per_step]
+        lo = pos % data.shape[0]
+        chunk = data[lo: lo + per_step]
         pos += per_step
         t0 = time.perf_counter()
         if w.ops == ("decode",):
             _oracle_decode_step(chunk, w)
         else:
-            _oracle_step(w, chunk)
+            _oracle_step(w, chunk, None if wts is None else wts[lo: lo + per_step])
         if i >= a.warmup:
             times.append(time.perf_counter() - t0)
     step_s = sum(times) / len(times)
@@ -277,6 +282,8 @@ def run_ours(a) -> None:
     if "bcjr_grad" in w.ops:
         ws_g = torch.empty(tcq.bcjr_workspace_size(w.L, 256, w.n_seq, True), dtype=torch.uint8, device=dev)
     ones = torch.ones((w.n_seq, W.SEQ_LEN), dtype=torch.float32, device=dev)
+    wts = W.weights(w.name, n_limit=w.n_seq)
+    Dd = torch.from_numpy(wts).to(dev) if wts is not None else None
 
     kern_ms: dict[str, list[float]] = {}
     launches_per_step = 0
@@ -302,17 +309,17 @@ def run_ours(a) -> None:
         else:
             mark("start")
             if "viterbi" in w.ops:
-                st, mse = tcq.viterbi_encode(inp, w.L, ws_v)
+                st, mse = tcq.viterbi_encode(inp, w.L, ws_v, D=Dd)
                 mark("viterbi")
                 n_launch += 2
                 outs += [st, mse]
             for i, temp in enumerate(w.temps):
-                soft, lz = tcq.bcjr_soft(inp, w.L, temp, ws_b)
+                soft, lz = tcq.bcjr_soft(inp, w.L, temp, ws_b, D=Dd)
                 mark(f"bcjr_soft_t{temp:g}")
                 n_launch += 1
                 outs += [soft, lz]
                 if "bcjr_grad" in w.ops and i == 0:
-                    g = tcq.bcjr_soft_backward(inp, w.L, temp, soft, ones, ws_g)
+                    g = tcq.bcjr_soft_backward(inp, w.L, temp, soft, ones, ws_g, D=Dd)
                     mark(f"bcjr_vjp_t{temp:g}")
                     n_launch += 1
                     outs.append(g)

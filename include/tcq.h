@@ -108,6 +108,11 @@ TCQ_API size_t tcq_stream_words(const tcq_trellis_t *trellis, int layout);
  * to the lowest predecessor digit a, and the final argmin to the lowest state.
  *
  *   s          [n_seq][seq_len] fp32 targets (input).
+ *   D          [n_seq][seq_len] fp32 per-weight curvature, or NULL for all
+ *              ones [XOR-Trellis explainer, "Cliff edges": the search
+ *              multiplies each step's squared error by that weight's D].  The
+ *              step cost becomes e = d*d, then e*D_t, each rounded on its own.
+ *              D must be >= 0 and finite (other values: unspecified walks).
  *   states     [n_seq][seq_len] uint16: the chosen walk, state (L-bit window)
  *              of every weight (output).
  *   mse        [n_seq] fp32: minimum total cost / seq_len (output).
@@ -117,9 +122,9 @@ TCQ_API size_t tcq_stream_words(const tcq_trellis_t *trellis, int layout);
  * ------------------------------------------------------------------------ */
 TCQ_API size_t tcq_viterbi_workspace_size(const tcq_trellis_t *trellis, int64_t n_seq);
 
-TCQ_API tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *trellis, const float *s, int64_t n_seq,
-                                uint16_t *states, float *mse, void *ws, size_t ws_bytes,
-                                void *stream);
+TCQ_API tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *trellis, const float *s,
+                                        const float *D, int64_t n_seq, uint16_t *states,
+                                        float *mse, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * Allocation-free Viterbi encode (the pages have no counterpart: this is a
@@ -158,6 +163,8 @@ TCQ_API tcq_status_t tcq_viterbi_encode_noalloc(const tcq_trellis_t *trellis, co
  * fp32, log domain (base 2 inside), renormalised every step.
  *
  *   s        [n_seq][seq_len] fp32 (input); temp > 0 and finite.
+ *   D        [n_seq][seq_len] fp32 curvature weights (>= 0) or NULL: the
+ *            energy becomes sum_t D_t (code(x_t) - s_t)^2.
  *   soft     [n_seq][seq_len] fp32 (output).
  *   log_z    [n_seq] fp32 (output, may be NULL).
  *   ws       device workspace of at least tcq_bcjr_workspace_size(.., 0)
@@ -165,15 +172,16 @@ TCQ_API tcq_status_t tcq_viterbi_encode_noalloc(const tcq_trellis_t *trellis, co
  * ------------------------------------------------------------------------ */
 TCQ_API size_t tcq_bcjr_workspace_size(const tcq_trellis_t *trellis, int64_t n_seq, int with_grad);
 
-TCQ_API tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *trellis, const float *s, int64_t n_seq,
-                           float temp, float *soft, float *log_z, void *ws, size_t ws_bytes,
-                           void *stream);
+TCQ_API tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *trellis, const float *s, const float *D,
+                                   int64_t n_seq, float temp, float *soft, float *log_z,
+                                   void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * Vector-Jacobian product of the soft codeword [BCJR: the relaxed code is a
  * smooth function of the targets]:
  *   grad_s[u] = sum_t grad_soft[t] d soft[t] / d s[u]
- *             = (2/temp) Cov_p( sum_t grad_soft[t] code(x_t), code(x_u) ).
+ *             = (2 D_u/temp) Cov_p( sum_t grad_soft[t] code(x_t), code(x_u) )
+ *   (D_u = 1 when D is NULL; D as in tcq_bcjr_soft).
  *   soft       [n_seq][seq_len] the forward output of tcq_bcjr_soft for the
  *              same s and temp (input; used to centre the covariance).
  *   grad_soft  [n_seq][seq_len] fp32 (input), grad_s [n_seq][seq_len] (output).
@@ -181,9 +189,10 @@ TCQ_API tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *trellis, const float *s,
  * L = 16 returns TCQ_ERR_UNSUPPORTED.
  * ------------------------------------------------------------------------ */
 TCQ_API tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *trellis, const float *s,
-                                    int64_t n_seq, float temp, const float *soft,
-                                    const float *grad_soft, float *grad_s, void *ws,
-                                    size_t ws_bytes, void *stream);
+                                            const float *D, int64_t n_seq, float temp,
+                                            const float *soft, const float *grad_soft,
+                                            float *grad_s, void *ws, size_t ws_bytes,
+                                            void *stream);
 
 /* ------------------------------------------------------------------------
  * Pack walks into bitstreams [QTIP, trellis: the state is a sliding L-bit

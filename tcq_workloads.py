@@ -39,6 +39,7 @@ class Workload:
     rows: int = 0
     cols: int = 0
     ops: tuple = field(default=())
+    curv_seed: int = 0             # > 0: curvature-weighted search, D drawn from this seed
 
 
 # The five workloads, seeds 1..5.
@@ -53,7 +54,20 @@ WORKLOADS = {
                                        (1.0, 0.1, 0.01), 2048, 8192, ops=("bcjr",)),
     "l16_decode_8192sq": Workload("l16_decode_8192sq", 16, 262144, "bitstream", 5, (),
                                   8192, 8192, ops=("decode",)),
+    # curvature-weighted variant of the L=12 workload (XOR-Trellis explainer,
+    # "Cliff edges"); D log-uniform on [0.1, 10] from seed 6
+    "l12_curv1024": Workload("l12_curv1024", 12, 1024, "gaussian", 2, (0.05,),
+                             ops=("viterbi", "bcjr", "bcjr_grad"), curv_seed=6),
 }
+
+
+def weights(name: str, n_limit: int | None = None) -> np.ndarray | None:
+    """Curvature weights [n, 256] of a weighted workload (None if unweighted)."""
+    w = WORKLOADS[name]
+    if not w.curv_seed:
+        return None
+    out = curvature(w.n_seq, w.curv_seed)
+    return out if n_limit is None else np.ascontiguousarray(out[:n_limit])
 
 
 def tiles_to_sequences(m: np.ndarray) -> np.ndarray:

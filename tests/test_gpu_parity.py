@@ -273,3 +273,51 @@ def test_vjp_random_cotangent_and_autograd(tcq):
     rg, _ = oracle.bcjr_vjp(s, v, 8, 0.2)
     for i in range(5):
         assert np.abs(g[i] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+
+
+# ---------------------------------------------------------------- curvature-weighted search
+@pytest.mark.parametrize("L,n", [(8, 64), (12, 256), (16, 6)])
+def test_weighted_viterbi_bit_exact(tcq, L, n):
+    s = W.gaussian(n, 600 + L)
+    D = W.curvature(n, 700 + L)
+    st, mse = tcq.viterbi_encode(_dev(s), L, D=_dev(D))
+    torch.cuda.synchronize()
+    st = st.cpu().view(torch.int16).numpy().view(np.uint16)
+    rst, rmse = oracle.viterbi_f32(s, L, D=D)
+    assert np.array_equal(st, rst)
+    assert np.array_equal(mse.cpu().numpy().view(np.uint32), rmse.view(np.uint32))
+
+
+def test_weighted_full_workload(tcq):
+    s = W.sequences("l12_curv1024")
+    D = W.weights("l12_curv1024")
+    sd, Dd = _dev(s), _dev(D)
+    st, mse = tcq.viterbi_encode(sd, 12, D=Dd)
+    rst, rmse = oracle.viterbi_f32(s, 12, D=D)
+    assert np.array_equal(st.cpu().view(torch.int16).numpy().view(np.uint16), rst)
+    assert np.array_equal(mse.cpu().numpy().view(np.uint32), rmse.view(np.uint32))
+    soft, lz = tcq.bcjr_soft(sd, 12, 0.05, D=Dd)
+    g = tcq.bcjr_soft_backward(sd, 12, 0.05, soft, torch.ones_like(sd), D=Dd)
+    torch.cuda.synchronize()
+    idx = np.random.default_rng(8).choice(1024, 10, replace=False)
+    rg, rsoft = oracle.bcjr_vjp(s[idx], np.ones((10, 256)), 12, 0.05, D=D[idx])
+    assert np.abs(soft.cpu().numpy()[idx] - rsoft).max() <= SOFT_ATOL
+    gn = g.cpu().numpy()[idx]
+    for i in range(10):
+        assert np.abs(gn[i] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+
+
+@pytest.mark.parametrize("L", [8, 16])
+def test_weighted_bcjr(tcq, L):
+    s = W.gaussian(3, 800 + L, seq_len=64)
+    D = W.curvature(3, 900 + L, seq_len=64)
+    soft, lz = _bcjr_gpu_w(tcq, s, L, 0.2, D)
+    rsoft, rlz = oracle.bcjr_soft(s, L, 0.2, D=D)
+    assert np.abs(soft - rsoft).max() <= SOFT_ATOL
+    assert np.all(np.abs(lz - rlz) <= 1e-5 * np.abs(rlz) + 1e-4)
+
+
+def _bcjr_gpu_w(tcq, s, L, temp, D):
+    soft, lz = tcq.bcjr_soft(_dev(s), L, temp, D=_dev(D))
+    torch.cuda.synchronize()
+    return soft.cpu().numpy(), lz.cpu().numpy()

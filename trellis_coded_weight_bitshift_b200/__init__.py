@@ -44,7 +44,7 @@ def _stream() -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+def _ptr(t: "torch.Tensor | None") -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
 
 
@@ -66,10 +66,22 @@ def bcjr_workspace_size(L: int, seq_len: int, n_seq: int, with_grad: bool = Fals
                                              int(bool(with_grad))))
 
 
-def viterbi_encode(s: torch.Tensor, L: int, workspace: torch.Tensor | None = None):
+def _weights(D: torch.Tensor | None, s: torch.Tensor) -> torch.Tensor | None:
+    if D is None:
+        return None
+    _require_cuda(D)
+    if D.shape != s.shape or D.dtype != torch.float32:
+        raise ValueError("D must be a float32 tensor shaped like s")
+    return D
+
+
+def viterbi_encode(s: torch.Tensor, L: int, workspace: torch.Tensor | None = None,
+                   D: torch.Tensor | None = None):
     """Min-MSE walk of every row of ``s`` [n, T] (fp32) on the (L, 2, 1)
-    bitshift trellis with the 1MAD code; returns (states uint16, mse fp32)."""
+    bitshift trellis with the 1MAD code; returns (states uint16, mse fp32).
+    ``D`` (optional, same shape) weights each step's squared error."""
     _require_cuda(s)
+    D = _weights(D, s)
     if s.dtype != torch.float32 or s.dim() != 2:
         raise ValueError("s must be a 2-D float32 tensor [n_seq, seq_len]")
     n, T = s.shape
@@ -78,15 +90,17 @@ def viterbi_encode(s: torch.Tensor, L: int, workspace: torch.Tensor | None = Non
     mse = torch.empty((n,), dtype=torch.float32, device=s.device)
     need = int(lib().tcq_viterbi_workspace_size(ctypes.byref(tr), n))
     ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
-    check(lib().tcq_viterbi_encode(ctypes.byref(tr), _ptr(s), n, _ptr(states), _ptr(mse), _ptr(ws),
-                                   ws.numel(), _stream()), "tcq_viterbi_encode")
+    check(lib().tcq_viterbi_encode(ctypes.byref(tr), _ptr(s), _ptr(D), n, _ptr(states), _ptr(mse),
+                                   _ptr(ws), ws.numel(), _stream()), "tcq_viterbi_encode")
     return states, mse
 
 
-def bcjr_soft(s: torch.Tensor, L: int, temp: float, workspace: torch.Tensor | None = None):
+def bcjr_soft(s: torch.Tensor, L: int, temp: float, workspace: torch.Tensor | None = None,
+              D: torch.Tensor | None = None):
     """Soft codeword (Boltzmann expectation of the code at temperature
     ``temp``) of every row of ``s``; returns (soft fp32 [n,T], log_z fp32 [n])."""
     _require_cuda(s)
+    D = _weights(D, s)
     if s.dtype != torch.float32 or s.dim() != 2:
         raise ValueError("s must be a 2-D float32 tensor [n_seq, seq_len]")
     n, T = s.shape
@@ -95,15 +109,17 @@ def bcjr_soft(s: torch.Tensor, L: int, temp: float, workspace: torch.Tensor | No
     logz = torch.empty((n,), dtype=torch.float32, device=s.device)
     need = int(lib().tcq_bcjr_workspace_size(ctypes.byref(tr), n, 0))
     ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
-    check(lib().tcq_bcjr_soft(ctypes.byref(tr), _ptr(s), n, float(temp), _ptr(soft), _ptr(logz),
-                              _ptr(ws), ws.numel(), _stream()), "tcq_bcjr_soft")
+    check(lib().tcq_bcjr_soft(ctypes.byref(tr), _ptr(s), _ptr(D), n, float(temp), _ptr(soft),
+                              _ptr(logz), _ptr(ws), ws.numel(), _stream()), "tcq_bcjr_soft")
     return soft, logz
 
 
 def bcjr_soft_backward(s: torch.Tensor, L: int, temp: float, soft: torch.Tensor,
-                       grad_soft: torch.Tensor, workspace: torch.Tensor | None = None):
+                       grad_soft: torch.Tensor, workspace: torch.Tensor | None = None,
+                       D: torch.Tensor | None = None):
     """Vector-Jacobian product: grad_s[u] = sum_t grad_soft[t] d soft[t] / d s[u]."""
     _require_cuda(s, soft, grad_soft)
+    D = _weights(D, s)
     if s.shape != soft.shape or s.shape != grad_soft.shape:
         raise ValueError("s, soft and grad_soft must have the same shape")
     n, T = s.shape
@@ -111,26 +127,26 @@ def bcjr_soft_backward(s: torch.Tensor, L: int, temp: float, soft: torch.Tensor,
     grad = torch.empty_like(s)
     need = int(lib().tcq_bcjr_workspace_size(ctypes.byref(tr), n, 1))
     ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
-    check(lib().tcq_bcjr_soft_backward(ctypes.byref(tr), _ptr(s), n, float(temp), _ptr(soft),
-                                       _ptr(grad_soft), _ptr(grad), _ptr(ws), ws.numel(),
-                                       _stream()), "tcq_bcjr_soft_backward")
+    check(lib().tcq_bcjr_soft_backward(ctypes.byref(tr), _ptr(s), _ptr(D), n, float(temp),
+                                       _ptr(soft), _ptr(grad_soft), _ptr(grad), _ptr(ws),
+                                       ws.numel(), _stream()), "tcq_bcjr_soft_backward")
     return grad
 
 
 class BcjrSoft(torch.autograd.Function):
-    """soft = BcjrSoft.apply(s, L, temp): differentiable soft codeword."""
+    """soft = BcjrSoft.apply(s, L, temp[, D]): differentiable soft codeword."""
 
     @staticmethod
-    def forward(ctx, s, L, temp):
-        soft, _ = bcjr_soft(s, L, temp)
-        ctx.save_for_backward(s, soft)
+    def forward(ctx, s, L, temp, D=None):
+        soft, _ = bcjr_soft(s, L, temp, D=D)
+        ctx.save_for_backward(s, soft, D)
         ctx.L, ctx.temp = L, temp
         return soft
 
     @staticmethod
     def backward(ctx, g):
-        s, soft = ctx.saved_tensors
-        return bcjr_soft_backward(s, ctx.L, ctx.temp, soft, g.contiguous()), None, None
+        s, soft, D = ctx.saved_tensors
+        return bcjr_soft_backward(s, ctx.L, ctx.temp, soft, g.contiguous(), D=D), None, None, None
 
 
 def pack_states(states: torch.Tensor, L: int, layout: int = FREE_START) -> torch.Tensor:
@@ -159,6 +175,11 @@ def decode(bits: torch.Tensor, L: int, seq_len: int = 256, layout: int = TAILBIT
         raise ValueError("bits must be a 2-D uint32 tensor")
     n = bits.shape[0]
     tr = trellis(L, seq_len)
+    words = int(lib().tcq_stream_words(ctypes.byref(tr), int(layout)))
+    if words == 0:
+        raise TcqError(_abi.TCQ_ERR_UNSUPPORTED, "tcq_stream_words")
+    if bits.shape[1] != words:
+        raise ValueError(f"bits must have {words} words per sequence for this trellis and layout")
     if out is None:
         shape = (rows, cols) if out_layout == OUT_TILE16 else (n, seq_len)
         out = torch.empty(shape, dtype=torch.float16, device=bits.device)

@@ -56,15 +56,15 @@ def lib() -> ctypes.CDLL:
     L.tcq_viterbi_workspace_size.restype = SZ
     L.tcq_viterbi_workspace_size.argtypes = [TP, I64]
     L.tcq_viterbi_encode.restype = I
-    L.tcq_viterbi_encode.argtypes = [TP, P, I64, P, P, P, SZ, P]
+    L.tcq_viterbi_encode.argtypes = [TP, P, P, I64, P, P, P, SZ, P]
     L.tcq_viterbi_encode_noalloc.restype = I
     L.tcq_viterbi_encode_noalloc.argtypes = [TP, P, I64, P, P, P]
     L.tcq_bcjr_workspace_size.restype = SZ
     L.tcq_bcjr_workspace_size.argtypes = [TP, I64, I]
     L.tcq_bcjr_soft.restype = I
-    L.tcq_bcjr_soft.argtypes = [TP, P, I64, F, P, P, P, SZ, P]
+    L.tcq_bcjr_soft.argtypes = [TP, P, P, I64, F, P, P, P, SZ, P]
     L.tcq_bcjr_soft_backward.restype = I
-    L.tcq_bcjr_soft_backward.argtypes = [TP, P, I64, F, P, P, P, P, SZ, P]
+    L.tcq_bcjr_soft_backward.argtypes = [TP, P, P, I64, F, P, P, P, P, SZ, P]
     L.tcq_pack_states.restype = I
     L.tcq_pack_states.argtypes = [TP, P, I64, I, P, P]
     L.tcq_decode.restype = I

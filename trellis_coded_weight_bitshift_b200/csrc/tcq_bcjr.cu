@@ -86,7 +86,7 @@ struct BcjrCfg {
   static constexpr size_t smem_floats() {
     return (size_t)SPC * NBUF * NV * NG                            // state vectors
            + (size_t)ASM * G * TPS                                  // smem code values
-           + (size_t)SPC * 256 * (GRAD ? 3 : 1)                     // s (+ v, soft)
+           + (size_t)SPC * 256 * (GRAD ? 4 : 2)                     // s, kappa*D (+ v, soft)
            + (size_t)SPC * 256                                       // CA_t prefix sums
            + (size_t)2 * SPC * NPART * PREC;                        // partial records
   }
@@ -160,7 +160,8 @@ __device__ __forceinline__ void write_run(float *vec, int base, const float *src
 
 template <class C>
 __global__ void __launch_bounds__(C::NT, C::MINB)
-bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, float two_over_temp,
+bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n_seq, int T,
+            float kappa, float two_over_temp,
             const float *__restrict__ vgrad, const float *__restrict__ soft_in,
             float *__restrict__ soft_out, float *__restrict__ logz_out,
             float *__restrict__ grad_out, float *__restrict__ ws) {
@@ -171,7 +172,8 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
   float *Vall = smem;                                      // [SPC][NB][NV][NG]
   float *Csm = Vall + SPC * NB * NV * NG;                  // [ASM][GQ][TPS][4]
   float *ssm = Csm + C::ASM * G * TPS;                     // [SPC][256]
-  float *vsm = ssm + SPC * 256;                            // GRAD: v, soft rows
+  float *ksm = ssm + SPC * 256;                            // [SPC][256] kappa * D_t
+  float *vsm = ksm + SPC * 256;                            // GRAD: v, soft rows
   float *fsm = vsm + (GRAD ? SPC * 256 : 0);
   float *cah = fsm + (GRAD ? SPC * 256 : 0);               // [SPC][256] CA_t
   float *part = cah + SPC * 256;                           // [2][SPC][NPART][PREC]
@@ -209,6 +211,7 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
       const int64_t sq = base + l;
       const bool ok = sq < n_seq;
       ssm[l * 256 + t] = ok ? s[sq * T + t] : 0.0f;
+      ksm[l * 256 + t] = kappa * ((ok && Dw) ? Dw[sq * T + t] : 1.0f);
       if (GRAD) {
         vsm[l * 256 + t] = ok ? vgrad[sq * T + t] : 0.0f;
         fsm[l * 256 + t] = ok ? soft_in[sq * T + t] : 0.0f;
@@ -261,7 +264,7 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
       const float fv = GRAD ? fsm[ls * 256 + t - 1] : 0.0f;
       float tmax = -INFINITY;
       if constexpr (!GRAD) {
-        const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa);
+        const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + t - 1], -ksm[ls * 256 + t - 1]);
 #pragma unroll
         for (int q = 0; q < GQ; ++q) {
           // x[a][r]: input of group 4q + r from predecessor digit a
@@ -288,7 +291,7 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
               make_float4(outA[0], outA[1], outA[2], outA[3]);
         }
       } else {
-        const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa), vv2 = f2(vv, vv);
+        const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + t - 1], -ksm[ls * 256 + t - 1]), vv2 = f2(vv, vv);
 #pragma unroll
         for (int q = 0; q < GQ; ++q) {
           float x[4][4], z[4][4];
@@ -356,7 +359,7 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
             const float d = code_at<C>(creg, Csm, a, 4 * k + b, w) - sT;
-            y[b] = -kappa * d * d;
+            y[b] = -ksm[ls * 256 + T - 1] * d * d;
           }
           const float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
           const float S = ex2(y[0] - mx) + ex2(y[1] - mx) + ex2(y[2] - mx) + ex2(y[3] - mx);
@@ -439,7 +442,9 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
           }
           const float inv = 1.0f / den;
           if (soft_out) soft_out[seq * T + tc + 1] = num * inv;
-          if (GRAD) grad_out[seq * T + tc + 1] = two_over_temp * (n2 * inv - (num * inv) * (n1 * inv));
+          if (GRAD)
+            grad_out[seq * T + tc + 1] = (1.3862943611198906f * ksm[ls * 256 + tc + 1]) *
+                                         (n2 * inv - (num * inv) * (n1 * inv));
         }
       }
       if (NB == 1) __syncthreads();
@@ -451,7 +456,7 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
       float *Bo = Bv + ((t + NB) % NB) * NV * NG;
       float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f, tmax = -INFINITY;
       if constexpr (!GRAD) {
-        const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa);
+        const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + tc], -ksm[ls * 256 + tc]);
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           float av[GQ];
@@ -490,7 +495,7 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
           if (t >= 0) write_run<C>(Bo, a * (NG / 4) + GQ * w, outB);
         }
       } else {
-        const f2_t sv2 = f2(sv, sv), nk2 = f2(-kappa, -kappa), vv2 = f2(vv, vv);
+        const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + tc], -ksm[ls * 256 + tc]), vv2 = f2(vv, vv);
         const float nvf = -vv * fv;
         // spilled (A, Phi) values of digit a, loaded one digit ahead
         constexpr int QN = (GQ + 3) / 4;
@@ -582,7 +587,8 @@ bcjr_kernel(const float *__restrict__ s, int64_t n_seq, int T, float kappa, floa
       }
       const float inv = 1.0f / den;
       if (soft_out) soft_out[seq * T] = num * inv;
-      if (GRAD) grad_out[seq * T] = two_over_temp * (n2 * inv - (num * inv) * (n1 * inv));
+      if (GRAD)   // 2 D_u / temp = 2 ln2 kappa D_u
+        grad_out[seq * T] = (1.3862943611198906f * ksm[ls * 256]) * (n2 * inv - (num * inv) * (n1 * inv));
     }
   }
 }
@@ -628,15 +634,15 @@ size_t ws_bytes_for(int64_t n_seq, int T) {
 }
 
 template <class C>
-tcq_status_t launch(const float *s, int64_t n_seq, int T, float kappa, float two_over_temp,
-                    const float *v,
+tcq_status_t launch(const float *s, const float *D, int64_t n_seq, int T, float kappa,
+                    float two_over_temp, const float *v,
                     const float *soft_in, float *soft, float *logz, float *grad, void *ws,
                     size_t ws_bytes, cudaStream_t stream) {
   if (!set_smem<C>()) return TCQ_ERR_CUDA;
   const int grid = grid_for<C>(n_seq);
   const size_t need = (size_t)grid * C::SPC * C::ws_floats_per_slot(T) * sizeof(float);
   if (ws_bytes < need) return TCQ_ERR_WORKSPACE;
-  bcjr_kernel<C><<<grid, C::NT, C::smem_bytes(), stream>>>(s, n_seq, T, kappa, two_over_temp, v,
+  bcjr_kernel<C><<<grid, C::NT, C::smem_bytes(), stream>>>(s, D, n_seq, T, kappa, two_over_temp, v,
                                                            soft_in, soft, logz, grad,
                                                            static_cast<float *>(ws));
   return launch_status();
@@ -663,15 +669,16 @@ extern "C" size_t tcq_bcjr_workspace_size(const tcq_trellis_t *tr, int64_t n_seq
 
 static bool temp_ok(float temp) { return temp > 0.0f && temp < INFINITY; }
 
-extern "C" tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *tr, const float *s, int64_t n_seq,
-                                      float temp, float *soft, float *log_z, void *ws,
-                                      size_t ws_bytes, void *stream) {
+extern "C" tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *tr, const float *s, const float *D,
+                                      int64_t n_seq, float temp, float *soft, float *log_z,
+                                      void *ws, size_t ws_bytes, void *stream) {
   tcq_status_t st = check_trellis(tr);
   if (st != TCQ_OK) return st;
   if (!temp_ok(temp)) return TCQ_ERR_INVALID_ARG;
   if (n_seq < 0 || n_seq > (int64_t)INT32_MAX) return TCQ_ERR_INVALID_ARG;
   if (n_seq == 0) return TCQ_OK;
-  if (!s || !soft || !aligned16(s) || !aligned16(soft) || (log_z && !aligned16(log_z)))
+  if (!s || !soft || !aligned16(s) || !aligned16(soft) || (log_z && !aligned16(log_z)) ||
+      (D && !aligned16(D)))
     return TCQ_ERR_INVALID_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
   const float kappa = (float)(1.4426950408889634 / (double)temp);
@@ -679,14 +686,15 @@ extern "C" tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *tr, const float *s, i
   cudaStream_t strm = (cudaStream_t)stream;
   const int T = tr->seq_len;
   switch (tr->L) {
-    case 8: return launch<Soft8>(s, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
-    case 12: return launch<Soft12>(s, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
-    default: return launch<Soft16>(s, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
+    case 8: return launch<Soft8>(s, D, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
+    case 12: return launch<Soft12>(s, D, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
+    default: return launch<Soft16>(s, D, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
   }
 }
 
 extern "C" tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *tr, const float *s,
-                                               int64_t n_seq, float temp, const float *soft,
+                                               const float *D, int64_t n_seq, float temp,
+                                               const float *soft,
                                                const float *grad_soft, float *grad_s, void *ws,
                                                size_t ws_bytes, void *stream) {
   tcq_status_t st = check_trellis(tr);
@@ -696,7 +704,7 @@ extern "C" tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *tr, const fl
   if (n_seq < 0 || n_seq > (int64_t)INT32_MAX) return TCQ_ERR_INVALID_ARG;
   if (n_seq == 0) return TCQ_OK;
   if (!s || !soft || !grad_soft || !grad_s || !aligned16(s) || !aligned16(soft) ||
-      !aligned16(grad_soft) || !aligned16(grad_s))
+      !aligned16(grad_soft) || !aligned16(grad_s) || (D && !aligned16(D)))
     return TCQ_ERR_INVALID_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
   const float kappa = (float)(1.4426950408889634 / (double)temp);
@@ -704,7 +712,7 @@ extern "C" tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *tr, const fl
   cudaStream_t strm = (cudaStream_t)stream;
   const int T = tr->seq_len;
   switch (tr->L) {
-    case 8: return launch<Grad8>(s, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
-    default: return launch<Grad12>(s, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
+    case 8: return launch<Grad8>(s, D, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
+    default: return launch<Grad12>(s, D, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
   }
 }

@@ -44,7 +44,7 @@ struct VitCfg {
   static constexpr int BPB = G / 4;            // backpointer bytes per thread per step
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
   static constexpr size_t smem_bytes() {
-    return sizeof(float) * ((size_t)SPC * NBUF * NG + (size_t)ASM * G * TPS + (size_t)SPC * 256) +
+    return sizeof(float) * ((size_t)SPC * NBUF * NG + (size_t)ASM * G * TPS + (size_t)SPC * 512) +
            sizeof(unsigned long long) * NT;
   }
   static_assert(NG % G == 0 && G % 4 == 0, "bad group split");
@@ -67,10 +67,10 @@ __device__ __forceinline__ void load_run(const float *base, int idx, float *dst)
   }
 }
 
-template <class C>
+template <class C, bool WEIGHTED>
 __global__ void __launch_bounds__(C::NT, C::MINB)
-viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
-                   uint8_t *__restrict__ bp, uint16_t *__restrict__ states,
+viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n_seq,
+                   int T, uint8_t *__restrict__ bp, uint16_t *__restrict__ states,
                    float *__restrict__ mse) {
   constexpr int NG = C::NG, G = C::G, GQ = C::GQ, TPS = C::TPS, AREG = C::AREG, ASM = C::ASM;
   constexpr int NB = C::NBUF;
@@ -78,7 +78,8 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
   float *Mall = smem;                                              // [SPC][NB][NG]
   float *Csm = Mall + C::SPC * NB * NG;                            // [ASM][G/4][TPS] float4
   float *ssm = Csm + ASM * G * TPS;                                // [SPC][256]
-  unsigned long long *red = reinterpret_cast<unsigned long long *>(ssm + C::SPC * 256);
+  float *dsm = ssm + C::SPC * 256;                                 // [SPC][256] weights
+  unsigned long long *red = reinterpret_cast<unsigned long long *>(dsm + C::SPC * 256);
 
   const int tid = threadIdx.x;
   const int ls = tid / TPS, w = tid - ls * TPS;
@@ -109,6 +110,7 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
     const int l = x / T, t = x - l * T;
     const int64_t sq = (int64_t)blockIdx.x * C::SPC + l;
     ssm[l * 256 + t] = sq < n_seq ? s[sq * T + t] : 0.0f;
+    if (WEIGHTED) dsm[l * 256 + t] = sq < n_seq ? Dw[sq * T + t] : 0.0f;
   }
   float *M = Mall + ls * NB * NG;
   for (int x = w; x < NG; x += TPS) M[x] = 0.0f;                 // M_0 = 0
@@ -150,6 +152,8 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
     // d = c - s, e = d*d (written fma(d, d, +0)), cost = M + e, each lane
     // rounded exactly like the scalar operation.
     const f2_t sv2 = f2(sv, sv);
+    const float dv = WEIGHTED ? dsm[ls * 256 + t - 1] : 1.0f;
+    const f2_t dv2 = f2(dv, dv);
 #pragma unroll
     for (int q = 0; q < GQ; ++q) {
       float4 csm[ASM > 0 ? ASM : 1];
@@ -168,7 +172,9 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
             cp = h == 0 ? f2(v.x, v.y) : f2(v.z, v.w);
           }
           const f2_t d = f2sub(cp, sv2);
-          const f2_t cost = f2add(f2(min_in[a][q], min_in[a][q]), f2fma(d, d, 0ull));
+          f2_t e = f2fma(d, d, 0ull);                     // RN(d*d)
+          if (WEIGHTED) e = f2fma(e, dv2, 0ull);          // RN(e*D), D >= 0
+          const f2_t cost = f2add(f2(min_in[a][q], min_in[a][q]), e);
           clo[a] = f2lo(cost);
           chi[a] = f2hi(cost);
         }
@@ -225,7 +231,9 @@ viterbi_fwd_kernel(const float *__restrict__ s, int64_t n_seq, int T,
             c = r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
           }
           const float d = __fsub_rn(c, sv);
-          const float cost = __fadd_rn(min_in[a][q], __fmul_rn(d, d));
+          float e = __fmul_rn(d, d);
+          if (WEIGHTED) e = __fmul_rn(e, dsm[ls * 256 + T - 1]);
+          const float cost = __fadd_rn(min_in[a][q], e);
           const unsigned long long key =
               ((unsigned long long)__float_as_uint(cost) << 32) | (uint32_t)(a * NG + G * w + i);
           best = key < best ? key : best;
@@ -315,18 +323,26 @@ using Vit16 = VitCfg<16, 32, 1, 2, 1>;   // 512 threads / sequence, half the cod
 
 size_t bp_bytes_per_seq(int L, int T) { return (size_t)(T - 1) * ((size_t)1 << (L - 4)); }
 
-template <class C>
-tcq_status_t launch_fwd(const float *s, int64_t n_seq, int T, uint8_t *bp, uint16_t *states,
-                        float *mse, cudaStream_t stream) {
+template <class C, bool WEIGHTED>
+tcq_status_t launch_fwd_w(const float *s, const float *D, int64_t n_seq, int T, uint8_t *bp,
+                          uint16_t *states, float *mse, cudaStream_t stream) {
   const size_t smem = C::smem_bytes();
   if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(viterbi_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(viterbi_fwd_kernel<C, WEIGHTED>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return TCQ_ERR_CUDA;
   }
   const int64_t blocks = (n_seq + C::SPC - 1) / C::SPC;
-  viterbi_fwd_kernel<C><<<(unsigned)blocks, C::NT, smem, stream>>>(s, n_seq, T, bp, states, mse);
+  viterbi_fwd_kernel<C, WEIGHTED><<<(unsigned)blocks, C::NT, smem, stream>>>(s, D, n_seq, T, bp,
+                                                                            states, mse);
   return launch_status();
+}
+
+template <class C>
+tcq_status_t launch_fwd(const float *s, int64_t n_seq, int T, uint8_t *bp, uint16_t *states,
+                        float *mse, cudaStream_t stream, const float *D = nullptr) {
+  return D ? launch_fwd_w<C, true>(s, D, n_seq, T, bp, states, mse, stream)
+           : launch_fwd_w<C, false>(s, nullptr, n_seq, T, bp, states, mse, stream);
 }
 
 template <int L>
@@ -360,14 +376,15 @@ extern "C" size_t tcq_viterbi_workspace_size(const tcq_trellis_t *tr, int64_t n_
   return ((bp_bytes_per_seq(tr->L, tr->seq_len) * (size_t)n_seq + 255) / 256) * 256 + 256;
 }
 
-extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float *s, int64_t n_seq,
-                                           uint16_t *states, float *mse, void *ws,
-                                           size_t ws_bytes, void *stream) {
+extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float *s,
+                                           const float *D, int64_t n_seq, uint16_t *states,
+                                           float *mse, void *ws, size_t ws_bytes, void *stream) {
   tcq_status_t st = check_trellis(tr);
   if (st != TCQ_OK) return st;
   if (n_seq < 0 || n_seq > (int64_t)INT32_MAX * 8) return TCQ_ERR_INVALID_ARG;
   if (n_seq == 0) return TCQ_OK;
-  if (!s || !states || !mse || !aligned16(s) || !aligned16(states) || !aligned16(mse))
+  if (!s || !states || !mse || !aligned16(s) || !aligned16(states) || !aligned16(mse) ||
+      (D && !aligned16(D)))
     return TCQ_ERR_INVALID_ARG;
   const size_t need = tcq_viterbi_workspace_size(tr, n_seq);
   if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
@@ -375,9 +392,9 @@ extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float 
   uint8_t *bp = static_cast<uint8_t *>(ws);
   cudaStream_t strm = (cudaStream_t)stream;
   switch (tr->L) {
-    case 8: st = launch_fwd<Vit8>(s, n_seq, T, bp, states, mse, strm); break;
-    case 12: st = launch_fwd<Vit12>(s, n_seq, T, bp, states, mse, strm); break;
-    default: st = launch_fwd<Vit16>(s, n_seq, T, bp, states, mse, strm); break;
+    case 8: st = launch_fwd<Vit8>(s, n_seq, T, bp, states, mse, strm, D); break;
+    case 12: st = launch_fwd<Vit12>(s, n_seq, T, bp, states, mse, strm, D); break;
+    default: st = launch_fwd<Vit16>(s, n_seq, T, bp, states, mse, strm, D); break;
   }
   if (st != TCQ_OK || T == 1) return st;
   return launch_traceback(tr->L, bp, n_seq, T, states, strm);
