@@ -79,6 +79,12 @@ def _lib():
     lib.orc_bcjr_vjp_f64.restype = I
     lib.orc_bruteforce_f64.argtypes = [I, I, I, D, P, P, P, P, P, P, P]
     lib.orc_bruteforce_f64.restype = ctypes.c_int64
+    lib.orc_viterbi_pinned_f32.argtypes = [I, I, I, P, P, P, I, P]
+    lib.orc_viterbi_pinned_f32.restype = ctypes.c_float
+    lib.orc_viterbi_pinned_f64.argtypes = [I, I, I, P, P, P, I, P]
+    lib.orc_viterbi_pinned_f64.restype = D
+    lib.orc_bruteforce_tailbiting_f64.argtypes = [I, I, I, P, P, P]
+    lib.orc_bruteforce_tailbiting_f64.restype = D
     return lib
 
 
@@ -171,6 +177,78 @@ def viterbi_f64(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = Non
         mse[i] = cost / T
         margin[i] = m.value
     return states, mse, margin
+
+
+# --------------------------------------------------------------------------
+# Tail-biting search (QTIP blog, "Tail-biting is worth its complexity")
+# --------------------------------------------------------------------------
+def viterbi_pinned_f32(s: np.ndarray, L: int, overlap, k: int = 2, D=None):
+    """fp32 Viterbi with the first state's top L-k bits and the last state's
+    low L-k bits both equal to ``overlap`` (per row); returns (states, cost)."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    if s.ndim == 1:
+        s = s[None]
+    n, T = s.shape
+    D = _rows(D, n, T, np.float32)
+    overlap = np.broadcast_to(np.asarray(overlap, dtype=np.int64), (n,))
+    code = codebook_f32(L)
+    states = np.empty((n, T), dtype=np.uint16)
+    cost = np.empty(n, dtype=np.float32)
+    for i in range(n):
+        cost[i] = _lib().orc_viterbi_pinned_f32(L, k, T, _ptr(s[i]), _row_ptr(D, i), _ptr(code),
+                                                int(overlap[i]), _ptr(states[i]))
+    return states, cost
+
+
+def viterbi_tailbiting_alg4_f32(s: np.ndarray, L: int, k: int = 2, D=None):
+    """The two-run tail-biting search: Viterbi on the sequence rotated by
+    T/2, the overlap read off the seam (the top L-k bits of the state that
+    lands on original position 0), then Viterbi on the original sequence with
+    both ends pinned to it.  fp32, the same arithmetic as viterbi_f32.
+    Returns (states [n, T] tail-biting walks, mse [n], overlap [n])."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    if s.ndim == 1:
+        s = s[None]
+    n, T = s.shape
+    h = T // 2
+    Dr = None if D is None else np.roll(_rows(D, n, T, np.float32), -h, axis=1)
+    st_rot, _ = viterbi_f32(np.roll(s, -h, axis=1), L, k=k, D=Dr)
+    overlap = st_rot[:, (T - h) % T].astype(np.int64) >> k     # rotated position of original 0
+    states, cost = viterbi_pinned_f32(s, L, overlap, k=k, D=D)
+    return states, (cost / np.float32(T)).astype(np.float32), overlap
+
+
+def viterbi_tailbiting_exact_f64(s: np.ndarray, L: int, k: int = 2, D=None):
+    """Exact tail-biting optimum: the best of the 2^(L-k) pinned runs (fp64).
+    Returns (states [n, T], mse [n])."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    if s.ndim == 1:
+        s = s[None]
+    n, T = s.shape
+    D = _rows(D, n, T, np.float64)
+    code = codebook_f64(L)
+    states = np.empty((n, T), dtype=np.uint16)
+    mse = np.empty(n)
+    buf = np.empty(T, dtype=np.uint16)
+    for i in range(n):
+        best = np.inf
+        for o in range(1 << (L - k)):
+            c = _lib().orc_viterbi_pinned_f64(L, k, T, _ptr(s[i]), _row_ptr(D, i), _ptr(code), o,
+                                              _ptr(buf))
+            if c < best:
+                best = c
+                states[i] = buf
+        mse[i] = best / T
+    return states, mse
+
+
+def bruteforce_tailbiting(s: np.ndarray, L: int, k: int = 2, D=None) -> float:
+    """Minimum energy over tail-biting walks only, by enumeration (tiny cases)."""
+    s = np.ascontiguousarray(s, dtype=np.float64).ravel()
+    T = s.shape[0]
+    Dr = None if D is None else np.ascontiguousarray(np.broadcast_to(np.asarray(D), (T,)), dtype=np.float64)
+    return float(_lib().orc_bruteforce_tailbiting_f64(L, k, T, _ptr(s), None if Dr is None else _ptr(Dr),
+                                                      _ptr(codebook_f64(L))))
 
 
 # --------------------------------------------------------------------------

@@ -407,3 +407,124 @@ int64_t orc_bruteforce_f64(int L, int k, int T, double temp, const double *s, co
     *min_energy = emin;
     return W;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Tail-biting search   [QTIP-blog, "Tail-biting is worth its complexity"]  */
+/* A tail-biting walk also wraps: the last state's low L-k bits equal the   */
+/* first state's high L-k bits, so the stream is exactly k*T bits.  With    */
+/* that shared value o fixed, the search is a Viterbi run whose first state */
+/* must have top bits o and whose last state must have low bits o; the      */
+/* exact optimum is the best of the 2^(L-k) runs, one per o.                */
+/* orc_viterbi_pinned_*: as orc_viterbi_* (same arithmetic and tie-breaks)  */
+/* with those two restrictions; returns the minimum cost (INFINITY if no    */
+/* walk satisfies them).                                                     */
+/* ------------------------------------------------------------------------ */
+float orc_viterbi_pinned_f32(int L, int k, int T, const float *s, const float *D,
+                             const float *code, int o, uint16_t *states)
+{
+    const int N = 1 << L, A = 1 << k;
+    const int low = (1 << (L - k)) - 1;
+    float *cost = (float *)malloc(sizeof(float) * N);
+    float *next = (float *)malloc(sizeof(float) * N);
+    int32_t *back = (int32_t *)malloc(sizeof(int32_t) * (size_t)T * N);
+
+    for (int j = 0; j < N; ++j) {
+        if ((j >> k) != o) { cost[j] = INFINITY; continue; }
+        float d = code[j] - s[0];
+        float e = d * d;
+        cost[j] = D ? e * D[0] : e;
+    }
+    for (int t = 1; t < T; ++t) {
+        for (int j = 0; j < N; ++j) {
+            float best = INFINITY;
+            int bestp = -1;
+            for (int a = 0; a < A; ++a) {
+                int p = (j >> k) | (a << (L - k));
+                if (bestp < 0 || cost[p] < best) { best = cost[p]; bestp = p; }
+            }
+            float d = code[j] - s[t];
+            float e = d * d;
+            if (D) e = e * D[t];
+            next[j] = best + e;
+            back[(size_t)t * N + j] = bestp;
+        }
+        float *tmp = cost; cost = next; next = tmp;
+    }
+    int st = -1;
+    for (int j = 0; j < N; ++j)
+        if ((j & low) == o && (st < 0 || cost[j] < cost[st])) st = j;
+    float total = cost[st];
+    states[T - 1] = (uint16_t)st;
+    for (int t = T - 1; t > 0; --t) {
+        st = back[(size_t)t * N + st];
+        states[t - 1] = (uint16_t)st;
+    }
+    free(cost); free(next); free(back);
+    return total;
+}
+
+double orc_viterbi_pinned_f64(int L, int k, int T, const double *s, const double *D,
+                              const double *code, int o, uint16_t *states)
+{
+    const int N = 1 << L, A = 1 << k;
+    const int low = (1 << (L - k)) - 1;
+    double *cost = (double *)malloc(sizeof(double) * N);
+    double *next = (double *)malloc(sizeof(double) * N);
+    int32_t *back = (int32_t *)malloc(sizeof(int32_t) * (size_t)T * N);
+
+    for (int j = 0; j < N; ++j) {
+        double d = code[j] - s[0];
+        cost[j] = (j >> k) == o ? (D ? D[0] : 1.0) * d * d : INFINITY;
+    }
+    for (int t = 1; t < T; ++t) {
+        for (int j = 0; j < N; ++j) {
+            double best = INFINITY;
+            int bestp = -1;
+            for (int a = 0; a < A; ++a) {
+                int p = (j >> k) | (a << (L - k));
+                if (bestp < 0 || cost[p] < best) { best = cost[p]; bestp = p; }
+            }
+            double d = code[j] - s[t];
+            next[j] = best + (D ? D[t] : 1.0) * d * d;
+            back[(size_t)t * N + j] = bestp;
+        }
+        double *tmp = cost; cost = next; next = tmp;
+    }
+    int st = -1;
+    for (int j = 0; j < N; ++j)
+        if ((j & low) == o && (st < 0 || cost[j] < cost[st])) st = j;
+    double total = cost[st];
+    states[T - 1] = (uint16_t)st;
+    for (int t = T - 1; t > 0; --t) {
+        st = back[(size_t)t * N + st];
+        states[t - 1] = (uint16_t)st;
+    }
+    free(cost); free(next); free(back);
+    return total;
+}
+
+/* Brute force over tail-biting walks only (tiny L, T): minimum energy. */
+double orc_bruteforce_tailbiting_f64(int L, int k, int T, const double *s, const double *D,
+                                     const double *code)
+{
+    const int bits = L + k * (T - 1);
+    if (bits > 24 || T < 1) return NAN;
+    const int64_t W = (int64_t)1 << bits;
+    const uint32_t mask = (1u << L) - 1u, low = (1u << (L - k)) - 1u;
+    double emin = INFINITY;
+    for (int64_t w = 0; w < W; ++w) {
+        uint64_t cb = (uint64_t)w;
+        uint32_t x = (uint32_t)(cb >> (k * (T - 1))) & mask, x0 = x;
+        double E = 0.0;
+        for (int t = 0; t < T; ++t) {
+            if (t > 0) {
+                uint32_t dgt = (uint32_t)(cb >> (k * (T - 1 - t))) & ((1u << k) - 1u);
+                x = ((x << k) | dgt) & mask;
+            }
+            double d = code[x] - s[t];
+            E += (D ? D[t] : 1.0) * d * d;
+        }
+        if ((x & low) == (x0 >> k) && E < emin) emin = E;
+    }
+    return emin;
+}
