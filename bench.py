@@ -54,6 +54,8 @@ def _metric_for(w: W.Workload) -> str:
     parts = []
     if "viterbi" in w.ops:
         parts.append("Viterbi")
+    if "viterbi_tb" in w.ops:
+        parts.append("tail-biting Viterbi (two-run)")
     if "bcjr" in w.ops:
         parts.append("BCJR soft" + (f" x{len(w.temps)} temps" if len(w.temps) > 1 else ""))
     if "bcjr_grad" in w.ops:
@@ -135,6 +137,8 @@ def _oracle_step(w: W.Workload, s: np.ndarray, D=None) -> None:
     import oracle
     if "viterbi" in w.ops:
         oracle.viterbi_f32(s, w.L, D=D)
+    if "viterbi_tb" in w.ops:
+        oracle.viterbi_tailbiting_alg4_f32(s, w.L, D=D)
     for temp in w.temps:
         if "bcjr_grad" in w.ops and temp == w.temps[0]:
             oracle.bcjr_vjp(s, np.ones_like(s, dtype=np.float64), w.L, temp, D=D)  # also yields soft
@@ -275,7 +279,7 @@ def run_ours(a) -> None:
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
     ws_v = ws_b = ws_g = None
-    if "viterbi" in w.ops:
+    if "viterbi" in w.ops or "viterbi_tb" in w.ops:
         ws_v = torch.empty(tcq.viterbi_workspace_size(w.L, 256, w.n_seq), dtype=torch.uint8, device=dev)
     if "bcjr" in w.ops:
         ws_b = torch.empty(tcq.bcjr_workspace_size(w.L, 256, w.n_seq), dtype=torch.uint8, device=dev)
@@ -312,6 +316,11 @@ def run_ours(a) -> None:
                 st, mse = tcq.viterbi_encode(inp, w.L, ws_v, D=Dd)
                 mark("viterbi")
                 n_launch += 2
+                outs += [st, mse]
+            if "viterbi_tb" in w.ops:
+                st, mse = tcq.viterbi_encode_tailbiting(inp, w.L, ws_v, D=Dd)
+                mark("viterbi_tb")
+                n_launch += 4
                 outs += [st, mse]
             for i, temp in enumerate(w.temps):
                 soft, lz = tcq.bcjr_soft(inp, w.L, temp, ws_b, D=Dd)

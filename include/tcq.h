@@ -127,6 +127,22 @@ TCQ_API tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *trellis, const floa
                                         float *mse, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Tail-biting Viterbi encode [QTIP, "Tail-biting is worth its complexity":
+ * the last state's low L-k bits equal the first state's high L-k bits, so a
+ * sequence costs exactly k*T bits; the two-run search rotates the sequence by
+ * T/2, runs Viterbi, reads the shared bits at the seam and re-runs with both
+ * ends pinned to them].
+ *   Same arguments, arithmetic and tie-breaks as tcq_viterbi_encode; the
+ *   output walk is tail-biting (pack it with TCQ_TAILBITING) and mse is its
+ *   cost / seq_len.  Needs k*seq_len >= L.  Workspace: as tcq_viterbi_encode.
+ *   `states` is also used as scratch between the two runs.
+ * ------------------------------------------------------------------------ */
+TCQ_API tcq_status_t tcq_viterbi_encode_tailbiting(const tcq_trellis_t *trellis, const float *s,
+                                                   const float *D, int64_t n_seq,
+                                                   uint16_t *states, float *mse, void *ws,
+                                                   size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * Allocation-free Viterbi encode (the pages have no counterpart: this is a
  * deployment convenience of this library).
  *

@@ -58,6 +58,9 @@ WORKLOADS = {
     # "Cliff edges"); D log-uniform on [0.1, 10] from seed 6
     "l12_curv1024": Workload("l12_curv1024", 12, 1024, "gaussian", 2, (0.05,),
                              ops=("viterbi", "bcjr", "bcjr_grad"), curv_seed=6),
+    # the 1024x1024 RHT block encoded tail-biting (exactly 2 bits per weight)
+    "l16_rht1024_tb": Workload("l16_rht1024_tb", 16, 4096, "rht_block", 3, (), 1024, 1024,
+                               ops=("viterbi_tb",)),
 }
 
 

@@ -321,3 +321,54 @@ def _bcjr_gpu_w(tcq, s, L, temp, D):
     soft, lz = tcq.bcjr_soft(_dev(s), L, temp, D=_dev(D))
     torch.cuda.synchronize()
     return soft.cpu().numpy(), lz.cpu().numpy()
+
+
+# ---------------------------------------------------------------- tail-biting encode
+def _tb_valid(st, L):
+    st = st.astype(np.int64)
+    low = (1 << (L - 2)) - 1
+    return _is_walk(st, L) & ((st[:, 0] >> 2) == (st[:, -1] & low))
+
+
+@pytest.mark.parametrize("L,n,T", [(8, 64, 256), (12, 96, 256), (16, 4, 256), (8, 9, 17), (12, 5, 6)])
+def test_tailbiting_matches_oracle_algorithm4(tcq, L, n, T):
+    s = W.gaussian(n, 1100 + L + T, seq_len=T)
+    st, mse = tcq.viterbi_encode_tailbiting(_dev(s), L)
+    torch.cuda.synchronize()
+    st = st.cpu().view(torch.int16).numpy().view(np.uint16)
+    rst, rmse, _ = oracle.viterbi_tailbiting_alg4_f32(s, L)
+    assert np.array_equal(st, rst)
+    assert np.array_equal(mse.cpu().numpy().view(np.uint32), rmse.view(np.uint32))
+    assert np.all(_tb_valid(st, L))
+
+
+def test_tailbiting_weighted(tcq):
+    s = W.gaussian(32, 1201)
+    D = W.curvature(32, 1202)
+    st, mse = tcq.viterbi_encode_tailbiting(_dev(s), 12, D=_dev(D))
+    torch.cuda.synchronize()
+    rst, rmse, _ = oracle.viterbi_tailbiting_alg4_f32(s, 12, D=D)
+    assert np.array_equal(st.cpu().view(torch.int16).numpy().view(np.uint16), rst)
+    assert np.array_equal(mse.cpu().numpy().view(np.uint32), rmse.view(np.uint32))
+
+
+def test_tailbiting_l16_rht_block_pack_decode(tcq):
+    s = W.sequences("l16_rht1024")
+    sd = _dev(s)
+    st_d, mse_d = tcq.viterbi_encode_tailbiting(sd, 16)
+    bits = tcq.pack_states(st_d, 16, tcq.TAILBITING)            # exactly 2 bits per weight
+    out = tcq.decode(bits, 16, 256, tcq.TAILBITING, tcq.OUT_TILE16, 1024, 1024)
+    torch.cuda.synchronize()
+    st = st_d.cpu().view(torch.int16).numpy().view(np.uint16)
+    mse = mse_d.cpu().numpy()
+    assert bits.shape == (4096, 16)
+    assert np.all(_tb_valid(st, 16))
+    assert np.array_equal(_seq_mse_f32(s, st, 16).view(np.uint32), mse.view(np.uint32))
+    ref = oracle.codebook_f16(16)[st.astype(np.int64)]            # decode = code of the walk
+    nr = 1024 // 16
+    tiles = out.cpu().numpy().view(np.uint16).reshape(nr, 16, nr, 16).transpose(0, 2, 1, 3).reshape(-1, 256)
+    assert np.array_equal(tiles, ref.view(np.uint16))
+    idx = np.array([0, 4095, 1234])
+    rst, rmse, _ = oracle.viterbi_tailbiting_alg4_f32(s[idx], 16)
+    assert np.array_equal(st[idx], rst)
+    assert abs(float(mse.mean()) - 0.0697) < 0.004               # page: L=16 tail-biting MSE

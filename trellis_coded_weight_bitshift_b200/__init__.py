@@ -9,6 +9,7 @@ no CPU fallback: without the built library or a CUDA device every call raises.
 Functions (QTIP blog "The trellis: a stateful codebook" / "The codebook is
 computed" / "Tail-biting is worth its complexity"; BCJR-QAT abstract):
   viterbi_encode(s, L)                   -> (states uint16 [n,T], mse f32 [n])
+  viterbi_encode_tailbiting(s, L)        -> tail-biting walks (2 bits per weight)
   bcjr_soft(s, L, temp)                  -> (soft f32 [n,T], log_z f32 [n])
   bcjr_soft_backward(s, L, temp, soft, g)-> grad_s f32 [n,T]
   BcjrSoft.apply(s, L, temp)             -> soft (autograd through the VJP)
@@ -26,7 +27,7 @@ from ._abi import (FREE_START, OUT_SEQ, OUT_TILE16, TAILBITING, TcqError, check,
                    status_string, trellis)
 
 __all__ = [
-    "viterbi_encode", "bcjr_soft", "bcjr_soft_backward", "BcjrSoft", "pack_states", "decode",
+    "viterbi_encode", "viterbi_encode_tailbiting", "bcjr_soft", "bcjr_soft_backward", "BcjrSoft", "pack_states", "decode",
     "stream_words", "viterbi_workspace_size", "bcjr_workspace_size", "TcqError",
     "TAILBITING", "FREE_START", "OUT_SEQ", "OUT_TILE16", "lib", "status_string",
 ]
@@ -92,6 +93,27 @@ def viterbi_encode(s: torch.Tensor, L: int, workspace: torch.Tensor | None = Non
     ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
     check(lib().tcq_viterbi_encode(ctypes.byref(tr), _ptr(s), _ptr(D), n, _ptr(states), _ptr(mse),
                                    _ptr(ws), ws.numel(), _stream()), "tcq_viterbi_encode")
+    return states, mse
+
+
+def viterbi_encode_tailbiting(s: torch.Tensor, L: int, workspace: torch.Tensor | None = None,
+                              D: torch.Tensor | None = None):
+    """Tail-biting walk of every row (two-run search: rotated free run, then a
+    run with both ends pinned to the overlap read at the seam); returns
+    (states uint16, mse fp32).  Pack the walk with layout TAILBITING."""
+    _require_cuda(s)
+    D = _weights(D, s)
+    if s.dtype != torch.float32 or s.dim() != 2:
+        raise ValueError("s must be a 2-D float32 tensor [n_seq, seq_len]")
+    n, T = s.shape
+    tr = trellis(L, T)
+    states = torch.empty((n, T), dtype=torch.uint16, device=s.device)
+    mse = torch.empty((n,), dtype=torch.float32, device=s.device)
+    need = int(lib().tcq_viterbi_workspace_size(ctypes.byref(tr), n))
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    check(lib().tcq_viterbi_encode_tailbiting(ctypes.byref(tr), _ptr(s), _ptr(D), n, _ptr(states),
+                                              _ptr(mse), _ptr(ws), ws.numel(), _stream()),
+          "tcq_viterbi_encode_tailbiting")
     return states, mse
 
 

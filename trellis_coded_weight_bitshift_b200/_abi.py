@@ -21,6 +21,7 @@ OUT_TILE16 = 1
 EXPORTS = (
     "tcq_version", "tcq_status_string", "tcq_stream_words",
     "tcq_viterbi_workspace_size", "tcq_viterbi_encode", "tcq_viterbi_encode_noalloc",
+    "tcq_viterbi_encode_tailbiting",
     "tcq_bcjr_workspace_size", "tcq_bcjr_soft", "tcq_bcjr_soft_backward",
     "tcq_pack_states", "tcq_decode",
 )
@@ -57,6 +58,8 @@ def lib() -> ctypes.CDLL:
     L.tcq_viterbi_workspace_size.argtypes = [TP, I64]
     L.tcq_viterbi_encode.restype = I
     L.tcq_viterbi_encode.argtypes = [TP, P, P, I64, P, P, P, SZ, P]
+    L.tcq_viterbi_encode_tailbiting.restype = I
+    L.tcq_viterbi_encode_tailbiting.argtypes = [TP, P, P, I64, P, P, P, SZ, P]
     L.tcq_viterbi_encode_noalloc.restype = I
     L.tcq_viterbi_encode_noalloc.argtypes = [TP, P, I64, P, P, P]
     L.tcq_bcjr_workspace_size.restype = SZ

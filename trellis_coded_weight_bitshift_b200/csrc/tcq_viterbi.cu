@@ -70,8 +70,8 @@ __device__ __forceinline__ void load_run(const float *base, int idx, float *dst)
 template <class C, bool WEIGHTED>
 __global__ void __launch_bounds__(C::NT, C::MINB)
 viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n_seq,
-                   int T, uint8_t *__restrict__ bp, uint16_t *__restrict__ states,
-                   float *__restrict__ mse) {
+                   int T, int rot, const uint16_t *pin_states, int pin_pos,
+                   uint8_t *__restrict__ bp, uint16_t *states, float *__restrict__ mse) {
   constexpr int NG = C::NG, G = C::G, GQ = C::GQ, TPS = C::TPS, AREG = C::AREG, ASM = C::ASM;
   constexpr int NB = C::NBUF;
   extern __shared__ __align__(16) float smem[];
@@ -106,14 +106,22 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
         reinterpret_cast<float4 *>(Csm)[(a * GQ + q) * TPS + w] = v;
       }
   }
+  // targets (and weights) of step t are element (t + rot) mod T of the row
   for (int x = tid; x < C::SPC * T; x += C::NT) {
     const int l = x / T, t = x - l * T;
     const int64_t sq = (int64_t)blockIdx.x * C::SPC + l;
-    ssm[l * 256 + t] = sq < n_seq ? s[sq * T + t] : 0.0f;
-    if (WEIGHTED) dsm[l * 256 + t] = sq < n_seq ? Dw[sq * T + t] : 0.0f;
+    int tr = t + rot;
+    if (tr >= T) tr -= T;
+    ssm[l * 256 + t] = sq < n_seq ? s[sq * T + tr] : 0.0f;
+    if (WEIGHTED) dsm[l * 256 + t] = sq < n_seq ? Dw[sq * T + tr] : 0.0f;
   }
+  // Pinned (tail-biting) run: the first state's top L-2 bits and the last
+  // state's low L-2 bits must both equal the overlap o, i.e. only group o may
+  // start (M_0 = 0 there, +inf elsewhere) and only states with low bits o may
+  // end the walk.
+  const int o = (pin_states != nullptr && active) ? (int)(pin_states[seq * T + pin_pos] >> 2) : -1;
   float *M = Mall + ls * NB * NG;
-  for (int x = w; x < NG; x += TPS) M[x] = 0.0f;                 // M_0 = 0
+  for (int x = w; x < NG; x += TPS) M[swz<C::SWZ>(x)] = (o < 0 || x == o) ? 0.0f : INFINITY;
   __syncthreads();
 
   uint8_t *bps = bp + (active ? seq : 0) * (int64_t)(T - 1) * (NG / 4);
@@ -236,7 +244,7 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
           const float cost = __fadd_rn(min_in[a][q], e);
           const unsigned long long key =
               ((unsigned long long)__float_as_uint(cost) << 32) | (uint32_t)(a * NG + G * w + i);
-          best = key < best ? key : best;
+          if (o < 0 || G * w + i == o) best = key < best ? key : best;
         }
       }
     }
@@ -325,7 +333,8 @@ size_t bp_bytes_per_seq(int L, int T) { return (size_t)(T - 1) * ((size_t)1 << (
 
 template <class C, bool WEIGHTED>
 tcq_status_t launch_fwd_w(const float *s, const float *D, int64_t n_seq, int T, uint8_t *bp,
-                          uint16_t *states, float *mse, cudaStream_t stream) {
+                          uint16_t *states, float *mse, cudaStream_t stream, int rot,
+                          const uint16_t *pin_states, int pin_pos) {
   const size_t smem = C::smem_bytes();
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(viterbi_fwd_kernel<C, WEIGHTED>,
@@ -333,16 +342,18 @@ tcq_status_t launch_fwd_w(const float *s, const float *D, int64_t n_seq, int T, 
       return TCQ_ERR_CUDA;
   }
   const int64_t blocks = (n_seq + C::SPC - 1) / C::SPC;
-  viterbi_fwd_kernel<C, WEIGHTED><<<(unsigned)blocks, C::NT, smem, stream>>>(s, D, n_seq, T, bp,
-                                                                            states, mse);
+  viterbi_fwd_kernel<C, WEIGHTED><<<(unsigned)blocks, C::NT, smem, stream>>>(
+      s, D, n_seq, T, rot, pin_states, pin_pos, bp, states, mse);
   return launch_status();
 }
 
 template <class C>
 tcq_status_t launch_fwd(const float *s, int64_t n_seq, int T, uint8_t *bp, uint16_t *states,
-                        float *mse, cudaStream_t stream, const float *D = nullptr) {
-  return D ? launch_fwd_w<C, true>(s, D, n_seq, T, bp, states, mse, stream)
-           : launch_fwd_w<C, false>(s, nullptr, n_seq, T, bp, states, mse, stream);
+                        float *mse, cudaStream_t stream, const float *D = nullptr, int rot = 0,
+                        const uint16_t *pin_states = nullptr, int pin_pos = 0) {
+  return D ? launch_fwd_w<C, true>(s, D, n_seq, T, bp, states, mse, stream, rot, pin_states, pin_pos)
+           : launch_fwd_w<C, false>(s, nullptr, n_seq, T, bp, states, mse, stream, rot, pin_states,
+                                    pin_pos);
 }
 
 template <int L>
@@ -398,6 +409,50 @@ extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float 
   }
   if (st != TCQ_OK || T == 1) return st;
   return launch_traceback(tr->L, bp, n_seq, T, states, strm);
+}
+
+// Tail-biting encode [QTIP blog, "Tail-biting is worth its complexity"]: two
+// runs.  First a free run on the sequence rotated by T/2, so that the wrap
+// point T-1 -> 0 sits in the middle of the walk; the state that lands on
+// original position 0 gives the overlap o (its top L-2 bits).  Then a run on
+// the original sequence with the first state's top bits and the last state's
+// low bits pinned to o: the result is a tail-biting walk whose stream is
+// exactly 2*T bits.  The first run's walk is written to `states` and read
+// back by the second run's prologue (stream order separates them).
+template <class C>
+static tcq_status_t tailbiting_passes(const float *s, const float *D, int64_t n_seq, int T,
+                                      uint8_t *bp, uint16_t *states, float *mse, int L,
+                                      cudaStream_t strm) {
+  const int h = T / 2;
+  tcq_status_t st = launch_fwd<C>(s, n_seq, T, bp, states, mse, strm, D, h);
+  if (st != TCQ_OK) return st;
+  if ((st = launch_traceback(L, bp, n_seq, T, states, strm)) != TCQ_OK) return st;
+  st = launch_fwd<C>(s, n_seq, T, bp, states, mse, strm, D, 0, states, (T - h) % T);
+  if (st != TCQ_OK) return st;
+  return launch_traceback(L, bp, n_seq, T, states, strm);
+}
+
+extern "C" tcq_status_t tcq_viterbi_encode_tailbiting(const tcq_trellis_t *tr, const float *s,
+                                                      const float *D, int64_t n_seq,
+                                                      uint16_t *states, float *mse, void *ws,
+                                                      size_t ws_bytes, void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if ((int64_t)tr->k * tr->seq_len < tr->L || tr->seq_len < 2) return TCQ_ERR_UNSUPPORTED;
+  if (n_seq < 0 || n_seq > (int64_t)INT32_MAX * 8) return TCQ_ERR_INVALID_ARG;
+  if (n_seq == 0) return TCQ_OK;
+  if (!s || !states || !mse || !aligned16(s) || !aligned16(states) || !aligned16(mse) ||
+      (D && !aligned16(D)))
+    return TCQ_ERR_INVALID_ARG;
+  const size_t need = tcq_viterbi_workspace_size(tr, n_seq);
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
+  uint8_t *bp = static_cast<uint8_t *>(ws);
+  cudaStream_t strm = (cudaStream_t)stream;
+  switch (tr->L) {
+    case 8: return tailbiting_passes<Vit8>(s, D, n_seq, tr->seq_len, bp, states, mse, 8, strm);
+    case 12: return tailbiting_passes<Vit12>(s, D, n_seq, tr->seq_len, bp, states, mse, 12, strm);
+    default: return tailbiting_passes<Vit16>(s, D, n_seq, tr->seq_len, bp, states, mse, 16, strm);
+  }
 }
 
 // ---------------------------------------------------------------------------

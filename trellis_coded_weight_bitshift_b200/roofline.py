@@ -84,6 +84,8 @@ def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str,
     states = float(1 << L)
     if kernel.startswith("decode"):
         return "hbm", n_seq * (T * 2 / 8 + T * 2), "bytes"
+    if kernel.startswith("viterbi_tb"):       # two Viterbi runs
+        return "alu", 2 * n_seq * T * states * 4.5, "lane-ops"
     if kernel.startswith("viterbi"):
         return "alu", n_seq * T * states * 4.5, "lane-ops"
     if kernel.startswith("bcjr_vjp"):
