@@ -5,7 +5,9 @@
 One step = one pass of the whole hot path over one batch of synthetic input:
 for the default workload (L=12, 1024 x 256 i.i.d. N(0,1) weights) that is
 Viterbi encode (forward + traceback, per-sequence MSE), the BCJR soft codeword
-at temp 0.05 and the gradient of the sum of soft codewords w.r.t. the targets.
+at temp 0.05 and the gradient of the sum of soft codewords w.r.t. the targets
+(soft codeword, log Z and gradient in one forward-backward sweep, since the
+cotangent is known up front).
 The metric is weights per second (whole job, all ranks).  Under torchrun each
 rank encodes its own batch (weak scaling, no data-path collective); the step
 time is the maximum over ranks of the CUDA-event time.
@@ -281,7 +283,7 @@ def run_ours(a) -> None:
     ws_v = ws_b = ws_g = None
     if "viterbi" in w.ops or "viterbi_tb" in w.ops:
         ws_v = torch.empty(tcq.viterbi_workspace_size(w.L, 256, w.n_seq), dtype=torch.uint8, device=dev)
-    if "bcjr" in w.ops:
+    if "bcjr" in w.ops and not ("bcjr_grad" in w.ops and len(w.temps) == 1):
         ws_b = torch.empty(tcq.bcjr_workspace_size(w.L, 256, w.n_seq), dtype=torch.uint8, device=dev)
     if "bcjr_grad" in w.ops:
         ws_g = torch.empty(tcq.bcjr_workspace_size(w.L, 256, w.n_seq, True), dtype=torch.uint8, device=dev)
@@ -323,15 +325,18 @@ def run_ours(a) -> None:
                 n_launch += 4
                 outs += [st, mse]
             for i, temp in enumerate(w.temps):
+                if "bcjr_grad" in w.ops and i == 0:
+                    # the cotangent (gradient of the sum of soft codewords) is
+                    # known up front: one sweep gives soft, log Z and grad
+                    soft, lz, g = tcq.bcjr_soft_and_grad(inp, w.L, temp, ones, ws_g, D=Dd)
+                    mark(f"bcjr_soft_vjp_t{temp:g}")
+                    n_launch += 1
+                    outs += [soft, lz, g]
+                    continue
                 soft, lz = tcq.bcjr_soft(inp, w.L, temp, ws_b, D=Dd)
                 mark(f"bcjr_soft_t{temp:g}")
                 n_launch += 1
                 outs += [soft, lz]
-                if "bcjr_grad" in w.ops and i == 0:
-                    g = tcq.bcjr_soft_backward(inp, w.L, temp, soft, ones, ws_g, D=Dd)
-                    mark(f"bcjr_vjp_t{temp:g}")
-                    n_launch += 1
-                    outs.append(g)
         launches_per_step = n_launch
         return outs, ev
 

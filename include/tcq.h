@@ -211,6 +211,23 @@ TCQ_API tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *trellis, const 
                                             void *stream);
 
 /* ------------------------------------------------------------------------
+ * Soft codeword and its vector-Jacobian product in one pass (same
+ * definitions as tcq_bcjr_soft and tcq_bcjr_soft_backward).  For callers that
+ * know the cotangent up front (e.g. the gradient of a fixed loss): one
+ * forward-backward sweep yields soft, log Z and grad_s, where the two
+ * separate calls take two sweeps.  The covariance is centred at the targets
+ * s instead of the soft codeword (an exact identity; only rounding differs).
+ *   grad_soft [n_seq][seq_len] (input); soft, log_z (outputs, each may be
+ *   NULL); grad_s (output).  Workspace: tcq_bcjr_workspace_size(.., 1).
+ *   L = 16 returns TCQ_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------ */
+TCQ_API tcq_status_t tcq_bcjr_soft_and_grad(const tcq_trellis_t *trellis, const float *s,
+                                            const float *D, int64_t n_seq, float temp,
+                                            const float *grad_soft, float *soft, float *log_z,
+                                            float *grad_s, void *ws, size_t ws_bytes,
+                                            void *stream);
+
+/* ------------------------------------------------------------------------
  * Pack walks into bitstreams [QTIP, trellis: the state is a sliding L-bit
  * window over the stream].  Stream bits [k t, k t + k) are the top k bits of
  * state t; a free-start stream ends with the low L-k bits of the last state.

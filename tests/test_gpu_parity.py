@@ -372,3 +372,25 @@ def test_tailbiting_l16_rht_block_pack_decode(tcq):
     rst, rmse, _ = oracle.viterbi_tailbiting_alg4_f32(s[idx], 16)
     assert np.array_equal(st[idx], rst)
     assert abs(float(mse.mean()) - 0.0697) < 0.004               # page: L=16 tail-biting MSE
+
+
+# ---------------------------------------------------------------- soft codeword + VJP in one sweep
+@pytest.mark.parametrize("name,temp,nsample,weighted", [("l12_gauss1024", 0.05, 12, False),
+                                                       ("l8_gauss64", 0.1, 64, True)])
+def test_soft_and_grad_one_sweep(tcq, name, temp, nsample, weighted):
+    w = W.WORKLOADS[name]
+    s = W.sequences(name)
+    D = W.curvature(s.shape[0], 31) if weighted else None
+    v = W.gaussian(s.shape[0], 32)
+    soft, lz, g = tcq.bcjr_soft_and_grad(_dev(s), w.L, temp, _dev(v), D=None if D is None else _dev(D))
+    torch.cuda.synchronize()
+    soft, lz, g = soft.cpu().numpy(), lz.cpu().numpy(), g.cpu().numpy()
+    idx = np.arange(s.shape[0]) if nsample >= s.shape[0] else \
+        np.random.default_rng(9).choice(s.shape[0], nsample, replace=False)
+    Di = None if D is None else D[idx]
+    rg, rsoft = oracle.bcjr_vjp(s[idx], v[idx], w.L, temp, D=Di)
+    _, rlz = oracle.bcjr_soft(s[idx], w.L, temp, D=Di)
+    assert np.abs(soft[idx] - rsoft).max() <= SOFT_ATOL
+    assert np.all(np.abs(lz[idx] - rlz) <= 1e-5 * np.abs(rlz) + 1e-3)
+    for i, j in enumerate(idx):
+        assert np.abs(g[j] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()

@@ -12,6 +12,7 @@ computed" / "Tail-biting is worth its complexity"; BCJR-QAT abstract):
   viterbi_encode_tailbiting(s, L)        -> tail-biting walks (2 bits per weight)
   bcjr_soft(s, L, temp)                  -> (soft f32 [n,T], log_z f32 [n])
   bcjr_soft_backward(s, L, temp, soft, g)-> grad_s f32 [n,T]
+  bcjr_soft_and_grad(s, L, temp, g)      -> (soft, log_z, grad_s) in one sweep
   BcjrSoft.apply(s, L, temp)             -> soft (autograd through the VJP)
   pack_states(states, L, layout)         -> bits uint32 [n, words]
   decode(bits, L, T, layout, ...)        -> fp16 weights
@@ -27,7 +28,7 @@ from ._abi import (FREE_START, OUT_SEQ, OUT_TILE16, TAILBITING, TcqError, check,
                    status_string, trellis)
 
 __all__ = [
-    "viterbi_encode", "viterbi_encode_tailbiting", "bcjr_soft", "bcjr_soft_backward", "BcjrSoft", "pack_states", "decode",
+    "viterbi_encode", "viterbi_encode_tailbiting", "bcjr_soft", "bcjr_soft_and_grad", "bcjr_soft_backward", "BcjrSoft", "pack_states", "decode",
     "stream_words", "viterbi_workspace_size", "bcjr_workspace_size", "TcqError",
     "TAILBITING", "FREE_START", "OUT_SEQ", "OUT_TILE16", "lib", "status_string",
 ]
@@ -153,6 +154,28 @@ def bcjr_soft_backward(s: torch.Tensor, L: int, temp: float, soft: torch.Tensor,
                                        _ptr(soft), _ptr(grad_soft), _ptr(grad), _ptr(ws),
                                        ws.numel(), _stream()), "tcq_bcjr_soft_backward")
     return grad
+
+
+def bcjr_soft_and_grad(s: torch.Tensor, L: int, temp: float, grad_soft: torch.Tensor,
+                       workspace: torch.Tensor | None = None, D: torch.Tensor | None = None):
+    """Soft codeword, log Z and the vector-Jacobian product for a known
+    cotangent ``grad_soft``, in one forward-backward sweep; returns
+    (soft, log_z, grad_s)."""
+    _require_cuda(s, grad_soft)
+    D = _weights(D, s)
+    if s.shape != grad_soft.shape or s.dtype != torch.float32:
+        raise ValueError("s and grad_soft must be float32 tensors of the same shape")
+    n, T = s.shape
+    tr = trellis(L, T)
+    soft = torch.empty_like(s)
+    logz = torch.empty((n,), dtype=torch.float32, device=s.device)
+    grad = torch.empty_like(s)
+    need = int(lib().tcq_bcjr_workspace_size(ctypes.byref(tr), n, 1))
+    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    check(lib().tcq_bcjr_soft_and_grad(ctypes.byref(tr), _ptr(s), _ptr(D), n, float(temp),
+                                       _ptr(grad_soft), _ptr(soft), _ptr(logz), _ptr(grad),
+                                       _ptr(ws), ws.numel(), _stream()), "tcq_bcjr_soft_and_grad")
+    return soft, logz, grad
 
 
 class BcjrSoft(torch.autograd.Function):

@@ -22,7 +22,7 @@ EXPORTS = (
     "tcq_version", "tcq_status_string", "tcq_stream_words",
     "tcq_viterbi_workspace_size", "tcq_viterbi_encode", "tcq_viterbi_encode_noalloc",
     "tcq_viterbi_encode_tailbiting",
-    "tcq_bcjr_workspace_size", "tcq_bcjr_soft", "tcq_bcjr_soft_backward",
+    "tcq_bcjr_workspace_size", "tcq_bcjr_soft", "tcq_bcjr_soft_backward", "tcq_bcjr_soft_and_grad",
     "tcq_pack_states", "tcq_decode",
 )
 
@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
     L.tcq_bcjr_soft.argtypes = [TP, P, P, I64, F, P, P, P, SZ, P]
     L.tcq_bcjr_soft_backward.restype = I
     L.tcq_bcjr_soft_backward.argtypes = [TP, P, P, I64, F, P, P, P, P, SZ, P]
+    L.tcq_bcjr_soft_and_grad.restype = I
+    L.tcq_bcjr_soft_and_grad.argtypes = [TP, P, P, I64, F, P, P, P, P, P, SZ, P]
     L.tcq_pack_states.restype = I
     L.tcq_pack_states.argtypes = [TP, P, I64, I, P, P]
     L.tcq_decode.restype = I

@@ -214,7 +214,9 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       ksm[l * 256 + t] = kappa * ((ok && Dw) ? Dw[sq * T + t] : 1.0f);
       if (GRAD) {
         vsm[l * 256 + t] = ok ? vgrad[sq * T + t] : 0.0f;
-        fsm[l * 256 + t] = ok ? soft_in[sq * T + t] : 0.0f;
+        // centre of the covariance: the forward soft codeword when given,
+        // else the targets themselves (any per-step constant is exact)
+        fsm[l * 256 + t] = ok ? (soft_in ? soft_in[sq * T + t] : s[sq * T + t]) : 0.0f;
       }
     }
     float *V = Vall + ls * NB * NV * NG;
@@ -689,6 +691,31 @@ extern "C" tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *tr, const float *s, c
     case 8: return launch<Soft8>(s, D, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
     case 12: return launch<Soft12>(s, D, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
     default: return launch<Soft16>(s, D, n_seq, T, kappa, tot, nullptr, nullptr, soft, log_z, nullptr, ws, ws_bytes, strm);
+  }
+}
+
+extern "C" tcq_status_t tcq_bcjr_soft_and_grad(const tcq_trellis_t *tr, const float *s,
+                                               const float *D, int64_t n_seq, float temp,
+                                               const float *grad_soft, float *soft,
+                                               float *log_z, float *grad_s, void *ws,
+                                               size_t ws_bytes, void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if (tr->L == 16) return TCQ_ERR_UNSUPPORTED;
+  if (!temp_ok(temp)) return TCQ_ERR_INVALID_ARG;
+  if (n_seq < 0 || n_seq > (int64_t)INT32_MAX) return TCQ_ERR_INVALID_ARG;
+  if (n_seq == 0) return TCQ_OK;
+  if (!s || !grad_soft || !grad_s || !aligned16(s) || !aligned16(grad_soft) || !aligned16(grad_s) ||
+      (soft && !aligned16(soft)) || (log_z && !aligned16(log_z)) || (D && !aligned16(D)))
+    return TCQ_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
+  const float kappa = (float)(1.4426950408889634 / (double)temp);
+  const float tot = (float)(2.0 / (double)temp);
+  cudaStream_t strm = (cudaStream_t)stream;
+  const int T = tr->seq_len;
+  switch (tr->L) {
+    case 8: return launch<Grad8>(s, D, n_seq, T, kappa, tot, grad_soft, nullptr, soft, log_z, grad_s, ws, ws_bytes, strm);
+    default: return launch<Grad12>(s, D, n_seq, T, kappa, tot, grad_soft, nullptr, soft, log_z, grad_s, ws, ws_bytes, strm);
   }
 }
 

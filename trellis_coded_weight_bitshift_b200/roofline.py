@@ -38,6 +38,9 @@ MUFU_PER_SM = 16               # special-function results per clock per SM
 # null.  (kernel prefix, workload): (bytes, sequences in the capture, sources)
 _CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 MEASURED_TRAFFIC = {
+    ("bcjr_soft_vjp", "l12_gauss1024"): (2.142159e9 + 2.176458e9, 1024, {
+        "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
+        "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
     ("bcjr_vjp", "l12_gauss1024"): (2.142159e9 + 2.176458e9, 1024, {
         "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
         "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
@@ -88,7 +91,7 @@ def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str,
         return "alu", 2 * n_seq * T * states * 4.5, "lane-ops"
     if kernel.startswith("viterbi"):
         return "alu", n_seq * T * states * 4.5, "lane-ops"
-    if kernel.startswith("bcjr_vjp"):
+    if kernel.startswith("bcjr_vjp") or kernel.startswith("bcjr_soft_vjp"):
         return "alu", n_seq * T * states * 11 / 4, "mufu-ops"
     if kernel.startswith("bcjr"):
         return "alu", n_seq * T * states * 9 / 4, "mufu-ops"
