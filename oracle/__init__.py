@@ -397,3 +397,27 @@ def pack(states: np.ndarray, L: int, layout: int, k: int = 2) -> np.ndarray:
             bits[:, k * (T - 1) + i] = (states[:, T - 1] >> (L - 1 - i)) & 1
     assert nb <= nw * 32
     return _bits_to_words(bits)
+
+
+# --------------------------------------------------------------------------
+# Random-sign Hadamard rotation (QTIP blog, "The trellis: a stateful codebook":
+# random signs, then a Hadamard matrix, on both sides of W -- from QuIP#).
+# --------------------------------------------------------------------------
+def hadamard(n: int) -> np.ndarray:
+    """Sylvester Hadamard matrix H_n (n a power of two): H_1 = [1],
+    H_2m = [[H_m, H_m], [H_m, -H_m]]."""
+    assert n >= 1 and n & (n - 1) == 0
+    h = np.array([[1.0]])
+    while h.shape[0] < n:
+        h = np.kron(np.array([[1.0, 1.0], [1.0, -1.0]]), h)
+    return h
+
+
+def rht(W: np.ndarray, sign_rows: np.ndarray, sign_cols: np.ndarray) -> np.ndarray:
+    """(H_R / sqrt R) diag(sign_rows) W diag(sign_cols) (H_C / sqrt C), fp64,
+    by dense matrix products (the definition)."""
+    W = np.asarray(W, dtype=np.float64)
+    R, C = W.shape
+    hr, hc = hadamard(R), hadamard(C)
+    return (hr @ (np.asarray(sign_rows, np.float64)[:, None] * W * np.asarray(sign_cols, np.float64)[None, :])
+            @ hc) / np.sqrt(R * C)
