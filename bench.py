@@ -51,6 +51,8 @@ def _args():
 
 
 def _metric_for(w: W.Workload) -> str:
+    if w.ops == ("rht",):
+        return "rotated weights/sec (random-sign Hadamard rotation, both sides, fp32)"
     if w.ops == ("decode",):
         return "decoded weights/sec (2-bit tail-biting stream -> fp16, 16x16 tiles)"
     parts = []
@@ -153,11 +155,34 @@ def _oracle_decode_step(bits: np.ndarray, w: W.Workload) -> None:
     oracle.decode(bits, w.L, 256, oracle.TAILBITING)
 
 
+_RHT_SAMPLE = (256, 1024)     # leading block the oracle rotates by its dense definition
+
+
+def _oracle_rht_sample(w: W.Workload) -> int:
+    """Dense-definition rotation of the leading 256 x 1024 block of the
+    workload's matrix (its own 256- and 1024-point transforms); returns the
+    weights rotated."""
+    import oracle
+    Wm, s1, s2 = W.rotation_input(w.name)
+    r, c = _RHT_SAMPLE
+    oracle.rht(Wm[:r, :c], s1[:r], s2[:c])
+    return r * c
+
+
 def cpu_baseline(w: W.Workload, budget_s: float = 12.0) -> dict:
     """Time the oracle, as it stands, on a bounded sample of the workload."""
     import oracle
     oracle.build()
     n_done, t0 = 0, time.perf_counter()
+    if w.ops == ("rht",):
+        done = 0
+        while time.perf_counter() - t0 < 2.0:
+            done += _oracle_rht_sample(w)
+        dt = time.perf_counter() - t0
+        return {"value": done / dt, "unit": "weights/s", "cores": os.cpu_count(), "kind": "oracle",
+                "sample": f"dense-definition rotation of the leading {_RHT_SAMPLE[0]} x "
+                          f"{_RHT_SAMPLE[1]} block of {w.name} (numpy matmul, all BLAS threads), "
+                          f"{dt:.1f} s wall"}
     if w.ops == ("decode",):
         bits = W.streams(w.name)
         chunk = 1024
@@ -185,6 +210,25 @@ def run_reference(a) -> None:
     oracle.build()
     per_step = 4 if w.ops != ("decode",) else 1024        # sequences per bounded step
     wts = None
+    if w.ops == ("rht",):
+        times = []
+        for i in range(a.warmup + a.steps):
+            t0 = time.perf_counter()
+            done = _oracle_rht_sample(w)
+            if i >= a.warmup:
+                times.append(time.perf_counter() - t0)
+        step_s = sum(times) / len(times)
+        value = done / step_s
+        print(json.dumps({
+            "impl": "reference", "metric": _metric_for(w), "value": value, "unit": "weights/s",
+            "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "rows": w.rows, "cols": w.cols},
+            "cpu_baseline": {"value": value, "unit": "weights/s", "cores": os.cpu_count(),
+                             "kind": "oracle", "sample": "leading 256 x 1024 block per step"},
+            "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
     if w.ops == ("decode",):
         data = W.streams(w.name)[: per_step * (a.steps + a.warmup)]
     else:
@@ -224,6 +268,8 @@ def rank_batch(w: W.Workload, rank: int) -> np.ndarray:
     """The batch rank `rank` encodes (weak scaling: every rank a batch of the
     workload's size, no data exchanged).  Rank 0 gets the workload itself;
     other ranks get draws of the same distribution from seed + 1000 * rank."""
+    if w.ops == ("rht",):
+        return W.student_t_block(w.seed + 1000 * rank, w.rows, w.cols)
     if w.ops == ("decode",):
         return W.bitstream(w.n_seq, w.seed + 1000 * rank)
     if rank == 0 or w.kind != "gaussian":
@@ -277,6 +323,10 @@ def run_ours(a) -> None:
     else:
         x = torch.from_numpy(host).to(dev)
     h2d_bytes = host.nbytes
+    if w.ops == ("rht",):
+        _, s1h, s2h = W.rotation_input(w.name)
+        sr, sc = torch.from_numpy(s1h).to(dev), torch.from_numpy(s2h).to(dev)
+        rot_out = torch.empty_like(x)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
@@ -306,7 +356,13 @@ def run_ours(a) -> None:
                 e.record(stream)
                 ev.append((name, e))
 
-        if w.ops == ("decode",):
+        if w.ops == ("rht",):
+            mark("start")
+            out = tcq.rht(inp, sr, sc, out=rot_out)
+            mark("rht")
+            n_launch += 3
+            outs.append(out)
+        elif w.ops == ("decode",):
             mark("start")
             out = tcq.decode(inp, w.L, 256, tcq.TAILBITING, tcq.OUT_TILE16, w.rows, w.cols)
             mark("decode_tile16")

@@ -250,6 +250,21 @@ TCQ_API tcq_status_t tcq_decode(const tcq_trellis_t *trellis, const uint32_t *bi
                         int layout, int out_layout, int64_t rows, int64_t cols,
                         uint16_t *out, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Random-sign Hadamard rotation [QTIP, trellis section: random signs, then a
+ * Hadamard matrix, on both sides of W, so that one data-independent code fits
+ * every layer]:
+ *   out = (H_R / sqrt R) diag(sign_rows) W diag(sign_cols) (H_C / sqrt C)
+ * with H_n the Sylvester Hadamard matrix (H_n[i][j] = (-1)^popcount(i & j)).
+ *   W [rows][cols] fp32 (input), out [rows][cols] fp32 (output; may equal W),
+ *   sign_rows [rows], sign_cols [cols] fp32 (+-1 expected; any values are
+ *   applied as multipliers).  rows, cols powers of two, 32 <= cols <= 8192,
+ *   32 <= rows <= 2^20.  fp32 butterflies; error ~ log2(rows*cols) rounding
+ *   steps of the partial sums.
+ * ------------------------------------------------------------------------ */
+TCQ_API tcq_status_t tcq_rht(const float *W, int64_t rows, int64_t cols, const float *sign_rows,
+                             const float *sign_cols, float *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

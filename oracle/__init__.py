@@ -421,3 +421,29 @@ def rht(W: np.ndarray, sign_rows: np.ndarray, sign_cols: np.ndarray) -> np.ndarr
     hr, hc = hadamard(R), hadamard(C)
     return (hr @ (np.asarray(sign_rows, np.float64)[:, None] * W * np.asarray(sign_cols, np.float64)[None, :])
             @ hc) / np.sqrt(R * C)
+
+
+def hadamard_entry(i, j):
+    """Closed form of the Sylvester matrix: H[i][j] = (-1)^popcount(i & j)."""
+    x = np.bitwise_and(np.asarray(i, dtype=np.int64), np.asarray(j, dtype=np.int64))
+    pc = np.zeros_like(x)
+    while np.any(x):
+        pc += x & 1
+        x >>= 1
+    return 1.0 - 2.0 * (pc & 1)
+
+
+def rht_entries(W: np.ndarray, sign_rows, sign_cols, rows_idx, cols_idx) -> np.ndarray:
+    """Selected entries of the rotation, each by its definition:
+    out[i, j] = sum_{r,c} H_R[i,r] s1[r] W[r,c] s2[c] H_C[c,j] / sqrt(R C)."""
+    W = np.asarray(W, dtype=np.float64)
+    R, C = W.shape
+    s1 = np.asarray(sign_rows, np.float64)
+    s2 = np.asarray(sign_cols, np.float64)
+    rr, cc = np.arange(R), np.arange(C)
+    out = np.empty((len(rows_idx), len(cols_idx)))
+    for b, j in enumerate(cols_idx):
+        u = W @ (s2 * hadamard_entry(cc, j))                      # [R]
+        for a, i in enumerate(rows_idx):
+            out[a, b] = np.dot(hadamard_entry(i, rr) * s1, u)
+    return out / np.sqrt(R * C)

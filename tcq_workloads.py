@@ -58,6 +58,9 @@ WORKLOADS = {
     # "Cliff edges"); D log-uniform on [0.1, 10] from seed 6
     "l12_curv1024": Workload("l12_curv1024", 12, 1024, "gaussian", 2, (0.05,),
                              ops=("viterbi", "bcjr", "bcjr_grad"), curv_seed=6),
+    # random-sign Hadamard rotation of an 8192x8192 Student-t (nu = 5) block
+    "rht_t5_8192sq": Workload("rht_t5_8192sq", 16, 262144, "matrix_t5", 7, (), 8192, 8192,
+                              ops=("rht",)),
     # the 1024x1024 RHT block encoded tail-biting (exactly 2 bits per weight)
     "l16_rht1024_tb": Workload("l16_rht1024_tb", 16, 4096, "rht_block", 3, (), 1024, 1024,
                                ops=("viterbi_tb",)),
@@ -137,6 +140,17 @@ def sequences(name: str, n_limit: int | None = None) -> np.ndarray:
     else:
         raise ValueError(f"{name} is a bitstream workload")
     return out if n_limit is None else np.ascontiguousarray(out[:n_limit])
+
+
+def rotation_input(name: str):
+    """(W [rows, cols] fp32, sign_rows, sign_cols) of a rotation workload."""
+    w = WORKLOADS[name]
+    assert w.kind == "matrix_t5"
+    W = student_t_block(w.seed, w.rows, w.cols)
+    rng = np.random.default_rng(w.seed + 100)
+    s1 = (rng.integers(0, 2, w.rows) * 2 - 1).astype(np.float32)
+    s2 = (rng.integers(0, 2, w.cols) * 2 - 1).astype(np.float32)
+    return W, s1, s2
 
 
 def streams(name: str) -> np.ndarray:

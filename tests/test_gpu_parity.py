@@ -394,3 +394,40 @@ def test_soft_and_grad_one_sweep(tcq, name, temp, nsample, weighted):
     assert np.all(np.abs(lz[idx] - rlz) <= 1e-5 * np.abs(rlz) + 1e-3)
     for i, j in enumerate(idx):
         assert np.abs(g[j] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+
+
+# ---------------------------------------------------------------- random-sign Hadamard rotation
+RHT_ATOL = 2e-5      # ~log2(R*C) fp32 rounding steps on partial sums of unit-variance data
+
+
+def _signs(n, seed):
+    return (np.random.default_rng(seed).integers(0, 2, n) * 2 - 1).astype(np.float32)
+
+
+@pytest.mark.parametrize("R,C", [(1024, 1024), (32, 8192), (8192, 32), (256, 64)])
+def test_rht_matches_dense_definition(tcq, R, C):
+    W = W_ = np.random.default_rng(R * 3 + C).standard_normal((R, C)).astype(np.float32)
+    s1, s2 = _signs(R, R), _signs(C, C + 1)
+    out = tcq.rht(_dev(W), _dev(s1), _dev(s2)).cpu().numpy()
+    ref = oracle.rht(W_, s1, s2) if R * C <= 1 << 20 else None
+    if ref is None:
+        ri = np.random.default_rng(1).choice(R, 6, replace=False)
+        ci = np.random.default_rng(2).choice(C, 6, replace=False)
+        ref = oracle.rht_entries(W_, s1, s2, ri, ci)
+        out = out[ri][:, ci]
+    assert np.abs(out - ref).max() <= RHT_ATOL
+
+
+def test_rht_in_place_and_8192_square_sampled(tcq):
+    R = C = 8192
+    W = np.random.default_rng(11).standard_t(5, (R, C)).astype(np.float32)
+    s1, s2 = _signs(R, 12), _signs(C, 13)
+    d = _dev(W)
+    tcq.rht(d, _dev(s1), _dev(s2), out=d)                        # in place
+    torch.cuda.synchronize()
+    got = d.cpu().numpy()
+    ri = np.array([0, 1, 4095, 8191])
+    ci = np.array([0, 77, 8190])
+    ref = oracle.rht_entries(W, s1, s2, ri, ci)
+    assert np.abs(got[ri][:, ci] - ref).max() <= 4 * RHT_ATOL * np.sqrt(5 / 3)
+    assert abs(float(np.linalg.norm(got.astype(np.float64))) / float(np.linalg.norm(W.astype(np.float64))) - 1) < 1e-5

@@ -57,3 +57,15 @@ def test_rht_gaussianises_heavy_tails():
     kurt = lambda a: np.mean((a - a.mean()) ** 4) / np.var(a) ** 2
     assert kurt(W) > 6
     assert abs(kurt(Y) - 3.0) < 0.2
+
+
+def test_closed_form_entries_match_the_kronecker_construction():
+    h = oracle.hadamard(64)
+    i, j = np.meshgrid(np.arange(64), np.arange(64), indexing="ij")
+    assert np.array_equal(oracle.hadamard_entry(i, j), h)
+    rng = np.random.default_rng(3)
+    W = rng.standard_normal((64, 32))
+    s1 = rng.integers(0, 2, 64) * 2.0 - 1
+    s2 = rng.integers(0, 2, 32) * 2.0 - 1
+    np.testing.assert_allclose(oracle.rht_entries(W, s1, s2, [0, 5, 63], [1, 31]),
+                               oracle.rht(W, s1, s2)[[0, 5, 63]][:, [1, 31]], atol=1e-12)

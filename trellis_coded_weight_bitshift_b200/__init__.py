@@ -16,6 +16,7 @@ computed" / "Tail-biting is worth its complexity"; BCJR-QAT abstract):
   BcjrSoft.apply(s, L, temp)             -> soft (autograd through the VJP)
   pack_states(states, L, layout)         -> bits uint32 [n, words]
   decode(bits, L, T, layout, ...)        -> fp16 weights
+  rht(W, sign_rows, sign_cols)           -> random-sign Hadamard rotation of W
 """
 from __future__ import annotations
 
@@ -29,7 +30,7 @@ from ._abi import (FREE_START, OUT_SEQ, OUT_TILE16, TAILBITING, TcqError, check,
 
 __all__ = [
     "viterbi_encode", "viterbi_encode_tailbiting", "bcjr_soft", "bcjr_soft_and_grad", "bcjr_soft_backward", "BcjrSoft", "pack_states", "decode",
-    "stream_words", "viterbi_workspace_size", "bcjr_workspace_size", "TcqError",
+    "stream_words", "viterbi_workspace_size", "bcjr_workspace_size", "TcqError", "rht",
     "TAILBITING", "FREE_START", "OUT_SEQ", "OUT_TILE16", "lib", "status_string",
 ]
 
@@ -231,4 +232,21 @@ def decode(bits: torch.Tensor, L: int, seq_len: int = 256, layout: int = TAILBIT
     _require_cuda(out)
     check(lib().tcq_decode(ctypes.byref(tr), _ptr(bits), n, int(layout), int(out_layout), int(rows),
                            int(cols), _ptr(out), _stream()), "tcq_decode")
+    return out
+
+
+def rht(W: torch.Tensor, sign_rows: torch.Tensor, sign_cols: torch.Tensor,
+        out: torch.Tensor | None = None) -> torch.Tensor:
+    """Random-sign Hadamard rotation (H_R/sqrt R) diag(sign_rows) W
+    diag(sign_cols) (H_C/sqrt C) of a fp32 matrix (``out`` may be ``W``)."""
+    _require_cuda(W, sign_rows, sign_cols)
+    if W.dim() != 2 or W.dtype != torch.float32:
+        raise ValueError("W must be a 2-D float32 tensor")
+    R, C = W.shape
+    if sign_rows.shape != (R,) or sign_cols.shape != (C,):
+        raise ValueError("sign vectors must match W's rows and columns")
+    out = torch.empty_like(W) if out is None else out
+    _require_cuda(out)
+    check(lib().tcq_rht(_ptr(W), R, C, _ptr(sign_rows.float().contiguous()),
+                        _ptr(sign_cols.float().contiguous()), _ptr(out), _stream()), "tcq_rht")
     return out

@@ -38,18 +38,13 @@ MUFU_PER_SM = 16               # special-function results per clock per SM
 # null.  (kernel prefix, workload): (bytes, sequences in the capture, sources)
 _CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 MEASURED_TRAFFIC = {
-    ("bcjr_soft_vjp", "l12_gauss1024"): (2.142159e9 + 2.176458e9, 1024, {
-        "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
+    ("bcjr_soft_vjp", "l12_gauss1024"): (2.139645e9 + 2.179336e9, 1024, {
+        "tcq_bcjr.cu": "96df19e5969718a26fb330fe71505390f1840110",
         "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
-    ("bcjr_vjp", "l12_gauss1024"): (2.142159e9 + 2.176458e9, 1024, {
-        "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
-        "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
-    ("bcjr_soft", "l12_gauss1024"): (1.020003e9 + 1.082902e9, 1024, {
-        "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
-        "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
-    # captured on the first 64 sequences; traffic scales with the sequences
-    ("bcjr_soft", "l16_studentt_2048x8192"): (0.99031168e9 + 1.080753e9, 64, {
-        "tcq_bcjr.cu": "1c21156a97de271bb2349030f97d2aac7083db3d",
+    # three launches (row pass, two column passes) of one 8192 x 8192 rotation
+    ("rht", "rht_t5_8192sq"): (268.563712e6 + 223.412224e6 + 268.515328e6 + 209.742592e6
+                               + 268.464896e6 + 209.4656e6, 262144, {
+        "tcq_rht.cu": "ccfacb475702414c5cd2f49317f76388abbd2f52",
         "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
 }
 
@@ -87,6 +82,8 @@ def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str,
     states = float(1 << L)
     if kernel.startswith("decode"):
         return "hbm", n_seq * (T * 2 / 8 + T * 2), "bytes"
+    if kernel.startswith("rht"):            # read W once, write the rotation once (fp32)
+        return "hbm", n_seq * T * 8.0, "bytes"
     if kernel.startswith("viterbi_tb"):       # two Viterbi runs
         return "alu", 2 * n_seq * T * states * 4.5, "lane-ops"
     if kernel.startswith("viterbi"):
