@@ -51,6 +51,8 @@ def _args():
 
 
 def _metric_for(w: W.Workload) -> str:
+    if w.ops == ("gemv",):
+        return "decoded weights/sec in a batch-1 GEMV (2-bit stream decoded in registers)"
     if w.ops == ("rht",):
         return "rotated weights/sec (random-sign Hadamard rotation, both sides, fp32)"
     if w.ops == ("decode",):
@@ -152,6 +154,12 @@ def _oracle_step(w: W.Workload, s: np.ndarray, D=None) -> None:
 
 def _oracle_decode_step(bits: np.ndarray, w: W.Workload) -> None:
     import oracle
+    if w.ops == ("gemv",):          # one band of tile-rows: decode, then the matvec
+        nc = w.cols // 16
+        bands = bits.shape[0] // nc
+        x = W.gemv_vector(w.name).astype(np.float64)
+        oracle.decode_tiles(bits[: bands * nc], 16 * bands, w.cols, L=w.L).astype(np.float64) @ x
+        return
     oracle.decode(bits, w.L, 256, oracle.TAILBITING)
 
 
@@ -183,7 +191,7 @@ def cpu_baseline(w: W.Workload, budget_s: float = 12.0) -> dict:
                 "sample": f"dense-definition rotation of the leading {_RHT_SAMPLE[0]} x "
                           f"{_RHT_SAMPLE[1]} block of {w.name} (numpy matmul, all BLAS threads), "
                           f"{dt:.1f} s wall"}
-    if w.ops == ("decode",):
+    if w.ops in (("decode",), ("gemv",)):
         bits = W.streams(w.name)
         chunk = 1024
         while time.perf_counter() - t0 < budget_s and n_done + chunk <= bits.shape[0]:
@@ -208,7 +216,7 @@ def run_reference(a) -> None:
     w = W.WORKLOADS[a.workload]
     import oracle
     oracle.build()
-    per_step = 4 if w.ops != ("decode",) else 1024        # sequences per bounded step
+    per_step = 1024 if w.ops in (("decode",), ("gemv",)) else 4   # sequences per bounded step
     wts = None
     if w.ops == ("rht",):
         times = []
@@ -229,7 +237,7 @@ def run_reference(a) -> None:
             "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}))
         return
-    if w.ops == ("decode",):
+    if w.ops in (("decode",), ("gemv",)):
         data = W.streams(w.name)[: per_step * (a.steps + a.warmup)]
     else:
         data = W.sequences(w.name, n_limit=min(w.n_seq, per_step * (a.steps + a.warmup)))
@@ -241,7 +249,7 @@ def run_reference(a) -> None:
         chunk = data[lo: lo + per_step]
         pos += per_step
         t0 = time.perf_counter()
-        if w.ops == ("decode",):
+        if w.ops in (("decode",), ("gemv",)):
             _oracle_decode_step(chunk, w)
         else:
             _oracle_step(w, chunk, None if wts is None else wts[lo: lo + per_step])
@@ -270,7 +278,7 @@ def rank_batch(w: W.Workload, rank: int) -> np.ndarray:
     other ranks get draws of the same distribution from seed + 1000 * rank."""
     if w.ops == ("rht",):
         return W.student_t_block(w.seed + 1000 * rank, w.rows, w.cols)
-    if w.ops == ("decode",):
+    if w.ops in (("decode",), ("gemv",)):
         return W.bitstream(w.n_seq, w.seed + 1000 * rank)
     if rank == 0 or w.kind != "gaussian":
         return W.sequences(w.name, n_limit=w.n_seq)
@@ -318,11 +326,14 @@ def run_ours(a) -> None:
 
     # ---- inputs (each rank its own batch) ----
     host = rank_batch(w, rank)
-    if w.ops == ("decode",):
+    if w.ops in (("decode",), ("gemv",)):
         x = torch.from_numpy(host.view(np.int32)).to(dev).view(torch.uint32)
     else:
         x = torch.from_numpy(host).to(dev)
     h2d_bytes = host.nbytes
+    if w.ops == ("gemv",):
+        xvec = torch.from_numpy(W.gemv_vector(w.name)).to(dev)
+        yvec = torch.empty((w.rows,), dtype=torch.float32, device=dev)
     if w.ops == ("rht",):
         _, s1h, s2h = W.rotation_input(w.name)
         sr, sc = torch.from_numpy(s1h).to(dev), torch.from_numpy(s2h).to(dev)
@@ -356,7 +367,13 @@ def run_ours(a) -> None:
                 e.record(stream)
                 ev.append((name, e))
 
-        if w.ops == ("rht",):
+        if w.ops == ("gemv",):
+            mark("start")
+            out = tcq.decode_gemv(inp, xvec, w.rows, w.cols, L=w.L, out=yvec)
+            mark("decode_gemv")
+            n_launch += 1
+            outs.append(out)
+        elif w.ops == ("rht",):
             mark("start")
             out = tcq.rht(inp, sr, sc, out=rot_out)
             mark("rht")
@@ -421,7 +438,8 @@ def run_ours(a) -> None:
     mean_ms = max_over_ranks(sum(step_ms) / len(step_ms), dist, dev)
 
     # ---- end to end through the public API with host buffers ----
-    pinned = torch.from_numpy(host.view(np.int32) if w.ops == ("decode",) else host).pin_memory()
+    as_words = w.ops in (("decode",), ("gemv",))
+    pinned = torch.from_numpy(host.view(np.int32) if as_words else host).pin_memory()
     e2e_ms = []
     d2h_bytes = 0
     for i in range(a.warmup + a.steps):
@@ -429,7 +447,7 @@ def run_ours(a) -> None:
         e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         inp = pinned.to(dev, non_blocking=True)
-        if w.ops == ("decode",):
+        if as_words:
             inp = inp.view(torch.uint32)
         outs, _ = step(inp, False)
         host_outs = []

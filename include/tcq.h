@@ -251,6 +251,21 @@ TCQ_API tcq_status_t tcq_decode(const tcq_trellis_t *trellis, const uint32_t *bi
                         uint16_t *out, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Decode fused into a matrix-vector product [QTIP, "What it buys end to end":
+ * each 16x16 tile decodes straight into the matmul operand]:
+ *   y[i] = sum_j W[i][j] x[j],  W [rows][cols] = the fp16 matrix that
+ *   tcq_decode(.., TCQ_OUT_TILE16, rows, cols) produces from `bits`,
+ * products and sums in fp32 (summation order unspecified).  The weights are
+ * decoded in registers and never written.
+ *   bits [rows/16 * cols/16][tcq_stream_words()] (input), x [cols] fp32
+ *   (input), y [rows] fp32 (output; zeroed, then accumulated with atomics on
+ *   `stream`).  seq_len must be 256.
+ * ------------------------------------------------------------------------ */
+TCQ_API tcq_status_t tcq_decode_gemv(const tcq_trellis_t *trellis, const uint32_t *bits, int layout,
+                                     int64_t rows, int64_t cols, const float *x, float *y,
+                                     void *stream);
+
+/* ------------------------------------------------------------------------
  * Random-sign Hadamard rotation [QTIP, trellis section: random signs, then a
  * Hadamard matrix, on both sides of W, so that one data-independent code fits
  * every layer]:

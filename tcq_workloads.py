@@ -58,6 +58,9 @@ WORKLOADS = {
     # "Cliff edges"); D log-uniform on [0.1, 10] from seed 6
     "l12_curv1024": Workload("l12_curv1024", 12, 1024, "gaussian", 2, (0.05,),
                              ops=("viterbi", "bcjr", "bcjr_grad"), curv_seed=6),
+    # decode fused into a batch-1 GEMV: the 8192^2 stream of l16_decode_8192sq, x from seed 8
+    "l16_gemv_8192sq": Workload("l16_gemv_8192sq", 16, 262144, "bitstream", 5, (), 8192, 8192,
+                                ops=("gemv",)),
     # random-sign Hadamard rotation of an 8192x8192 Student-t (nu = 5) block
     "rht_t5_8192sq": Workload("rht_t5_8192sq", 16, 262144, "matrix_t5", 7, (), 8192, 8192,
                               ops=("rht",)),
@@ -151,6 +154,11 @@ def rotation_input(name: str):
     s1 = (rng.integers(0, 2, w.rows) * 2 - 1).astype(np.float32)
     s2 = (rng.integers(0, 2, w.cols) * 2 - 1).astype(np.float32)
     return W, s1, s2
+
+
+def gemv_vector(name: str) -> np.ndarray:
+    w = WORKLOADS[name]
+    return np.random.default_rng(8).standard_normal(w.cols).astype(np.float32)
 
 
 def streams(name: str) -> np.ndarray:

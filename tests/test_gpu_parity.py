@@ -431,3 +431,43 @@ def test_rht_in_place_and_8192_square_sampled(tcq):
     ref = oracle.rht_entries(W, s1, s2, ri, ci)
     assert np.abs(got[ri][:, ci] - ref).max() <= 4 * RHT_ATOL * np.sqrt(5 / 3)
     assert abs(float(np.linalg.norm(got.astype(np.float64))) / float(np.linalg.norm(W.astype(np.float64))) - 1) < 1e-5
+
+
+# ---------------------------------------------------------------- decode fused into a GEMV
+def _gemv_ref(bits, rows, cols, x, L=16, layout=0, tile_rows=None):
+    """fp64 y = W x from the oracle's fp16 decode, and the rigorous fp32
+    summation bound (cols + 1) 2^-24 sum_j |W_ij x_j| for each row."""
+    nc = cols // 16
+    if tile_rows is None:
+        Wm = oracle.decode_tiles(bits, rows, cols, L=L, layout=layout).astype(np.float64)
+        terms = Wm * x[None, :].astype(np.float64)
+        return terms.sum(1), (cols + 1) * 2.0 ** -24 * np.abs(terms).sum(1)
+    ys, bs = [], []
+    for R in tile_rows:
+        blk = oracle.decode_tiles(bits[R * nc:(R + 1) * nc], 16, cols, L=L, layout=layout).astype(np.float64)
+        terms = blk * x[None, :].astype(np.float64)
+        ys.append(terms.sum(1)); bs.append((cols + 1) * 2.0 ** -24 * np.abs(terms).sum(1))
+    return np.concatenate(ys), np.concatenate(bs)
+
+
+@pytest.mark.parametrize("L,layout,rows,cols", [(16, 0, 256, 512), (8, 1, 96, 160), (12, 0, 1024, 2048)])
+def test_decode_gemv_matches_oracle(tcq, L, layout, rows, cols):
+    rng = np.random.default_rng(rows + cols + L)
+    n = (rows // 16) * (cols // 16)
+    nw = oracle.stream_words(L, 2, 256, layout)
+    bits = rng.integers(0, 2 ** 32, (n, nw), dtype=np.uint32)
+    x = rng.standard_normal(cols).astype(np.float32)
+    y = tcq.decode_gemv(_dev(bits.view(np.int32)).view(torch.uint32), _dev(x), rows, cols, L=L,
+                        layout=layout).cpu().numpy()
+    ref, bound = _gemv_ref(bits, rows, cols, x, L=L, layout=layout)
+    assert np.all(np.abs(y - ref) <= bound + 1e-30)
+
+
+def test_decode_gemv_8192_square_sampled_rows(tcq):
+    bits = W.streams("l16_decode_8192sq")
+    x = np.random.default_rng(8).standard_normal(8192).astype(np.float32)
+    y = tcq.decode_gemv(_dev(bits.view(np.int32)).view(torch.uint32), _dev(x), 8192, 8192).cpu().numpy()
+    trs = [0, 1, 255, 511]
+    ref, bound = _gemv_ref(bits, 8192, 8192, x, tile_rows=trs)
+    got = np.concatenate([y[16 * R:16 * R + 16] for R in trs])
+    assert np.all(np.abs(got - ref) <= bound)

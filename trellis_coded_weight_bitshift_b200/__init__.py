@@ -31,6 +31,7 @@ from ._abi import (FREE_START, OUT_SEQ, OUT_TILE16, TAILBITING, TcqError, check,
 __all__ = [
     "viterbi_encode", "viterbi_encode_tailbiting", "bcjr_soft", "bcjr_soft_and_grad", "bcjr_soft_backward", "BcjrSoft", "pack_states", "decode",
     "stream_words", "viterbi_workspace_size", "bcjr_workspace_size", "TcqError", "rht",
+    "decode_gemv",
     "TAILBITING", "FREE_START", "OUT_SEQ", "OUT_TILE16", "lib", "status_string",
 ]
 
@@ -250,3 +251,20 @@ def rht(W: torch.Tensor, sign_rows: torch.Tensor, sign_cols: torch.Tensor,
     check(lib().tcq_rht(_ptr(W), R, C, _ptr(sign_rows.float().contiguous()),
                         _ptr(sign_cols.float().contiguous()), _ptr(out), _stream()), "tcq_rht")
     return out
+
+
+def decode_gemv(bits: torch.Tensor, x: torch.Tensor, rows: int, cols: int, L: int = 16,
+                layout: int = TAILBITING, out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = W x with W the fp16 matrix decoded from 16x16-tile streams ``bits``,
+    decoded in registers (never materialised); fp32 products and sums."""
+    _require_cuda(bits, x)
+    if bits.dtype != torch.uint32 or x.dtype != torch.float32 or x.shape != (cols,):
+        raise ValueError("bits must be uint32 [tiles, words] and x float32 [cols]")
+    tr = trellis(L, 256)
+    words = int(lib().tcq_stream_words(ctypes.byref(tr), int(layout)))
+    if bits.shape != ((rows // 16) * (cols // 16), words):
+        raise ValueError("bits must hold one stream per 16x16 tile")
+    y = torch.empty((rows,), dtype=torch.float32, device=x.device) if out is None else out
+    check(lib().tcq_decode_gemv(ctypes.byref(tr), _ptr(bits), int(layout), int(rows), int(cols),
+                                _ptr(x), _ptr(y), _stream()), "tcq_decode_gemv")
+    return y

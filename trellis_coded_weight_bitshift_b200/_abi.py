@@ -23,7 +23,7 @@ EXPORTS = (
     "tcq_viterbi_workspace_size", "tcq_viterbi_encode", "tcq_viterbi_encode_noalloc",
     "tcq_viterbi_encode_tailbiting",
     "tcq_bcjr_workspace_size", "tcq_bcjr_soft", "tcq_bcjr_soft_backward", "tcq_bcjr_soft_and_grad",
-    "tcq_pack_states", "tcq_decode", "tcq_rht",
+    "tcq_pack_states", "tcq_decode", "tcq_decode_gemv", "tcq_rht",
 )
 
 
@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
     L.tcq_bcjr_soft_and_grad.argtypes = [TP, P, P, I64, F, P, P, P, P, P, SZ, P]
     L.tcq_pack_states.restype = I
     L.tcq_pack_states.argtypes = [TP, P, I64, I, P, P]
+    L.tcq_decode_gemv.restype = I
+    L.tcq_decode_gemv.argtypes = [TP, P, I, I64, I64, P, P, P]
     L.tcq_rht.restype = I
     L.tcq_rht.argtypes = [P, I64, I64, P, P, P, P]
     L.tcq_decode.restype = I

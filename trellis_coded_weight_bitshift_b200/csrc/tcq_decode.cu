@@ -219,3 +219,119 @@ extern "C" tcq_status_t tcq_decode(const tcq_trellis_t *tr, const uint32_t *bits
     default: return decode_launch<16>(tr, bits, n_seq, layout, out_layout, rows, cols, out, s, (int)wps);
   }
 }
+
+// ---------------------------------------------------------------------------
+// Decode fused into a matrix-vector product [QTIP blog, "What it buys end to
+// end": each 16x16 tile is one 256-weight sequence that decodes straight into
+// the matmul operand, so the weights never exist in memory at 16 bits].
+//   y[i] = sum_j W[i][j] x[j],  W = the fp16 matrix tcq_decode (TILE16) gives,
+// accumulated in fp32.  A warp takes a run of tiles along one tile-row; lane
+// (r, h) decodes the 8 weights of row r, half h of each tile, rounds them to
+// fp16 exactly as the decode does, multiplies by x and accumulates; the two
+// halves combine by a shuffle and each tile-row's runs by one fp32 atomic add
+// per row into y (zeroed first on the same stream).
+namespace tcq {
+
+template <int L, int LAYOUT>
+__global__ void __launch_bounds__(256) decode_gemv_kernel(const uint32_t *__restrict__ bits,
+                                                          int n_tr, int n_tc, int runs, int wps,
+                                                          const float *__restrict__ x,
+                                                          float *__restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int r = lane >> 1, h = lane & 1;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int per_run = (n_tc + runs - 1) / runs;
+  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wid < (int64_t)n_tr * runs; wid += warps) {
+    const int tr = (int)(wid / runs), run = (int)(wid - (int64_t)tr * runs);
+    const int c0 = run * per_run, c1 = min(n_tc, c0 + per_run);
+    float acc = 0.0f;
+    // four tiles per round: all their loads are issued before any decode, so
+    // the stream's HBM latency overlaps across tiles
+    constexpr int U = 4;
+    for (int tb = c0; tb < c1; tb += U) {
+      uint32_t w0[U], w1[U];
+      float4 xa[U], xb[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int tc = min(tb + u, c1 - 1);
+        const uint32_t *src = bits + ((int64_t)tr * n_tc + tc) * wps;
+        w0[u] = __ldg(src + r);
+        w1[u] = LAYOUT == TCQ_TAILBITING ? __ldg(src + ((r + 1) & 15)) : __ldg(src + r + 1);
+        xa[u] = __ldg(reinterpret_cast<const float4 *>(x + tc * 16 + h * 8));
+        xb[u] = __ldg(reinterpret_cast<const float4 *>(x + tc * 16 + h * 8 + 4));
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (tb + u >= c1) break;
+        const float xv[8] = {xa[u].x, xa[u].y, xa[u].z, xa[u].w, xb[u].x, xb[u].y, xb[u].z, xb[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const unsigned long long c2 =
+              one_mad_decode_f32x2(window_at<L>(w0[u], w1[u], 16 * h + 4 * j),
+                                   window_at<L>(w0[u], w1[u], 16 * h + 4 * j + 2));
+          const __half2 hw = __floats2half2_rn(__uint_as_float((uint32_t)c2),
+                                               __uint_as_float((uint32_t)(c2 >> 32)));
+          const float2 wf = __half22float2(hw);
+          acc = fmaf(wf.x, xv[2 * j], acc);
+          acc = fmaf(wf.y, xv[2 * j + 1], acc);
+        }
+      }
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    if (h == 0 && c0 < c1) atomicAdd(y + (int64_t)tr * 16 + r, acc);
+  }
+}
+
+}  // namespace tcq
+
+extern "C" tcq_status_t tcq_decode_gemv(const tcq_trellis_t *tr, const uint32_t *bits, int layout,
+                                        int64_t rows, int64_t cols, const float *x, float *y,
+                                        void *stream) {
+  tcq_status_t st = check_trellis(tr);
+  if (st != TCQ_OK) return st;
+  if (layout != TCQ_TAILBITING && layout != TCQ_FREE_START) return TCQ_ERR_INVALID_ARG;
+  if (tr->seq_len != 256) return TCQ_ERR_UNSUPPORTED;
+  if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return TCQ_ERR_INVALID_ARG;
+  if (rows / 16 > INT32_MAX || cols / 16 > INT32_MAX) return TCQ_ERR_UNSUPPORTED;
+  const size_t wps = tcq_stream_words(tr, layout);
+  if (wps == 0 || wps > 17) return TCQ_ERR_UNSUPPORTED;
+  if (!bits || !x || !y || !aligned16(bits) || !aligned16(x) || !aligned16(y))
+    return TCQ_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(y, 0, sizeof(float) * (size_t)rows, s) != cudaSuccess) return TCQ_ERR_CUDA;
+  const int n_tr = (int)(rows / 16), n_tc = (int)(cols / 16);
+  // One wave: as many warps as can be resident, each a run of tiles along a
+  // tile-row (runs per tile-row chosen so that all runs fit at once).
+  int per_sm = 0;
+  {
+    const void *fn = nullptr;
+    switch (tr->L) {
+      case 8: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_kernel<8, TCQ_TAILBITING>
+                                            : (const void *)decode_gemv_kernel<8, TCQ_FREE_START>; break;
+      case 12: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_kernel<12, TCQ_TAILBITING>
+                                             : (const void *)decode_gemv_kernel<12, TCQ_FREE_START>; break;
+      default: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_kernel<16, TCQ_TAILBITING>
+                                             : (const void *)decode_gemv_kernel<16, TCQ_FREE_START>; break;
+    }
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 256, 0) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+  }
+  const int64_t resident_warps = (int64_t)sm_count() * per_sm * 8;
+  const int runs = (int)std::max<int64_t>(1, std::min<int64_t>(n_tc, resident_warps / n_tr));
+  const int64_t warps = (int64_t)n_tr * runs;
+  const unsigned blocks = (unsigned)((warps + 7) / 8);
+#define TCQ_GEMV(LL)                                                                          \
+  (layout == TCQ_TAILBITING                                                                   \
+       ? decode_gemv_kernel<LL, TCQ_TAILBITING><<<blocks, 256, 0, s>>>(bits, n_tr, n_tc, runs, \
+                                                                        (int)wps, x, y)        \
+       : decode_gemv_kernel<LL, TCQ_FREE_START><<<blocks, 256, 0, s>>>(bits, n_tr, n_tc, runs, \
+                                                                        (int)wps, x, y))
+  switch (tr->L) {
+    case 8: TCQ_GEMV(8); break;
+    case 12: TCQ_GEMV(12); break;
+    default: TCQ_GEMV(16); break;
+  }
+#undef TCQ_GEMV
+  return launch_status();
+}

@@ -80,6 +80,8 @@ def load_measured_peaks(root: str) -> dict:
 def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str, float, str]:
     """(bound, algorithmic work per launch, unit of work) for a benchmark kernel."""
     states = float(1 << L)
+    if kernel.startswith("decode_gemv"):    # 2-bit stream in; x and y are a rounding error
+        return "hbm", n_seq * (T * 2 / 8), "bytes"
     if kernel.startswith("decode"):
         return "hbm", n_seq * (T * 2 / 8 + T * 2), "bytes"
     if kernel.startswith("rht"):            # read W once, write the rotation once (fp32)
