@@ -225,11 +225,12 @@ extern "C" tcq_status_t tcq_decode(const tcq_trellis_t *tr, const uint32_t *bits
 // end": each 16x16 tile is one 256-weight sequence that decodes straight into
 // the matmul operand, so the weights never exist in memory at 16 bits].
 //   y[i] = sum_j W[i][j] x[j],  W = the fp16 matrix tcq_decode (TILE16) gives,
-// accumulated in fp32.  A warp takes a run of tiles along one tile-row; lane
-// (r, h) decodes the 8 weights of row r, half h of each tile, rounds them to
-// fp16 exactly as the decode does, multiplies by x and accumulates; the two
-// halves combine by a shuffle and each tile-row's runs by one fp32 atomic add
-// per row into y (zeroed first on the same stream).
+// accumulated in fp32.  A warp takes a run of tile-columns along two
+// tile-rows; each lane owns one row of one of them and decodes that row's 16
+// weights in every tile of the run, rounds them to fp16 exactly as the decode
+// does and multiplies by x; the stream words of the next tile are loaded while
+// the current one decodes.  Runs combine by one fp32 atomic add per row into y
+// (zeroed first on the same stream).
 namespace tcq {
 
 template <int L, int LAYOUT>
@@ -237,49 +238,46 @@ __global__ void __launch_bounds__(256) decode_gemv_kernel(const uint32_t *__rest
                                                           int n_tr, int n_tc, int runs, int wps,
                                                           const float *__restrict__ x,
                                                           float *__restrict__ y) {
+  // lane l: tile-row 2*pair + (l >> 4), row r = l & 15 of it; the lane decodes
+  // the 16 weights of its row in every tile of the warp's run and owns y[row]
   const int lane = threadIdx.x & 31;
-  const int r = lane >> 1, h = lane & 1;
+  const int r = lane & 15, half = lane >> 4;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int n_pairs = (n_tr + 1) >> 1;
   const int per_run = (n_tc + runs - 1) / runs;
   for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       wid < (int64_t)n_tr * runs; wid += warps) {
-    const int tr = (int)(wid / runs), run = (int)(wid - (int64_t)tr * runs);
+       wid < (int64_t)n_pairs * runs; wid += warps) {
+    const int pair = (int)(wid / runs), run = (int)(wid - (int64_t)pair * runs);
+    const int tr = min(2 * pair + half, n_tr - 1);
+    const bool owner = 2 * pair + half < n_tr;
     const int c0 = run * per_run, c1 = min(n_tc, c0 + per_run);
+    if (c0 >= c1) continue;
+    const uint32_t *row_src = bits + (int64_t)tr * n_tc * wps + r;
+    const int r1 = LAYOUT == TCQ_TAILBITING ? (((r + 1) & 15) - r) : 1;   // offset of word r+1
+    uint32_t nw0 = __ldg(row_src + (int64_t)c0 * wps), nw1 = __ldg(row_src + (int64_t)c0 * wps + r1);
     float acc = 0.0f;
-    // four tiles per round: all their loads are issued before any decode, so
-    // the stream's HBM latency overlaps across tiles
-    constexpr int U = 4;
-    for (int tb = c0; tb < c1; tb += U) {
-      uint32_t w0[U], w1[U];
-      float4 xa[U], xb[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int tc = min(tb + u, c1 - 1);
-        const uint32_t *src = bits + ((int64_t)tr * n_tc + tc) * wps;
-        w0[u] = __ldg(src + r);
-        w1[u] = LAYOUT == TCQ_TAILBITING ? __ldg(src + ((r + 1) & 15)) : __ldg(src + r + 1);
-        xa[u] = __ldg(reinterpret_cast<const float4 *>(x + tc * 16 + h * 8));
-        xb[u] = __ldg(reinterpret_cast<const float4 *>(x + tc * 16 + h * 8 + 4));
+    for (int tc = c0; tc < c1; ++tc) {
+      const uint32_t w0 = nw0, w1 = nw1;
+      if (tc + 1 < c1) {                               // next tile's words, one tile ahead
+        nw0 = __ldg(row_src + (int64_t)(tc + 1) * wps);
+        nw1 = __ldg(row_src + (int64_t)(tc + 1) * wps + r1);
       }
+      const float4 *xq = reinterpret_cast<const float4 *>(x + tc * 16);
+      const float4 x0 = __ldg(xq), x1 = __ldg(xq + 1), x2 = __ldg(xq + 2), x3 = __ldg(xq + 3);
+      const float xv[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                            x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (tb + u >= c1) break;
-        const float xv[8] = {xa[u].x, xa[u].y, xa[u].z, xa[u].w, xb[u].x, xb[u].y, xb[u].z, xb[u].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const unsigned long long c2 =
-              one_mad_decode_f32x2(window_at<L>(w0[u], w1[u], 16 * h + 4 * j),
-                                   window_at<L>(w0[u], w1[u], 16 * h + 4 * j + 2));
-          const __half2 hw = __floats2half2_rn(__uint_as_float((uint32_t)c2),
-                                               __uint_as_float((uint32_t)(c2 >> 32)));
-          const float2 wf = __half22float2(hw);
-          acc = fmaf(wf.x, xv[2 * j], acc);
-          acc = fmaf(wf.y, xv[2 * j + 1], acc);
-        }
+      for (int j = 0; j < 8; ++j) {                    // weights 2j, 2j+1 of the row
+        const unsigned long long c2 = one_mad_decode_f32x2(window_at<L>(w0, w1, 4 * j),
+                                                           window_at<L>(w0, w1, 4 * j + 2));
+        const __half2 hw = __floats2half2_rn(__uint_as_float((uint32_t)c2),
+                                             __uint_as_float((uint32_t)(c2 >> 32)));
+        const float2 wf = __half22float2(hw);
+        acc = fmaf(wf.x, xv[2 * j], acc);
+        acc = fmaf(wf.y, xv[2 * j + 1], acc);
       }
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    if (h == 0 && c0 < c1) atomicAdd(y + (int64_t)tr * 16 + r, acc);
+    if (owner) atomicAdd(y + (int64_t)tr * 16 + r, acc);
   }
 }
 
@@ -318,8 +316,9 @@ extern "C" tcq_status_t tcq_decode_gemv(const tcq_trellis_t *tr, const uint32_t 
       per_sm = 1;
   }
   const int64_t resident_warps = (int64_t)sm_count() * per_sm * 8;
-  const int runs = (int)std::max<int64_t>(1, std::min<int64_t>(n_tc, resident_warps / n_tr));
-  const int64_t warps = (int64_t)n_tr * runs;
+  const int64_t n_pairs = (n_tr + 1) / 2;
+  const int runs = (int)std::max<int64_t>(1, std::min<int64_t>(n_tc, resident_warps / n_pairs));
+  const int64_t warps = n_pairs * runs;
   const unsigned blocks = (unsigned)((warps + 7) / 8);
 #define TCQ_GEMV(LL)                                                                          \
   (layout == TCQ_TAILBITING                                                                   \
