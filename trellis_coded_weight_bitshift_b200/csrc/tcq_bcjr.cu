@@ -78,6 +78,7 @@ struct BcjrCfg {
   static constexpr int NT = TPS * SPC;
   static constexpr int GQ = G / 4;
   static constexpr int ASM = 4 - AREG;
+  static constexpr int HREG = AREG / 2, HS = 2 - HREG;          // digit pairs: registers | smem
   static constexpr int NPART = TPS >= 32 ? TPS / 32 : 1;       // partial records per sequence
   static constexpr int PREC = 8;                                 // floats per partial record
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
@@ -93,24 +94,30 @@ struct BcjrCfg {
   static constexpr size_t smem_bytes() { return smem_floats() * sizeof(float); }
   __host__ __device__ static constexpr size_t ws_floats_per_slot(int T) { return (size_t)T * NV * NG; }
   static_assert(NG % G == 0 && G % 4 == 0, "bad split");
+  static_assert(AREG % 2 == 0, "code values are held in digit pairs");
   static_assert(SPILL % 4 == 0, "spill in float4 chunks");
 };
 
+// Code values are held as vertical pairs over the predecessor digit:
+// cv[h][i] = (code of state 2h NG + G w + i, code of state (2h+1) NG + G w + i),
+// digit pairs h < HREG in registers, the others in shared memory as float2
+// [HS][G][TPS] (consecutive lanes read consecutive pairs).
 template <class C>
-__device__ __forceinline__ float code_at(const float (&creg)[C::AREG > 0 ? C::AREG : 1][C::G],
-                                         const float *Csm, int a, int i, int w) {
-  if (a < C::AREG) return creg[a < C::AREG ? a : 0][i];
-  return Csm[((a - C::AREG) * C::GQ + (i >> 2)) * C::TPS * 4 + w * 4 + (i & 3)];
+using CodeRegs = f2_t[C::HREG > 0 ? C::HREG : 1][C::G];
+
+template <class C>
+__device__ __forceinline__ f2_t code_vpair(const CodeRegs<C> &cv, const float2 *Csm, int h, int i,
+                                          int w) {
+  if (h < C::HREG) return cv[h < C::HREG ? h : 0][i];
+  const float2 v = Csm[((h - C::HREG) * C::G + i) * C::TPS + w];
+  return f2(v.x, v.y);
 }
 
-// Code values of predecessor states (a, i) and (a, i+1) as a packed pair (i even).
 template <class C>
-__device__ __forceinline__ f2_t code_pair(const float (&creg)[C::AREG > 0 ? C::AREG : 1][C::G],
-                                         const float *Csm, int a, int i, int w) {
-  if (a < C::AREG) return f2(creg[a < C::AREG ? a : 0][i], creg[a < C::AREG ? a : 0][i + 1]);
-  const float2 v = *reinterpret_cast<const float2 *>(
-      &Csm[((a - C::AREG) * C::GQ + (i >> 2)) * C::TPS * 4 + w * 4 + (i & 3)]);
-  return f2(v.x, v.y);
+__device__ __forceinline__ float code_at(const CodeRegs<C> &cv, const float2 *Csm, int a, int i,
+                                         int w) {
+  const f2_t v = code_vpair<C>(cv, Csm, a >> 1, i, w);
+  return (a & 1) ? f2hi(v) : f2lo(v);
 }
 
 // Reduce within the TPS lanes of a sequence (TPS < 32) or the whole warp.
@@ -123,6 +130,46 @@ __device__ __forceinline__ float lane_reduce(float v, Op op) {
 }
 
 struct MaxOp { __device__ float operator()(float a, float b) const { return fmaxf(a, b); } };
+
+// Maximum over the TPS lanes of a sequence: one warp-wide redux when the
+// sequence spans whole warps, else a shuffle tree.
+template <int TPS>
+__device__ __forceinline__ float seq_max(float v) {
+  if constexpr (TPS >= 32) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+  } else {
+    return lane_reduce<TPS>(v, MaxOp());
+  }
+}
+
+// Sums of NQ (2 or 4) values over the WL = min(TPS, 32) lanes of a sequence
+// in one shuffle tree: the first levels exchange different quantities, so the
+// lane at offset o (within the WL lanes) ends with the full sum of quantity
+// o / (WL / NQ).
+template <int TPS, int NQ>
+__device__ __forceinline__ float seq_sums(const float (&v)[NQ], int lane) {
+  constexpr int WL = TPS < 32 ? TPS : 32;
+  static_assert(NQ == 2 || NQ == 4, "two or four quantities");
+  float y;
+  if constexpr (NQ == 4) {
+    const bool h1 = lane & (WL / 2);
+    float k0 = h1 ? v[2] : v[0], k1 = h1 ? v[3] : v[1];
+    k0 += __shfl_xor_sync(0xffffffffu, h1 ? v[0] : v[2], WL / 2);
+    k1 += __shfl_xor_sync(0xffffffffu, h1 ? v[1] : v[3], WL / 2);
+    const bool h2 = lane & (WL / 4);
+    y = (h2 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, h2 ? k0 : k1, WL / 4);
+#pragma unroll
+    for (int off = WL / 8; off > 0; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+  } else {
+    const bool h1 = lane & (WL / 2);
+    y = (h1 ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, h1 ? v[0] : v[1], WL / 2);
+#pragma unroll
+    for (int off = WL / 4; off > 0; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+  }
+  return y;
+}
 struct SumOp { __device__ float operator()(float a, float b) const { return a + b; } };
 
 // GQ contiguous state-vector values of run `base` (swizzled shared memory).
@@ -158,6 +205,18 @@ __device__ __forceinline__ void write_run(float *vec, int base, const float *src
   }
 }
 
+// N (1, 2 or 4) contiguous state-vector values at base (N | base).
+template <class C, int N>
+__device__ __forceinline__ void write_sub(float *vec, int base, const float *src) {
+  if constexpr (N == 1) {
+    vec[swz<C::SWZ>(base)] = src[0];
+  } else if constexpr (N == 2) {
+    *reinterpret_cast<float2 *>(vec + swz<C::SWZ>(base)) = make_float2(src[0], src[1]);
+  } else {
+    *reinterpret_cast<float4 *>(vec + swz<C::SWZ>(base)) = make_float4(src[0], src[1], src[2], src[3]);
+  }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::NT, C::MINB)
 bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n_seq, int T,
@@ -170,8 +229,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   constexpr bool GRAD = C::GRAD;
   extern __shared__ __align__(16) float smem[];
   float *Vall = smem;                                      // [SPC][NB][NV][NG]
-  float *Csm = Vall + SPC * NB * NV * NG;                  // [ASM][GQ][TPS][4]
-  float *ssm = Csm + C::ASM * G * TPS;                     // [SPC][256]
+  float2 *Csm = reinterpret_cast<float2 *>(Vall + SPC * NB * NV * NG);  // [HS][G][TPS]
+  float *ssm = reinterpret_cast<float *>(Csm + C::HS * G * TPS);        // [SPC][256]
   float *ksm = ssm + SPC * 256;                            // [SPC][256] kappa * D_t
   float *vsm = ksm + SPC * 256;                            // GRAD: v, soft rows
   float *fsm = vsm + (GRAD ? SPC * 256 : 0);
@@ -184,16 +243,19 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   const int pidx = TPS >= 32 ? (w >> 5) : 0;
   const bool plead = TPS >= 32 ? (lane == 0) : (w == 0);
 
-  float creg[C::AREG > 0 ? C::AREG : 1][G];
+  CodeRegs<C> cv;
 #pragma unroll
-  for (int a = 0; a < C::AREG; ++a)
+  for (int h = 0; h < C::HREG; ++h)
 #pragma unroll
-    for (int i = 0; i < G; ++i) creg[a][i] = one_mad_f32((uint32_t)(a * NG + G * w + i));
+    for (int i = 0; i < G; ++i)
+      cv[h][i] = f2(one_mad_f32((uint32_t)(2 * h * NG + G * w + i)),
+                    one_mad_f32((uint32_t)((2 * h + 1) * NG + G * w + i)));
   if (ls == 0) {
-    for (int a = 0; a < C::ASM; ++a)
+    for (int h = C::HREG; h < 2; ++h)
       for (int i = 0; i < G; ++i)
-        Csm[(a * GQ + (i >> 2)) * TPS * 4 + w * 4 + (i & 3)] =
-            one_mad_f32((uint32_t)((a + C::AREG) * NG + G * w + i));
+        Csm[((h - C::HREG) * G + i) * TPS + w] =
+            make_float2(one_mad_f32((uint32_t)(2 * h * NG + G * w + i)),
+                        one_mad_f32((uint32_t)((2 * h + 1) * NG + G * w + i)));
   }
 
   // thread-private spill: [T][NCH][TPS] float4; step t holds A_t (and Phi_t)
@@ -265,67 +327,56 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       const float vv = GRAD ? vsm[ls * 256 + t - 1] : 0.0f;
       const float fv = GRAD ? fsm[ls * 256 + t - 1] : 0.0f;
       float tmax = -INFINITY;
+      const f2_t sv2 = f2(sv, sv), cm2 = f2(cmax, cmax);
+      const f2_t nk2 = f2(-ksm[ls * 256 + t - 1], -ksm[ls * 256 + t - 1]);
       if constexpr (!GRAD) {
-        const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + t - 1], -ksm[ls * 256 + t - 1]);
 #pragma unroll
         for (int q = 0; q < GQ; ++q) {
-          // x[a][r]: input of group 4q + r from predecessor digit a
-          float x[4][4];
-#pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            const float am = ain[a][q] - cmax;
-            const f2_t am2 = f2(am, am);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const f2_t d = f2sub(code_pair<C>(creg, Csm, a, 4 * q + 2 * h, w), sv2);
-              const f2_t xv = f2fma(f2mul(d, nk2), d, am2);
-              x[a][2 * h] = f2lo(xv);
-              x[a][2 * h + 1] = f2hi(xv);
-            }
-          }
+          // inputs of group 4q + r from predecessor digits (0, 1) and (2, 3)
+          const f2_t am0 = f2sub(f2(ain[0][q], ain[1][q]), cm2);
+          const f2_t am1 = f2sub(f2(ain[2][q], ain[3][q]), cm2);
           float outA[4];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            outA[r] = lse4_base2(x[0][r], x[1][r], x[2][r], x[3][r]);
+            const f2_t d0 = f2sub(code_vpair<C>(cv, Csm, 0, 4 * q + r, w), sv2);
+            const f2_t d1 = f2sub(code_vpair<C>(cv, Csm, 1, 4 * q + r, w), sv2);
+            const f2_t x0 = f2fma(f2mul(d0, nk2), d0, am0);
+            const f2_t x1 = f2fma(f2mul(d1, nk2), d1, am1);
+            outA[r] = lse4_base2(f2lo(x0), f2hi(x0), f2lo(x1), f2hi(x1));
             tmax = fmaxf(tmax, outA[r]);
           }
           *reinterpret_cast<float4 *>(Ao + swz<C::SWZ>(G * w + 4 * q)) =
               make_float4(outA[0], outA[1], outA[2], outA[3]);
         }
       } else {
-        const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + t - 1], -ksm[ls * 256 + t - 1]), vv2 = f2(vv, vv);
+        const f2_t vv2 = f2(vv, vv), vf2 = f2(vv * fv, vv * fv);
 #pragma unroll
         for (int q = 0; q < GQ; ++q) {
-          float x[4][4], z[4][4];
-#pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            const float am = ain[a][q] - cmax;
-            const float ph = fin[a < (GRAD ? 4 : 1) ? a : 0][q] - vv * fv;
-            const f2_t am2 = f2(am, am), ph2 = f2(ph, ph);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const f2_t cp = code_pair<C>(creg, Csm, a, 4 * q + 2 * h, w);
-              const f2_t d = f2sub(cp, sv2);
-              const f2_t xv = f2fma(f2mul(d, nk2), d, am2);
-              const f2_t zv = f2fma(vv2, cp, ph2);        // phi_{t-1}(p) = Phi + v (c - soft)
-              x[a][2 * h] = f2lo(xv); x[a][2 * h + 1] = f2hi(xv);
-              z[a][2 * h] = f2lo(zv); z[a][2 * h + 1] = f2hi(zv);
-            }
-          }
+          const f2_t am0 = f2sub(f2(ain[0][q], ain[1][q]), cm2);
+          const f2_t am1 = f2sub(f2(ain[2][q], ain[3][q]), cm2);
+          const f2_t ph0 = f2sub(f2(fin[0][q], fin[1][q]), vf2);
+          const f2_t ph1 = f2sub(f2(fin[2][q], fin[3][q]), vf2);
           float outA[4], outF[4];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const float mx = fmaxf(fmaxf(x[0][r], x[1][r]), fmaxf(x[2][r], x[3][r]));
-            const f2_t e01 = f2sub(f2(x[0][r], x[1][r]), f2(mx, mx));
-            const f2_t e23 = f2sub(f2(x[2][r], x[3][r]), f2(mx, mx));
-            const f2_t u01 = f2(ex2(f2lo(e01)), ex2(f2hi(e01)));
-            const f2_t u23 = f2(ex2(f2lo(e23)), ex2(f2hi(e23)));
-            const f2_t su = f2add(u01, u23);
-            const f2_t sz = f2fma(u23, f2(z[2][r], z[3][r]), f2mul(u01, f2(z[0][r], z[1][r])));
+            const f2_t c0 = code_vpair<C>(cv, Csm, 0, 4 * q + r, w);
+            const f2_t c1 = code_vpair<C>(cv, Csm, 1, 4 * q + r, w);
+            const f2_t d0 = f2sub(c0, sv2), d1 = f2sub(c1, sv2);
+            const f2_t x0 = f2fma(f2mul(d0, nk2), d0, am0);
+            const f2_t x1 = f2fma(f2mul(d1, nk2), d1, am1);
+            const f2_t z0 = f2fma(vv2, c0, ph0);            // phi_{t-1}(p) = Phi + v (c - soft)
+            const f2_t z1 = f2fma(vv2, c1, ph1);
+            const float mx = fmaxf(fmaxf(f2lo(x0), f2hi(x0)), fmaxf(f2lo(x1), f2hi(x1)));
+            const f2_t mx2 = f2(mx, mx);
+            const f2_t e0 = f2sub(x0, mx2), e1 = f2sub(x1, mx2);
+            const f2_t u0 = f2(ex2(f2lo(e0)), ex2(f2hi(e0)));
+            const f2_t u1 = f2(ex2(f2lo(e1)), ex2(f2hi(e1)));
+            const f2_t su = f2add(u0, u1);
+            const f2_t sz = f2fma(u1, z1, f2mul(u0, z0));
             const float S = f2lo(su) + f2hi(su);
             outA[r] = mx + lg2(S);
             tmax = fmaxf(tmax, outA[r]);
-            outF[r] = (f2lo(sz) + f2hi(sz)) * __frcp_rn(S);
+            outF[r] = (f2lo(sz) + f2hi(sz)) * rcp(S);
           }
           *reinterpret_cast<float4 *>(Ao + swz<C::SWZ>(G * w + 4 * q)) =
               make_float4(outA[0], outA[1], outA[2], outA[3]);
@@ -333,7 +384,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
               make_float4(outF[0], outF[1], outF[2], outF[3]);
         }
       }
-      tmax = lane_reduce<TPS>(tmax, MaxOp());
+      tmax = seq_max<TPS>(tmax);
       if (plead) prec(t & 1)[pidx * PREC] = tmax;
       __syncthreads();
     }
@@ -360,7 +411,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           float y[4];
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
-            const float d = code_at<C>(creg, Csm, a, 4 * k + b, w) - sT;
+            const float d = code_at<C>(cv, Csm, a, 4 * k + b, w) - sT;
             y[b] = -ksm[ls * 256 + T - 1] * d * d;
           }
           const float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
@@ -457,125 +508,116 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       const float fv = GRAD ? fsm[ls * 256 + tc] : 0.0f;
       float *Bo = Bv + ((t + NB) % NB) * NV * NG;
       float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f, tmax = -INFINITY;
-      if constexpr (!GRAD) {
-        const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + tc], -ksm[ls * 256 + tc]);
+      const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + tc], -ksm[ls * 256 + tc]);
+      const f2_t K2 = f2(K, K), dp2 = f2(dprev, dprev), vv2 = f2(vv, vv);
+      f2_t num2 = f2(0.0f, 0.0f), den2 = num2, n12 = num2, n22 = num2;
+      // KB values of this thread's spilled vector at flat index f (KB | f)
+      constexpr int KB = GQ < 2 ? GQ : 2;
+      auto spilled_run = [&](int f, float *dst) {
+        float4 v;
+        if constexpr (PREFETCH) v = avq[PREFETCH ? (f >> 2) : 0];
+        else v = spill[((size_t)tc * NCH + (f >> 2)) * TPS + w];
+        const float e4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          float av[GQ];
+        for (int j = 0; j < KB; ++j) dst[j] = e4[(f & 3) + j];
+      };
+      const float nvf = -vv * fv;
+      // digit pair h: groups r = a NG/4 + GQ w + k of digits a = 2h, 2h+1 side by
+      // side; their successors 4r + b share the B_{tc+1} value bin[4k + b]
 #pragma unroll
-          for (int q = 0; q < (GQ + 3) / 4; ++q) {
-            const int f = a * GQ + 4 * q;
-            float4 v;
-            if constexpr (PREFETCH) v = avq[PREFETCH ? (f >> 2) : 0];
-            else v = spill[((size_t)tc * NCH + (f >> 2)) * TPS + w];
-            const float e4[4] = {v.x, v.y, v.z, v.w};
+      for (int h = 0; h < 2; ++h) {
 #pragma unroll
-            for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) av[4 * q + k] = e4[(f & 3) + k];
+        for (int kb = 0; kb < GQ / KB; ++kb) {
+          float avl[KB], avh[KB], fal[GRAD ? KB : 1], fah[GRAD ? KB : 1];
+          spilled_run(2 * h * GQ + KB * kb, avl);
+          spilled_run((2 * h + 1) * GQ + KB * kb, avh);
+          if constexpr (GRAD) {
+            spilled_run(G + 2 * h * GQ + KB * kb, fal);
+            spilled_run(G + (2 * h + 1) * GQ + KB * kb, fah);
           }
-          float outB[GQ];
+          float outL[KB], outH[KB], outPL[GRAD ? KB : 1], outPH[GRAD ? KB : 1];
 #pragma unroll
-          for (int k = 0; k < GQ; ++k) {
-            const f2_t c01 = code_pair<C>(creg, Csm, a, 4 * k, w);
-            const f2_t c23 = code_pair<C>(creg, Csm, a, 4 * k + 2, w);
-            const f2_t d01 = f2sub(c01, sv2), d23 = f2sub(c23, sv2);
-            const f2_t y01 = f2fma(f2mul(d01, nk2), d01, f2(bin[4 * k], bin[4 * k + 1]));
-            const f2_t y23 = f2fma(f2mul(d23, nk2), d23, f2(bin[4 * k + 2], bin[4 * k + 3]));
-            const float mx = fmaxf(fmaxf(f2lo(y01), f2hi(y01)), fmaxf(f2lo(y23), f2hi(y23)));
-            const f2_t mx2 = f2(mx, mx);
-            const f2_t e01 = f2sub(y01, mx2), e23 = f2sub(y23, mx2);
-            const f2_t u01 = f2(ex2(f2lo(e01)), ex2(f2hi(e01)));
-            const f2_t u23 = f2(ex2(f2lo(e23)), ex2(f2hi(e23)));
-            const f2_t su = f2add(u01, u23);
-            const f2_t sc = f2fma(u23, c23, f2mul(u01, c01));
-            const float S = f2lo(su) + f2hi(su), Sc = f2lo(sc) + f2hi(sc);
-            outB[k] = (mx - dprev) + lg2(S);
-            tmax = fmaxf(tmax, outB[k]);
-            const float wgt = ex2((av[k] - K) + mx);
-            den = fmaf(wgt, S, den);
-            num = fmaf(wgt, Sc, num);
-          }
-          if (t >= 0) write_run<C>(Bo, a * (NG / 4) + GQ * w, outB);
-        }
-      } else {
-        const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + tc], -ksm[ls * 256 + tc]), vv2 = f2(vv, vv);
-        const float nvf = -vv * fv;
-        // spilled (A, Phi) values of digit a, loaded one digit ahead
-        constexpr int QN = (GQ + 3) / 4;
-        float4 nv[QN], nu[QN];
+          for (int j = 0; j < KB; ++j) {
+            const int k = KB * kb + j;
+            f2_t cc[4], y[4];
 #pragma unroll
-        for (int q = 0; q < QN; ++q) {
-          nv[q] = spill[((size_t)tc * NCH + ((0 * GQ + 4 * q) >> 2)) * TPS + w];
-          nu[q] = spill[((size_t)tc * NCH + ((G + 0 * GQ + 4 * q) >> 2)) * TPS + w];
-        }
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          float av[GQ], fa[GQ];
-#pragma unroll
-          for (int q = 0; q < QN; ++q) {
-            const int f = a * GQ + 4 * q, g = G + a * GQ + 4 * q;
-            const float e4[4] = {nv[q].x, nv[q].y, nv[q].z, nv[q].w};
-            const float g4[4] = {nu[q].x, nu[q].y, nu[q].z, nu[q].w};
-#pragma unroll
-            for (int k = 0; k < 4 && 4 * q + k < GQ; ++k) {
-              av[4 * q + k] = e4[(f & 3) + k];
-              fa[4 * q + k] = g4[(g & 3) + k];
+            for (int b = 0; b < 4; ++b) {
+              cc[b] = code_vpair<C>(cv, Csm, h, 4 * k + b, w);
+              const f2_t d = f2sub(cc[b], sv2);
+              y[b] = f2fma(f2mul(d, nk2), d, f2(bin[4 * k + b], bin[4 * k + b]));
             }
-          }
-          if (a < 3) {
+            const float mxl = fmaxf(fmaxf(f2lo(y[0]), f2lo(y[1])), fmaxf(f2lo(y[2]), f2lo(y[3])));
+            const float mxh = fmaxf(fmaxf(f2hi(y[0]), f2hi(y[1])), fmaxf(f2hi(y[2]), f2hi(y[3])));
+            const f2_t mx2 = f2(mxl, mxh);
+            f2_t u[4];
 #pragma unroll
-            for (int q = 0; q < QN; ++q) {
-              nv[q] = spill[((size_t)tc * NCH + (((a + 1) * GQ + 4 * q) >> 2)) * TPS + w];
-              nu[q] = spill[((size_t)tc * NCH + ((G + (a + 1) * GQ + 4 * q) >> 2)) * TPS + w];
+            for (int b = 0; b < 4; ++b) {
+              const f2_t e = f2sub(y[b], mx2);
+              u[b] = f2(ex2(f2lo(e)), ex2(f2hi(e)));
             }
-          }
-          float outB[GQ], outP[GQ];
+            const f2_t su = f2add(f2add(u[0], u[2]), f2add(u[1], u[3]));
+            const f2_t ob = f2add(f2sub(mx2, dp2), f2(lg2(f2lo(su)), lg2(f2hi(su))));
+            outL[j] = f2lo(ob);
+            outH[j] = f2hi(ob);
+            tmax = fmaxf(tmax, fmaxf(outL[j], outH[j]));
+            const f2_t wv = f2add(f2sub(f2(avl[j], avh[j]), K2), mx2);
+            const f2_t wgt = f2(ex2(f2lo(wv)), ex2(f2hi(wv)));
+            den2 = f2fma(wgt, su, den2);
+            if constexpr (!GRAD) {
+              const f2_t sc = f2add(f2fma(u[2], cc[2], f2mul(u[0], cc[0])),
+                                    f2fma(u[3], cc[3], f2mul(u[1], cc[1])));
+              num2 = f2fma(wgt, sc, num2);
+            } else {
+              // z_b = psi_{tc}(succ) + v_tc (c_b - soft_tc)
+              f2_t z[4], uc[4];
 #pragma unroll
-          for (int k = 0; k < GQ; ++k) {
-            const f2_t c01 = code_pair<C>(creg, Csm, a, 4 * k, w);
-            const f2_t c23 = code_pair<C>(creg, Csm, a, 4 * k + 2, w);
-            const f2_t d01 = f2sub(c01, sv2), d23 = f2sub(c23, sv2);
-            const f2_t y01 = f2fma(f2mul(d01, nk2), d01, f2(bin[4 * k], bin[4 * k + 1]));
-            const f2_t y23 = f2fma(f2mul(d23, nk2), d23, f2(bin[4 * k + 2], bin[4 * k + 3]));
-            // z_b = psi_{tc}(succ) + v_tc (c_b - soft_tc)
-            const f2_t z01 = f2fma(vv2, c01, f2add(f2(pin[4 * k], pin[4 * k + 1]), f2(nvf, nvf)));
-            const f2_t z23 = f2fma(vv2, c23, f2add(f2(pin[4 * k + 2], pin[4 * k + 3]), f2(nvf, nvf)));
-            const float mx = fmaxf(fmaxf(f2lo(y01), f2hi(y01)), fmaxf(f2lo(y23), f2hi(y23)));
-            const f2_t mx2 = f2(mx, mx);
-            const f2_t e01 = f2sub(y01, mx2), e23 = f2sub(y23, mx2);
-            const f2_t u01 = f2(ex2(f2lo(e01)), ex2(f2hi(e01)));
-            const f2_t u23 = f2(ex2(f2lo(e23)), ex2(f2hi(e23)));
-            const f2_t uc01 = f2mul(u01, c01), uc23 = f2mul(u23, c23);
-            const f2_t su = f2add(u01, u23);
-            const f2_t sc = f2add(uc01, uc23);
-            const f2_t sz = f2fma(u23, z23, f2mul(u01, z01));
-            const f2_t scz = f2fma(uc23, z23, f2mul(uc01, z01));
-            const float S = f2lo(su) + f2hi(su), Sc = f2lo(sc) + f2hi(sc);
-            const float Sz = f2lo(sz) + f2hi(sz), Scz = f2lo(scz) + f2hi(scz);
-            outB[k] = (mx - dprev) + lg2(S);
-            tmax = fmaxf(tmax, outB[k]);
-            outP[k] = Sz * __frcp_rn(S);
-            const float wgt = ex2((av[k] - K) + mx);
-            den = fmaf(wgt, S, den);
-            num = fmaf(wgt, Sc, num);
-            n1 = fmaf(wgt, fmaf(fa[k], S, Sz), n1);
-            n2 = fmaf(wgt, fmaf(fa[k], Sc, Scz), n2);
+              for (int b = 0; b < 4; ++b) {
+                const float pz = pin[4 * k + b] + nvf;
+                z[b] = f2fma(vv2, cc[b], f2(pz, pz));
+                uc[b] = f2mul(u[b], cc[b]);
+              }
+              const f2_t sc = f2add(f2add(uc[0], uc[2]), f2add(uc[1], uc[3]));
+              const f2_t sz = f2add(f2fma(u[2], z[2], f2mul(u[0], z[0])),
+                                    f2fma(u[3], z[3], f2mul(u[1], z[1])));
+              const f2_t scz = f2add(f2fma(uc[2], z[2], f2mul(uc[0], z[0])),
+                                     f2fma(uc[3], z[3], f2mul(uc[1], z[1])));
+              const f2_t op = f2mul(sz, f2(rcp(f2lo(su)), rcp(f2hi(su))));
+              outPL[j] = f2lo(op);
+              outPH[j] = f2hi(op);
+              const f2_t fa2 = f2(fal[j], fah[j]);
+              num2 = f2fma(wgt, sc, num2);
+              n12 = f2fma(wgt, f2fma(fa2, su, sz), n12);
+              n22 = f2fma(wgt, f2fma(fa2, sc, scz), n22);
+            }
           }
           if (t >= 0) {
-            write_run<C>(Bo, a * (NG / 4) + GQ * w, outB);
-            write_run<C>(Bo + NG, a * (NG / 4) + GQ * w, outP);
+            const int bl = 2 * h * (NG / 4) + GQ * w + KB * kb, bh = bl + NG / 4;
+            write_sub<C, KB>(Bo, bl, outL);
+            write_sub<C, KB>(Bo, bh, outH);
+            if constexpr (GRAD) {
+              write_sub<C, KB>(Bo + NG, bl, outPL);
+              write_sub<C, KB>(Bo + NG, bh, outPH);
+            }
           }
         }
       }
-      tmax = lane_reduce<TPS>(tmax, MaxOp());
-      num = lane_reduce<TPS>(num, SumOp());
-      den = lane_reduce<TPS>(den, SumOp());
-      if (GRAD) {
-        n1 = lane_reduce<TPS>(n1, SumOp());
-        n2 = lane_reduce<TPS>(n2, SumOp());
+      num = f2lo(num2) + f2hi(num2);
+      den = f2lo(den2) + f2hi(den2);
+      if constexpr (GRAD) {
+        n1 = f2lo(n12) + f2hi(n12);
+        n2 = f2lo(n22) + f2hi(n22);
       }
-      if (plead) {
+      tmax = seq_max<TPS>(tmax);
+      {
+        constexpr int NQ = GRAD ? 4 : 2, WL = TPS < 32 ? TPS : 32;
+        float q4[NQ];
+        q4[0] = num; q4[1] = den;
+        if constexpr (GRAD) { q4[NQ > 2 ? 2 : 0] = n1; q4[NQ > 3 ? 3 : 0] = n2; }
+        const float mine = seq_sums<TPS, NQ>(q4, lane);
+        const int o = lane & (WL - 1);
         float *pp = prec(tc & 1) + pidx * PREC;
-        pp[0] = tmax; pp[1] = num; pp[2] = den; pp[3] = n1; pp[4] = n2;
+        if ((o & (WL / NQ - 1)) == 0) pp[1 + o / (WL / NQ)] = mine;   // num, den, n1, n2
+        if (plead) pp[0] = tmax;
       }
       __syncthreads();
     }
@@ -603,10 +645,13 @@ using namespace tcq_host;
 namespace {
 
 using Soft8 = BcjrCfg<8, 4, 8, 4, 2, false>;
-using Soft12 = BcjrCfg<12, 8, 1, 4, 2, false, 7>;    // 128 threads / sequence, 7 per SM: one wave of 1,036
+// L = 12: 128 threads / sequence, 7 per SM (one wave of 1,036); the soft pass
+// reads every code value from shared memory, the gradient pass keeps digits
+// 0 and 1 in registers (the register file allows 72 per thread)
+using Soft12 = BcjrCfg<12, 8, 1, 0, 2, false, 7>;
 using Soft16 = BcjrCfg<16, 32, 1, 2, 1, false>;
 using Grad8 = BcjrCfg<8, 4, 8, 4, 2, true>;
-using Grad12 = BcjrCfg<12, 8, 1, 4, 2, true, 7>;     // 128 threads / sequence, 7 per SM
+using Grad12 = BcjrCfg<12, 8, 1, 2, 2, true, 7>;
 
 template <class C>
 int grid_for(int64_t n_seq) {

@@ -3,7 +3,8 @@
 //   * the 1MAD computed code [QTIP blog, "The codebook is computed"]: a 32-bit
 //     LCG step, the byte sum of its output (one VABSDIFF4 against zero), the
 //     centring by 510 and the scale 1/147.8;
-//   * base-2 exponent/logarithm on the MUFU unit (PTX ex2/lg2.approx);
+//   * base-2 exponent/logarithm and reciprocal on the MUFU unit (PTX
+//     ex2/lg2/rcp.approx);
 //   * the shared-memory swizzle used by every state-vector exchange;
 //   * small launch/validation helpers for the C ABI.
 #pragma once
@@ -110,6 +111,13 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ float lg2(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Reciprocal on the MUFU unit (PTX rcp.approx, a single special-function op).
+__device__ __forceinline__ float rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
