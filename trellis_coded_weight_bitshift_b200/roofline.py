@@ -38,14 +38,15 @@ MUFU_PER_SM = 16               # special-function results per clock per SM
 # null.  (kernel prefix, workload): (bytes, sequences in the capture, sources)
 _CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 MEASURED_TRAFFIC = {
-    ("bcjr_soft_vjp", "l12_gauss1024"): (2.139645e9 + 2.179336e9, 1024, {
-        "tcq_bcjr.cu": "96df19e5969718a26fb330fe71505390f1840110",
-        "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
+    ("bcjr_soft_vjp", "l12_gauss1024"): (2.106506e9 + 2.182354e9, 1024, {
+        "tcq_bcjr.cu": "74c770c6300308e4af2802c9ca117ef3f97ebf3d",
+        "tcq_device.cuh": "804f75be759c65adfd0397217b44b3edffd5549a"}),
     # three launches (row pass, two column passes) of one 8192 x 8192 rotation
     ("rht", "rht_t5_8192sq"): (268.563712e6 + 223.412224e6 + 268.515328e6 + 209.742592e6
                                + 268.464896e6 + 209.4656e6, 262144, {
         "tcq_rht.cu": "ccfacb475702414c5cd2f49317f76388abbd2f52",
-        "tcq_device.cuh": "467d6627e2313e263e66c0a462e11bdfa05261d7"}),
+        # the header has since gained only a reciprocal helper the rotation does not use
+        "tcq_device.cuh": "804f75be759c65adfd0397217b44b3edffd5549a"}),
 }
 
 
