@@ -482,6 +482,8 @@ def run_ours(a) -> None:
                    "l2": "flushed (256 MiB write) before every timed step, outside its events",
                    "parallelism": f"dp{world} (independent batches, no data-path collective)"},
         "kernels_ms": {k: round(v, 4) for k, v in kern_mean.items()},
+        "edges_per_s": {k: RL.trellis_edges(k, w) * world / (v * 1e-3) for k, v in kern_mean.items()
+                        if RL.trellis_edges(k, w) > 0},
         "roofline": roof,
         "e2e": {"value": units / (e2e_mean * 1e-3), "unit": "weights/s",
                 "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes)},

@@ -263,6 +263,27 @@ def test_vjp_matches_oracle(tcq, name, temp, nsample):
         assert np.abs(g[j] - rg[i]).max() <= tol, (j, np.abs(g[j] - rg[i]).max(), tol)
 
 
+@pytest.mark.parametrize("L", [8, 12])
+@pytest.mark.parametrize("T,n,temp", [(1, 2, 0.3), (2, 3, 0.3), (5, 9, 0.3), (33, 3, 0.3),
+                                      (64, 2, 0.01)])
+def test_vjp_edge_shapes_random_cotangent(tcq, L, T, n, temp):
+    # ragged batches, short sequences and a low temperature, through both
+    # gradient entry points (separate backward and the one-sweep form)
+    s = W.gaussian(n, 1300 + T, seq_len=T)
+    v = W.gaussian(n, 1400 + T, seq_len=T)
+    sd, vd = _dev(s), _dev(v)
+    soft, _ = tcq.bcjr_soft(sd, L, temp)
+    g1 = tcq.bcjr_soft_backward(sd, L, temp, soft, vd)
+    soft2, lz2, g2 = tcq.bcjr_soft_and_grad(sd, L, temp, vd)
+    torch.cuda.synchronize()
+    rg, rsoft = oracle.bcjr_vjp(s, v, L, temp)
+    assert np.abs(soft2.cpu().numpy() - rsoft).max() <= SOFT_ATOL
+    for g in (g1.cpu().numpy(), g2.cpu().numpy()):
+        for i in range(n):
+            tol = GRAD_RTOL_OF_MAX * np.abs(rg[i]).max() + 1e-6
+            assert np.abs(g[i] - rg[i]).max() <= tol, (i, np.abs(g[i] - rg[i]).max(), tol)
+
+
 def test_vjp_random_cotangent_and_autograd(tcq):
     s = W.gaussian(5, 61, seq_len=40)
     v = W.gaussian(5, 62, seq_len=40)

@@ -98,6 +98,15 @@ def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str,
     raise KeyError(kernel)
 
 
+def trellis_edges(kernel: str, workload, T: int = SEQ_LEN) -> float:
+    """Trellis edges one launch covers, 2^(L+k) (T-1) n with k = 2 (twice for
+    the two-run tail-biting encode); 0 for kernels that walk no trellis."""
+    if kernel.startswith(("viterbi", "bcjr")):
+        runs = 2 if kernel.startswith("viterbi_tb") else 1
+        return runs * float(1 << (workload.L + 2)) * (T - 1) * workload.n_seq
+    return 0.0
+
+
 def roofline_entry(kernel: str, workload, ms: float, peaks: dict) -> dict:
     bound, work, unit = kernel_work(kernel, workload.L, workload.n_seq)
     traffic = measured_traffic(kernel, workload)
