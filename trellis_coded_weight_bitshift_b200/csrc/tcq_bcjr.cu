@@ -68,7 +68,8 @@ __device__ __forceinline__ float lse4_base2(float x0, float x1, float x2, float 
   return mx + lg2(S);
 }
 
-template <int L_, int G_, int SPC_, int AREG_, int NBUF_, bool GRAD_, int MINB_ = 1>
+template <int L_, int G_, int SPC_, int AREG_, int NBUF_, bool GRAD_, int MINB_ = 1,
+          bool TMEMC_ = false>
 struct BcjrCfg {
   static constexpr int L = L_, G = G_, SPC = SPC_, AREG = AREG_, NBUF = NBUF_;
   static constexpr int MINB = MINB_;                // CTAs per SM the registers must allow
@@ -78,7 +79,11 @@ struct BcjrCfg {
   static constexpr int NT = TPS * SPC;
   static constexpr int GQ = G / 4;
   static constexpr int ASM = 4 - AREG;
-  static constexpr int HREG = AREG / 2, HS = 2 - HREG;          // digit pairs: registers | smem
+  static constexpr int HREG = AREG / 2, HS = 2 - HREG;          // digit pairs: registers | elsewhere
+  // the HS pairs not in registers sit in tensor memory (TMEMC) or shared memory
+  static constexpr bool TMEMC = TMEMC_;
+  static constexpr int TCPT = TMEMC ? HS * G * 2 : 0;              // TMEM columns per thread
+  static constexpr int TCOLS = TCPT * (NT / 128) <= 32 ? 32 : TCPT * (NT / 128);  // per CTA
   static constexpr int NPART = TPS >= 32 ? TPS / 32 : 1;       // partial records per sequence
   static constexpr int PREC = 8;                                 // floats per partial record
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
@@ -86,7 +91,7 @@ struct BcjrCfg {
   static constexpr int SPILL = NV * G;                           // floats spilled per thread-step
   static constexpr size_t smem_floats() {
     return (size_t)SPC * NBUF * NV * NG                            // state vectors
-           + (size_t)ASM * G * TPS                                  // smem code values
+           + (TMEMC ? 0 : (size_t)ASM * G * TPS)                    // smem code values
            + (size_t)SPC * 256 * (GRAD ? 4 : 2)                     // s, kappa*D (+ v, soft)
            + (size_t)SPC * 256                                       // CA_t prefix sums
            + (size_t)2 * SPC * NPART * PREC;                        // partial records
@@ -95,30 +100,48 @@ struct BcjrCfg {
   __host__ __device__ static constexpr size_t ws_floats_per_slot(int T) { return (size_t)T * NV * NG; }
   static_assert(NG % G == 0 && G % 4 == 0, "bad split");
   static_assert(AREG % 2 == 0, "code values are held in digit pairs");
+  static_assert(!TMEMC || (SPC == 1 && NT % 128 == 0 && (TCOLS & (TCOLS - 1)) == 0 && TCOLS <= 512 &&
+                           G % 8 == 0), "tensor-memory code layout");
   static_assert(SPILL % 4 == 0, "spill in float4 chunks");
 };
 
 // Code values are held as vertical pairs over the predecessor digit:
-// cv[h][i] = (code of state 2h NG + G w + i, code of state (2h+1) NG + G w + i),
-// digit pairs h < HREG in registers, the others in shared memory as float2
-// [HS][G][TPS] (consecutive lanes read consecutive pairs).
+// pair (h, i) = (code of state 2h NG + G w + i, code of state (2h+1) NG + G w + i).
+// Digit pairs h < HREG live in registers; the others in tensor memory (this
+// thread's lane, columns col0 + 2 ((h - HREG) G + i) and + 1) or in shared
+// memory as float2 [HS][G][TPS] (consecutive lanes read consecutive pairs).
 template <class C>
 using CodeRegs = f2_t[C::HREG > 0 ? C::HREG : 1][C::G];
 
 template <class C>
-__device__ __forceinline__ f2_t code_vpair(const CodeRegs<C> &cv, const float2 *Csm, int h, int i,
-                                          int w) {
-  if (h < C::HREG) return cv[h < C::HREG ? h : 0][i];
-  const float2 v = Csm[((h - C::HREG) * C::G + i) * C::TPS + w];
-  return f2(v.x, v.y);
-}
-
-template <class C>
-__device__ __forceinline__ float code_at(const CodeRegs<C> &cv, const float2 *Csm, int a, int i,
-                                         int w) {
-  const f2_t v = code_vpair<C>(cv, Csm, a >> 1, i, w);
-  return (a & 1) ? f2hi(v) : f2lo(v);
-}
+struct CodeSrc {
+  const CodeRegs<C> &cv;
+  const float2 *Csm;
+  uint32_t taddr;                                          // this thread's TMEM lane, column 0
+  int w;
+  // N consecutive pairs (h, i0 .. i0 + N - 1); N = 4 or 8, i0 a multiple of N
+  template <int N>
+  __device__ __forceinline__ void pairs(int h, int i0, f2_t (&out)[N]) const {
+    if (h < C::HREG) {
+#pragma unroll
+      for (int n = 0; n < N; ++n) out[n] = cv[h < C::HREG ? h : 0][i0 + n];
+    } else if constexpr (C::TMEMC) {
+      float r[2 * N];
+      const uint32_t col = 2 * ((h - C::HREG) * C::G + i0);
+      if constexpr (N == 4) tmem_ld8(taddr + col, r);
+      else tmem_ld16(taddr + col, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int n = 0; n < N; ++n) out[n] = f2(r[2 * n], r[2 * n + 1]);
+    } else {
+#pragma unroll
+      for (int n = 0; n < N; ++n) {
+        const float2 v = Csm[((h - C::HREG) * C::G + i0 + n) * C::TPS + w];
+        out[n] = f2(v.x, v.y);
+      }
+    }
+  }
+};
 
 // Reduce within the TPS lanes of a sequence (TPS < 32) or the whole warp.
 template <int TPS, class Op>
@@ -230,7 +253,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   extern __shared__ __align__(16) float smem[];
   float *Vall = smem;                                      // [SPC][NB][NV][NG]
   float2 *Csm = reinterpret_cast<float2 *>(Vall + SPC * NB * NV * NG);  // [HS][G][TPS]
-  float *ssm = reinterpret_cast<float *>(Csm + C::HS * G * TPS);        // [SPC][256]
+  float *ssm = reinterpret_cast<float *>(Csm + (C::TMEMC ? 0 : C::HS * G * TPS));  // [SPC][256]
   float *ksm = ssm + SPC * 256;                            // [SPC][256] kappa * D_t
   float *vsm = ksm + SPC * 256;                            // GRAD: v, soft rows
   float *fsm = vsm + (GRAD ? SPC * 256 : 0);
@@ -250,13 +273,36 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     for (int i = 0; i < G; ++i)
       cv[h][i] = f2(one_mad_f32((uint32_t)(2 * h * NG + G * w + i)),
                     one_mad_f32((uint32_t)((2 * h + 1) * NG + G * w + i)));
-  if (ls == 0) {
+  __shared__ uint32_t tmem_base;
+  uint32_t taddr = 0;
+  if constexpr (C::TMEMC) {
+    // one allocation per CTA; thread (warp, lane) owns TMEM lane 32 (warp % 4) +
+    // lane, columns (warp / 4) TCPT .. + TCPT - 1
+    if (tid < 32) tmem_alloc(&tmem_base, C::TCOLS);
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    const int warp = tid >> 5;
+    taddr = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)((warp >> 2) * C::TCPT);
+    for (int h = C::HREG; h < 2; ++h)
+      for (int i = 0; i < G; i += 4) {
+        float v[8];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          v[2 * n] = one_mad_f32((uint32_t)(2 * h * NG + G * w + i + n));
+          v[2 * n + 1] = one_mad_f32((uint32_t)((2 * h + 1) * NG + G * w + i + n));
+        }
+        tmem_st8(taddr + 2 * ((h - C::HREG) * G + i), v);
+      }
+    tmem_wait_st();
+  } else if (ls == 0) {
     for (int h = C::HREG; h < 2; ++h)
       for (int i = 0; i < G; ++i)
         Csm[((h - C::HREG) * G + i) * TPS + w] =
             make_float2(one_mad_f32((uint32_t)(2 * h * NG + G * w + i)),
                         one_mad_f32((uint32_t)((2 * h + 1) * NG + G * w + i)));
   }
+  const CodeSrc<C> codes{cv, Csm, taddr, w};
 
   // thread-private spill: [T][NCH][TPS] float4; step t holds A_t (and Phi_t)
   // at this thread's groups r = a*NG/4 + GQ*w + k, flattened as a*GQ + k.
@@ -336,10 +382,13 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           const f2_t am0 = f2sub(f2(ain[0][q], ain[1][q]), cm2);
           const f2_t am1 = f2sub(f2(ain[2][q], ain[3][q]), cm2);
           float outA[4];
+          f2_t cq0[4], cq1[4];
+          codes.template pairs<4>(0, 4 * q, cq0);
+          codes.template pairs<4>(1, 4 * q, cq1);
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const f2_t d0 = f2sub(code_vpair<C>(cv, Csm, 0, 4 * q + r, w), sv2);
-            const f2_t d1 = f2sub(code_vpair<C>(cv, Csm, 1, 4 * q + r, w), sv2);
+            const f2_t d0 = f2sub(cq0[r], sv2);
+            const f2_t d1 = f2sub(cq1[r], sv2);
             const f2_t x0 = f2fma(f2mul(d0, nk2), d0, am0);
             const f2_t x1 = f2fma(f2mul(d1, nk2), d1, am1);
             outA[r] = lse4_base2(f2lo(x0), f2hi(x0), f2lo(x1), f2hi(x1));
@@ -357,10 +406,13 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           const f2_t ph0 = f2sub(f2(fin[0][q], fin[1][q]), vf2);
           const f2_t ph1 = f2sub(f2(fin[2][q], fin[3][q]), vf2);
           float outA[4], outF[4];
+          f2_t cq0[4], cq1[4];
+          codes.template pairs<4>(0, 4 * q, cq0);
+          codes.template pairs<4>(1, 4 * q, cq1);
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const f2_t c0 = code_vpair<C>(cv, Csm, 0, 4 * q + r, w);
-            const f2_t c1 = code_vpair<C>(cv, Csm, 1, 4 * q + r, w);
+            const f2_t c0 = cq0[r];
+            const f2_t c1 = cq1[r];
             const f2_t d0 = f2sub(c0, sv2), d1 = f2sub(c1, sv2);
             const f2_t x0 = f2fma(f2mul(d0, nk2), d0, am0);
             const f2_t x1 = f2fma(f2mul(d1, nk2), d1, am1);
@@ -409,9 +461,11 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
 #pragma unroll
         for (int k = 0; k < GQ; ++k) {
           float y[4];
+          f2_t cp[4];
+          codes.template pairs<4>(a >> 1, 4 * k, cp);
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
-            const float d = code_at<C>(cv, Csm, a, 4 * k + b, w) - sT;
+            const float d = ((a & 1) ? f2hi(cp[b]) : f2lo(cp[b])) - sT;
             y[b] = -ksm[ls * 256 + T - 1] * d * d;
           }
           const float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
@@ -536,13 +590,23 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
             spilled_run(G + (2 * h + 1) * GQ + KB * kb, fah);
           }
           float outL[KB], outH[KB], outPL[GRAD ? KB : 1], outPH[GRAD ? KB : 1];
+          // code pairs (h, 4k + b) of this block: one tensor-memory load for the
+          // block, else four pairs per group index as it is reached
+          constexpr bool BLK = C::TMEMC && KB == 2;
+          f2_t cb[BLK ? 8 : 1];
+          if constexpr (BLK) codes.template pairs<8>(h, 8 * kb, cb);
 #pragma unroll
           for (int j = 0; j < KB; ++j) {
             const int k = KB * kb + j;
             f2_t cc[4], y[4];
+            if constexpr (BLK) {
+#pragma unroll
+              for (int b = 0; b < 4; ++b) cc[b] = cb[BLK ? 4 * j + b : 0];
+            } else {
+              codes.template pairs<4>(h, 4 * k, cc);
+            }
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-              cc[b] = code_vpair<C>(cv, Csm, h, 4 * k + b, w);
               const f2_t d = f2sub(cc[b], sv2);
               y[b] = f2fma(f2mul(d, nk2), d, f2(bin[4 * k + b], bin[4 * k + b]));
             }
@@ -635,6 +699,12 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         grad_out[seq * T] = (1.3862943611198906f * ksm[ls * 256]) * (n2 * inv - (num * inv) * (n1 * inv));
     }
   }
+  if constexpr (C::TMEMC) {                                // every thread is done with its lane
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    if (tid < 32) tmem_dealloc(tmem_base, C::TCOLS);
+  }
 }
 
 }  // namespace tcq
@@ -649,7 +719,14 @@ using Soft8 = BcjrCfg<8, 4, 8, 4, 2, false>;
 // reads every code value from shared memory, the gradient pass keeps digits
 // 0 and 1 in registers (the register file allows 72 per thread)
 using Soft12 = BcjrCfg<12, 8, 1, 0, 2, false, 7>;
-using Soft16 = BcjrCfg<16, 32, 1, 2, 1, false>;
+// L = 16: one 512-thread CTA per SM; all 2^16 code values sit in tensor memory
+// (128 columns per thread, the whole 512-column allocation), which leaves the
+// shared memory for a double-buffered state vector (one barrier per step).
+// Measured against code values half in registers and half in shared memory
+// with a single buffer: 32.1 vs 36.2 ms on 2,048 sequences.  At L = 12 (seven
+// CTAs per SM) the same layout was 2.2x slower than shared memory, so it is
+// used here only.
+using Soft16 = BcjrCfg<16, 32, 1, 0, 2, false, 1, true>;
 using Grad8 = BcjrCfg<8, 4, 8, 4, 2, true>;
 using Grad12 = BcjrCfg<12, 8, 1, 2, 2, true, 7>;
 
