@@ -119,7 +119,7 @@ struct CodeSrc {
   const float2 *Csm;
   uint32_t taddr;                                          // this thread's TMEM lane, column 0
   int w;
-  // N consecutive pairs (h, i0 .. i0 + N - 1); N = 4 or 8, i0 a multiple of N
+  // N consecutive pairs (h, i0 .. i0 + N - 1); N = 4, 8 or 16, i0 a multiple of N
   template <int N>
   __device__ __forceinline__ void pairs(int h, int i0, f2_t (&out)[N]) const {
     if (h < C::HREG) {
@@ -129,7 +129,8 @@ struct CodeSrc {
       float r[2 * N];
       const uint32_t col = 2 * ((h - C::HREG) * C::G + i0);
       if constexpr (N == 4) tmem_ld8(taddr + col, r);
-      else tmem_ld16(taddr + col, r);
+      else if constexpr (N == 8) tmem_ld16(taddr + col, r);
+      else tmem_ld32(taddr + col, r);
       tmem_wait_ld();
 #pragma unroll
       for (int n = 0; n < N; ++n) out[n] = f2(r[2 * n], r[2 * n + 1]);
@@ -139,6 +140,24 @@ struct CodeSrc {
         const float2 v = Csm[((h - C::HREG) * C::G + i0 + n) * C::TPS + w];
         out[n] = f2(v.x, v.y);
       }
+    }
+  }
+  // pairs (0, i0 ..) and (1, i0 ..) of 4 consecutive indices, with a single
+  // tensor-memory wait when both come from there
+  __device__ __forceinline__ void both_pairs4(int i0, f2_t (&out0)[4], f2_t (&out1)[4]) const {
+    if constexpr (C::TMEMC && C::HREG == 0) {
+      float r0[8], r1[8];
+      tmem_ld8(taddr + 2 * i0, r0);
+      tmem_ld8(taddr + 2 * (C::G + i0), r1);
+      tmem_wait_ld();
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        out0[n] = f2(r0[2 * n], r0[2 * n + 1]);
+        out1[n] = f2(r1[2 * n], r1[2 * n + 1]);
+      }
+    } else {
+      pairs<4>(0, i0, out0);
+      pairs<4>(1, i0, out1);
     }
   }
 };
@@ -383,8 +402,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           const f2_t am1 = f2sub(f2(ain[2][q], ain[3][q]), cm2);
           float outA[4];
           f2_t cq0[4], cq1[4];
-          codes.template pairs<4>(0, 4 * q, cq0);
-          codes.template pairs<4>(1, 4 * q, cq1);
+          codes.both_pairs4(4 * q, cq0, cq1);
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const f2_t d0 = f2sub(cq0[r], sv2);
@@ -407,8 +425,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           const f2_t ph1 = f2sub(f2(fin[2][q], fin[3][q]), vf2);
           float outA[4], outF[4];
           f2_t cq0[4], cq1[4];
-          codes.template pairs<4>(0, 4 * q, cq0);
-          codes.template pairs<4>(1, 4 * q, cq1);
+          codes.both_pairs4(4 * q, cq0, cq1);
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const f2_t c0 = cq0[r];
@@ -566,7 +583,9 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       const f2_t K2 = f2(K, K), dp2 = f2(dprev, dprev), vv2 = f2(vv, vv);
       f2_t num2 = f2(0.0f, 0.0f), den2 = num2, n12 = num2, n22 = num2;
       // KB values of this thread's spilled vector at flat index f (KB | f)
-      constexpr int KB = GQ < 2 ? GQ : 2;
+      // sub-run width: 4 when the code values come from tensor memory (the
+      // registers they free hold the wider block), else 2
+      constexpr int KB = GQ < 2 ? GQ : (C::TMEMC && GQ >= 4 ? 4 : 2);
       auto spilled_run = [&](int f, float *dst) {
         float4 v;
         if constexpr (PREFETCH) v = avq[PREFETCH ? (f >> 2) : 0];
@@ -592,9 +611,9 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           float outL[KB], outH[KB], outPL[GRAD ? KB : 1], outPH[GRAD ? KB : 1];
           // code pairs (h, 4k + b) of this block: one tensor-memory load for the
           // block, else four pairs per group index as it is reached
-          constexpr bool BLK = C::TMEMC && KB == 2;
-          f2_t cb[BLK ? 8 : 1];
-          if constexpr (BLK) codes.template pairs<8>(h, 8 * kb, cb);
+          constexpr bool BLK = C::TMEMC && KB >= 2;
+          f2_t cb[BLK ? 4 * KB : 1];
+          if constexpr (BLK) codes.template pairs<BLK ? 4 * KB : 4>(h, 4 * KB * kb, cb);
 #pragma unroll
           for (int j = 0; j < KB; ++j) {
             const int k = KB * kb + j;
