@@ -80,9 +80,11 @@ __global__ void __launch_bounds__(256) rht_rows_kernel(const float *__restrict__
 //            column signs and runs the log2(E) butterfly levels over a in
 //            registers, then stores to shared memory;
 //   stage 2: thread (group a, m < P = 256/E) reads the E consecutive values
-//            a*256 + m*E .. + E-1, runs log2(E) levels in registers and the
-//            last log2(P) levels across the P lanes of its group with
-//            shuffles, and writes its E outputs (row sign and 1/sqrt C).
+//            a*256 + m*E .. + E-1 and runs log2(E) levels in registers;
+//   stage 3: the last log2(P) levels: for E >= 16 after a second pass through
+//            shared memory, in registers, with coalesced stores; for E = 8
+//            across the P lanes of a group with shuffles.  Row sign and
+//            1/sqrt C on the store.
 // Shared memory holds the row with 4 floats of padding per 32, which keeps
 // both the stage-1 stores and the stage-2 vector loads bank-conflict free.
 template <int LC>
@@ -131,20 +133,53 @@ __global__ void __launch_bounds__(256, LC == 13 ? 3 : 4) rht_rows_reg_kernel(con
           v[i] = x + y;
           v[i + h] = x - y;
         }
-#pragma unroll
-    for (int d = 1; d < P; d <<= 1) {
-      const bool upper = (m & d) != 0;
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, v[i], d);
-        v[i] = upper ? o - v[i] : v[i] + o;
-      }
-    }
     const float f = sign_rows[r] * scale;
-    float4 *dst = reinterpret_cast<float4 *>(out + (int64_t)r * C + base);
+    if constexpr (E >= 16) {
+      // stage 3: back through shared memory; thread (lane, warp) takes the P
+      // values a*256 + m*E + bl (m < P) for bl = its lane (mod E) and E*E/256
+      // values of a, and runs the last log2(P) levels in registers
 #pragma unroll
-    for (int q = 0; q < E / 4; ++q)
-      dst[q] = make_float4(v[4 * q] * f, v[4 * q + 1] * f, v[4 * q + 2] * f, v[4 * q + 3] * f);
+      for (int q = 0; q < E / 4; ++q)
+        *reinterpret_cast<float4 *>(xs + pad(base + 4 * q)) =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      __syncthreads();
+      constexpr int NA = E * E / 256;                     // values of a per thread
+      const int lane = t & 31, w = t >> 5;
+      const int bl = lane & (E - 1);
+#pragma unroll
+      for (int k = 0; k < NA; ++k) {
+        const int a = (E == 32) ? (w * NA + k) : (2 * w + (lane >> 4));
+        float u[P];
+#pragma unroll
+        for (int mm = 0; mm < P; ++mm) u[mm] = xs[pad(a * 256 + mm * E + bl)];
+#pragma unroll
+        for (int h = 1; h < P; h <<= 1)
+#pragma unroll
+          for (int i = 0; i < P; ++i)
+            if ((i & h) == 0) {
+              const float x = u[i], y = u[i + h];
+              u[i] = x + y;
+              u[i + h] = x - y;
+            }
+        float *dst = out + (int64_t)r * C + a * 256 + bl;
+#pragma unroll
+        for (int mm = 0; mm < P; ++mm) dst[mm * E] = u[mm] * f;
+      }
+    } else {
+#pragma unroll
+      for (int d = 1; d < P; d <<= 1) {
+        const bool upper = (m & d) != 0;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const float o = __shfl_xor_sync(0xffffffffu, v[i], d);
+          v[i] = upper ? o - v[i] : v[i] + o;
+        }
+      }
+      float4 *dst = reinterpret_cast<float4 *>(out + (int64_t)r * C + base);
+#pragma unroll
+      for (int q = 0; q < E / 4; ++q)
+        dst[q] = make_float4(v[4 * q] * f, v[4 * q + 1] * f, v[4 * q + 2] * f, v[4 * q + 3] * f);
+    }
     __syncthreads();                                      // xs is rewritten by the next row
   }
 }
