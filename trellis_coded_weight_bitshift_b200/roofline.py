@@ -42,11 +42,10 @@ MEASURED_TRAFFIC = {
         "tcq_bcjr.cu": "74c770c6300308e4af2802c9ca117ef3f97ebf3d",
         "tcq_device.cuh": "804f75be759c65adfd0397217b44b3edffd5549a"}),
     # three launches (row pass, two column passes) of one 8192 x 8192 rotation
-    ("rht", "rht_t5_8192sq"): (268.563712e6 + 223.412224e6 + 268.515328e6 + 209.742592e6
-                               + 268.464896e6 + 209.4656e6, 262144, {
-        "tcq_rht.cu": "ccfacb475702414c5cd2f49317f76388abbd2f52",
-        # the header has since gained only a reciprocal helper the rotation does not use
-        "tcq_device.cuh": "804f75be759c65adfd0397217b44b3edffd5549a"}),
+    ("rht", "rht_t5_8192sq"): (270.228992e6 + 227.542272e6 + 268.456448e6 + 211.080448e6
+                               + 268.458496e6 + 210.584832e6, 262144, {
+        "tcq_rht.cu": "2eca83490f30669a46e44c81714f1c900931fb37",
+        "tcq_device.cuh": "e3ed67190c0bcd2311f690b228049c02882ca990"}),
 }
 
 
