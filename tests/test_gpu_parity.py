@@ -487,6 +487,29 @@ def test_decode_gemv_matches_oracle(tcq, L, layout, rows, cols):
     assert np.all(np.abs(y - ref) <= bound + 1e-30)
 
 
+@pytest.mark.parametrize("case", ["wide_range", "large", "zeros", "tiny"])
+def test_decode_gemv_activation_ranges(tcq, case):
+    # fp32 activations spanning many decades, far above fp16's range, exactly
+    # zero, or far below it: the products stay fp32, so the same bound holds
+    rows, cols = 64, 4096
+    rng = np.random.default_rng(77)
+    bits = rng.integers(0, 2 ** 32, ((rows // 16) * (cols // 16), 16), dtype=np.uint32)
+    x = rng.standard_normal(cols)
+    if case == "wide_range":
+        x = x * 10.0 ** rng.uniform(-4, 5, cols)
+    elif case == "large":
+        x = x * 1e7
+    elif case == "zeros":
+        x = np.zeros(cols)
+    else:
+        x = x * 1e-9
+    x = x.astype(np.float32)
+    y = tcq.decode_gemv(_dev(bits.view(np.int32)).view(torch.uint32), _dev(x), rows, cols).cpu().numpy()
+    ref, bound = _gemv_ref(bits, rows, cols, x)
+    assert np.all(np.isfinite(y))
+    assert np.all(np.abs(y - ref) <= bound + 1e-30)
+
+
 def test_decode_gemv_8192_square_sampled_rows(tcq):
     bits = W.streams("l16_decode_8192sq")
     x = np.random.default_rng(8).standard_normal(8192).astype(np.float32)
