@@ -632,13 +632,26 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
             const float mxl = fmaxf(fmaxf(f2lo(y[0]), f2lo(y[1])), fmaxf(f2lo(y[2]), f2lo(y[3])));
             const float mxh = fmaxf(fmaxf(f2hi(y[0]), f2hi(y[1])), fmaxf(f2hi(y[2]), f2hi(y[3])));
             const f2_t mx2 = f2(mxl, mxh);
-            f2_t u[4];
+            // sums over the four successors, accumulated one successor at a
+            // time (fewer live registers than four separate weights)
+            f2_t su, sc, sz, scz;
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
               const f2_t e = f2sub(y[b], mx2);
-              u[b] = f2(ex2(f2lo(e)), ex2(f2hi(e)));
+              const f2_t u = f2(ex2(f2lo(e)), ex2(f2hi(e)));
+              su = b == 0 ? u : f2add(su, u);
+              if constexpr (!GRAD) {
+                sc = b == 0 ? f2mul(u, cc[b]) : f2fma(u, cc[b], sc);
+              } else {
+                const f2_t uc = f2mul(u, cc[b]);
+                sc = b == 0 ? uc : f2add(sc, uc);
+                // z_b = psi_{tc}(succ) + v_tc (c_b - soft_tc)
+                const float pz = pin[4 * k + b] + nvf;
+                const f2_t z = f2fma(vv2, cc[b], f2(pz, pz));
+                sz = b == 0 ? f2mul(u, z) : f2fma(u, z, sz);
+                scz = b == 0 ? f2mul(uc, z) : f2fma(uc, z, scz);
+              }
             }
-            const f2_t su = f2add(f2add(u[0], u[2]), f2add(u[1], u[3]));
             const f2_t ob = f2add(f2sub(mx2, dp2), f2(lg2(f2lo(su)), lg2(f2hi(su))));
             outL[j] = f2lo(ob);
             outH[j] = f2hi(ob);
@@ -646,29 +659,12 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
             const f2_t wv = f2add(f2sub(f2(avl[j], avh[j]), K2), mx2);
             const f2_t wgt = f2(ex2(f2lo(wv)), ex2(f2hi(wv)));
             den2 = f2fma(wgt, su, den2);
-            if constexpr (!GRAD) {
-              const f2_t sc = f2add(f2fma(u[2], cc[2], f2mul(u[0], cc[0])),
-                                    f2fma(u[3], cc[3], f2mul(u[1], cc[1])));
-              num2 = f2fma(wgt, sc, num2);
-            } else {
-              // z_b = psi_{tc}(succ) + v_tc (c_b - soft_tc)
-              f2_t z[4], uc[4];
-#pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                const float pz = pin[4 * k + b] + nvf;
-                z[b] = f2fma(vv2, cc[b], f2(pz, pz));
-                uc[b] = f2mul(u[b], cc[b]);
-              }
-              const f2_t sc = f2add(f2add(uc[0], uc[2]), f2add(uc[1], uc[3]));
-              const f2_t sz = f2add(f2fma(u[2], z[2], f2mul(u[0], z[0])),
-                                    f2fma(u[3], z[3], f2mul(u[1], z[1])));
-              const f2_t scz = f2add(f2fma(uc[2], z[2], f2mul(uc[0], z[0])),
-                                     f2fma(uc[3], z[3], f2mul(uc[1], z[1])));
+            num2 = f2fma(wgt, sc, num2);
+            if constexpr (GRAD) {
               const f2_t op = f2mul(sz, f2(rcp(f2lo(su)), rcp(f2hi(su))));
               outPL[j] = f2lo(op);
               outPH[j] = f2hi(op);
               const f2_t fa2 = f2(fal[j], fah[j]);
-              num2 = f2fma(wgt, sc, num2);
               n12 = f2fma(wgt, f2fma(fa2, su, sz), n12);
               n22 = f2fma(wgt, f2fma(fa2, sc, scz), n22);
             }
