@@ -66,21 +66,13 @@ __device__ __forceinline__ unsigned long long one_mad_decode_f32x2(uint32_t x0, 
 // square as fma(d, d, +0), which rounds exactly like d * d for d * d >= 0 and
 // cannot be fused further.
 typedef unsigned long long f2_t;
+// Pair construction and halves in plain C++ (bit moves the compiler sees
+// through, so a pair can live in two adjacent registers without copies).
 __device__ __forceinline__ f2_t f2(float lo, float hi) {
-  f2_t r;
-  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
+  return ((f2_t)__float_as_uint(hi) << 32) | (f2_t)__float_as_uint(lo);
 }
-__device__ __forceinline__ float f2lo(f2_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
-}
-__device__ __forceinline__ float f2hi(f2_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
-}
+__device__ __forceinline__ float f2lo(f2_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2hi(f2_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
 __device__ __forceinline__ f2_t f2sub(f2_t a, f2_t b) {
   f2_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
