@@ -38,14 +38,14 @@ MUFU_PER_SM = 16               # special-function results per clock per SM
 # null.  (kernel prefix, workload): (bytes, sequences in the capture, sources)
 _CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 MEASURED_TRAFFIC = {
-    ("bcjr_soft_vjp", "l12_gauss1024"): (2.105008384e9 + 2.183070976e9, 1024, {
-        "tcq_bcjr.cu": "a99d7cebe4737199a15bbfe56abf5c52b3fb1763",
-        "tcq_device.cuh": "e3ed67190c0bcd2311f690b228049c02882ca990"}),
+    ("bcjr_soft_vjp", "l12_gauss1024"): (2.105408e9 + 2.181073664e9, 1024, {
+        "tcq_bcjr.cu": "6617a7096717c0495f8afc8a697e8984401ea6f4",
+        "tcq_device.cuh": "18b7f3a092c947f32accdefd8d22f8b99f58c38e"}),
     # three launches (row pass, two column passes) of one 8192 x 8192 rotation
-    ("rht", "rht_t5_8192sq"): (270.228992e6 + 227.542272e6 + 268.456448e6 + 211.080448e6
-                               + 268.458496e6 + 210.584832e6, 262144, {
+    ("rht", "rht_t5_8192sq"): (269.954048e6 + 226.045952e6 + 268.44288e6 + 206.207232e6
+                               + 268.502272e6 + 206.875136e6, 262144, {
         "tcq_rht.cu": "2eca83490f30669a46e44c81714f1c900931fb37",
-        "tcq_device.cuh": "e3ed67190c0bcd2311f690b228049c02882ca990"}),
+        "tcq_device.cuh": "18b7f3a092c947f32accdefd8d22f8b99f58c38e"}),
 }
 
 
