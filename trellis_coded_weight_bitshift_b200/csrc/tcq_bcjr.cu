@@ -97,7 +97,16 @@ struct BcjrCfg {
            + (size_t)2 * SPC * NPART * PREC;                        // partial records
   }
   static constexpr size_t smem_bytes() { return smem_floats() * sizeof(float); }
-  __host__ __device__ static constexpr size_t ws_floats_per_slot(int T) { return (size_t)T * NV * NG; }
+  // The soft pass finishes its steps after the backward (the per-step sums go
+  // to the workspace); the gradient pass, short of registers, finishes each
+  // step one step later from the shared partial records.
+  static constexpr bool DEFER = !GRAD;
+  // per resident sequence: the spilled messages, then (DEFER) the per-step
+  // partial sums (numerator, denominator) of each warp; a whole number of
+  // 256-byte units, so that every slot (read as float4) stays 16-byte aligned
+  __host__ __device__ static constexpr size_t ws_floats_per_slot(int T) {
+    return ((size_t)T * NV * NG + (DEFER ? (size_t)T * NPART * 2 : 0) + 63) / 64 * 64;
+  }
   static_assert(NG % G == 0 && G % 4 == 0, "bad split");
   static_assert(AREG % 2 == 0, "code values are held in digit pairs");
   static_assert(!TMEMC || (SPC == 1 && NT % 128 == 0 && (TCOLS & (TCOLS - 1)) == 0 && TCOLS <= 512 &&
@@ -327,6 +336,9 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   // at this thread's groups r = a*NG/4 + GQ*w + k, flattened as a*GQ + k.
   float4 *spill = reinterpret_cast<float4 *>(ws + (size_t)(blockIdx.x * SPC + ls) *
                                                       C::ws_floats_per_slot(T));
+  // DEFER: [T][NPART] records of (numerator, denominator), read back once the
+  // backward is done
+  float *sums = reinterpret_cast<float *>(spill) + (size_t)T * NV * NG;
   auto prec = [&](int parity) { return part + ((parity * SPC + ls) * NPART) * PREC; };
 
   for (int64_t base = (int64_t)blockIdx.x * SPC; base < n_seq; base += (int64_t)gridDim.x * SPC) {
@@ -557,7 +569,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         dprev = pp[0];
 #pragma unroll
         for (int x = 1; x < NPART; ++x) dprev = fmaxf(dprev, pp[x * PREC]);
-        if (w == 0 && active) {                              // finish step tc + 1
+        if (!C::DEFER && w == 0 && active) {                 // finish step tc + 1
           float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f;
 #pragma unroll
           for (int x = 0; x < NPART; ++x) {
@@ -695,12 +707,28 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         const float mine = seq_sums<TPS, NQ>(q4, lane);
         const int o = lane & (WL - 1);
         float *pp = prec(tc & 1) + pidx * PREC;
-        if ((o & (WL / NQ - 1)) == 0) pp[1 + o / (WL / NQ)] = mine;   // num, den, n1, n2
+        if ((o & (WL / NQ - 1)) == 0) {                                  // num, den (n1, n2)
+          if constexpr (C::DEFER) sums[((size_t)tc * NPART + pidx) * 2 + o / (WL / NQ)] = mine;
+          else pp[1 + o / (WL / NQ)] = mine;
+        }
         if (plead) pp[0] = tmax;
       }
       __syncthreads();
     }
-    if (w == 0 && active) {                                  // finish step 0
+    if (C::DEFER && active) {
+      // every step's sums are in the workspace (the barrier that closed the
+      // last step orders them): the sequence's threads finish them in parallel
+      for (int u = w; u < T; u += TPS) {
+        float num = 0.0f, den = 0.0f;
+#pragma unroll
+        for (int x = 0; x < NPART; ++x) {
+          num += sums[((size_t)u * NPART + x) * 2];
+          den += sums[((size_t)u * NPART + x) * 2 + 1];
+        }
+        if (soft_out) soft_out[seq * T + u] = num / den;
+      }
+    }
+    if (!C::DEFER && w == 0 && active) {                     // finish step 0
       const float *pp = prec(0);
       float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f;
 #pragma unroll
