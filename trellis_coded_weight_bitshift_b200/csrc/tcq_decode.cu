@@ -176,7 +176,10 @@ static tcq_status_t decode_launch(const tcq_trellis_t *tr, const uint32_t *bits,
   if (out_layout == TCQ_OUT_TILE16) {
     const int64_t ntc = cols / 16;
     const int64_t items = n_seq * 2;
-    const int64_t blocks = std::min<int64_t>((items + 255) / 256, (int64_t)sm_count() * 8);
+    // one item per thread: the block scheduler overlaps one CTA's loads with
+    // another's stores better than a capped grid-stride loop (26.6 vs 28.7 us
+    // on the 8192^2 matrix)
+    const int64_t blocks = std::min<int64_t>((items + 255) / 256, (int64_t)INT32_MAX);
     if (layout == TCQ_TAILBITING)
       decode_tile16_kernel<L, TCQ_TAILBITING><<<(unsigned)blocks, 256, 0, stream>>>(
           bits, (int)ntc, items, wps, (int)cols, out);
