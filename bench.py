@@ -4,7 +4,8 @@
 
 One step = one pass of the whole hot path over one batch of synthetic input:
 for the default workload (L=12, 1024 x 256 i.i.d. N(0,1) weights) that is
-Viterbi encode (forward + traceback, per-sequence MSE), the BCJR soft codeword
+Viterbi encode (forward + traceback, per-sequence MSE), packing the walks into
+2-bit streams and decoding them back to fp16 weights, the BCJR soft codeword
 at temp 0.05 and the gradient of the sum of soft codewords w.r.t. the targets
 (soft codeword, log Z and gradient in one forward-backward sweep, since the
 cotangent is known up front).
@@ -37,7 +38,7 @@ if ROOT not in sys.path:
 import tcq_workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "l12_gauss1024"
-METRIC = "weights quantized/sec (Viterbi + BCJR soft + BCJR gradient)"
+
 
 
 def _args():
@@ -65,6 +66,8 @@ def _metric_for(w: W.Workload) -> str:
         parts.append("Viterbi")
     if "viterbi_tb" in w.ops:
         parts.append("tail-biting Viterbi (two-run)")
+    if "pack_decode" in w.ops:
+        parts.append("pack + decode")
     if "bcjr" in w.ops:
         parts.append("BCJR soft" + (f" x{len(w.temps)} temps" if len(w.temps) > 1 else ""))
     if "bcjr_grad" in w.ops:
@@ -145,7 +148,9 @@ class ClockSampler:
 def _oracle_step(w: W.Workload, s: np.ndarray, D=None) -> None:
     import oracle
     if "viterbi" in w.ops:
-        oracle.viterbi_f32(s, w.L, D=D)
+        st, _ = oracle.viterbi_f32(s, w.L, D=D)
+        if "pack_decode" in w.ops:
+            oracle.decode(oracle.pack(st, w.L, oracle.FREE_START), w.L, s.shape[1], oracle.FREE_START)
     if "viterbi_tb" in w.ops:
         oracle.viterbi_tailbiting_alg4_f32(s, w.L, D=D)
     for temp in w.temps:
@@ -404,6 +409,12 @@ def run_ours(a) -> None:
                 mark("viterbi")
                 n_launch += 2
                 outs += [st, mse]
+                if "pack_decode" in w.ops:
+                    bits = tcq.pack_states(st, w.L, tcq.FREE_START)
+                    dec = tcq.decode(bits, w.L, W.SEQ_LEN, tcq.FREE_START, tcq.OUT_SEQ)
+                    mark("pack_decode_seq")
+                    n_launch += 2
+                    outs.append(dec)
             if "viterbi_tb" in w.ops:
                 st, mse = tcq.viterbi_encode_tailbiting(inp, w.L, ws_v, D=Dd)
                 mark("viterbi_tb")

@@ -201,8 +201,9 @@ TCQ_API tcq_status_t tcq_bcjr_soft(const tcq_trellis_t *trellis, const float *s,
  *   soft       [n_seq][seq_len] the forward output of tcq_bcjr_soft for the
  *              same s and temp (input; used to centre the covariance).
  *   grad_soft  [n_seq][seq_len] fp32 (input), grad_s [n_seq][seq_len] (output).
- *   ws         at least tcq_bcjr_workspace_size(.., 1) bytes.
- * L = 16 returns TCQ_ERR_UNSUPPORTED.
+ *   ws         at least tcq_bcjr_workspace_size(.., 1) bytes (one slot per
+ *              sequence resident on the GPU; at seq_len 256 and L = 16 a slot
+ *              is 32 MiB and one sequence runs per SM, about 5 GB on B200).
  * ------------------------------------------------------------------------ */
 TCQ_API tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *trellis, const float *s,
                                             const float *D, int64_t n_seq, float temp,
@@ -219,7 +220,6 @@ TCQ_API tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *trellis, const 
  * s instead of the soft codeword (an exact identity; only rounding differs).
  *   grad_soft [n_seq][seq_len] (input); soft, log_z (outputs, each may be
  *   NULL); grad_s (output).  Workspace: tcq_bcjr_workspace_size(.., 1).
- *   L = 16 returns TCQ_ERR_UNSUPPORTED.
  * ------------------------------------------------------------------------ */
 TCQ_API tcq_status_t tcq_bcjr_soft_and_grad(const tcq_trellis_t *trellis, const float *s,
                                             const float *D, int64_t n_seq, float temp,

@@ -47,7 +47,7 @@ WORKLOADS = {
     "l8_gauss64": Workload("l8_gauss64", 8, 64, "gaussian", 1, (1.0, 0.1),
                            ops=("viterbi", "bcjr")),
     "l12_gauss1024": Workload("l12_gauss1024", 12, 1024, "gaussian", 2, (0.05,),
-                              ops=("viterbi", "bcjr", "bcjr_grad")),
+                              ops=("viterbi", "pack_decode", "bcjr", "bcjr_grad")),
     "l16_rht1024": Workload("l16_rht1024", 16, 4096, "rht_block", 3, (), 1024, 1024,
                             ops=("viterbi",)),
     "l16_studentt_2048x8192": Workload("l16_studentt_2048x8192", 16, 65536, "student_t", 4,
@@ -64,6 +64,10 @@ WORKLOADS = {
     # random-sign Hadamard rotation of an 8192x8192 Student-t (nu = 5) block
     "rht_t5_8192sq": Workload("rht_t5_8192sq", 16, 262144, "matrix_t5", 7, (), 8192, 8192,
                               ops=("rht",)),
+    # soft codeword and gradient of the sum of soft codewords at L = 16 (QAT at
+    # the 2-bit QTIP setting) on the 1024x1024 RHT block, temp 0.1
+    "l16_rht1024_grad": Workload("l16_rht1024_grad", 16, 4096, "rht_block", 3, (0.1,), 1024, 1024,
+                                 ops=("bcjr", "bcjr_grad")),
     # the 1024x1024 RHT block encoded tail-biting (exactly 2 bits per weight)
     "l16_rht1024_tb": Workload("l16_rht1024_tb", 16, 4096, "rht_block", 3, (), 1024, 1024,
                                ops=("viterbi_tb",)),

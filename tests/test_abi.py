@@ -69,7 +69,9 @@ def test_invalid_arguments_return_status_without_launch(L):
     assert L.tcq_bcjr_soft(ctypes.byref(tr), bad, None, 4, ctypes.c_float(0.0), bad, None, bad, 1 << 30, None) == _abi.TCQ_ERR_INVALID_ARG
     assert L.tcq_bcjr_soft(ctypes.byref(tr), bad, None, 4, ctypes.c_float(float("inf")), bad, None, bad, 1 << 30, None) == _abi.TCQ_ERR_INVALID_ARG
     tr16 = _abi.trellis(16, 256)
-    assert L.tcq_bcjr_soft_backward(ctypes.byref(tr16), bad, None, 4, ctypes.c_float(0.1), bad, bad, bad, bad, 1 << 30, None) == _abi.TCQ_ERR_UNSUPPORTED
+    # the gradient entry points take L = 16 too; a missing workspace is caught on the host
+    assert L.tcq_bcjr_soft_backward(ctypes.byref(tr16), bad, None, 4, ctypes.c_float(0.1), bad, bad, bad, None, 1 << 30, None) == _abi.TCQ_ERR_WORKSPACE
+    assert L.tcq_bcjr_soft_and_grad(ctypes.byref(tr16), bad, None, 4, ctypes.c_float(0.1), bad, bad, None, bad, None, 1 << 30, None) == _abi.TCQ_ERR_WORKSPACE
     # decode: tile shape must cover exactly n_seq tiles
     assert L.tcq_decode(ctypes.byref(tr16), bad, 4, 0, 1, 32, 48, bad, None) == _abi.TCQ_ERR_INVALID_ARG
     assert L.tcq_decode(ctypes.byref(tr16), bad, 4, 0, 1, 32, 30, bad, None) == _abi.TCQ_ERR_INVALID_ARG

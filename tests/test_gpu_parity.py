@@ -263,7 +263,7 @@ def test_vjp_matches_oracle(tcq, name, temp, nsample):
         assert np.abs(g[j] - rg[i]).max() <= tol, (j, np.abs(g[j] - rg[i]).max(), tol)
 
 
-@pytest.mark.parametrize("L", [8, 12])
+@pytest.mark.parametrize("L", [8, 12, 16])
 @pytest.mark.parametrize("T,n,temp", [(1, 2, 0.3), (2, 3, 0.3), (5, 9, 0.3), (33, 3, 0.3),
                                       (64, 2, 0.01)])
 def test_vjp_edge_shapes_random_cotangent(tcq, L, T, n, temp):
@@ -282,6 +282,32 @@ def test_vjp_edge_shapes_random_cotangent(tcq, L, T, n, temp):
         for i in range(n):
             tol = GRAD_RTOL_OF_MAX * np.abs(rg[i]).max() + 1e-6
             assert np.abs(g[i] - rg[i]).max() <= tol, (i, np.abs(g[i] - rg[i]).max(), tol)
+
+
+def test_vjp_l16_rht_block_full(tcq):
+    # L = 16 gradient of the sum of soft codewords on the whole 1024 x 1024 RHT
+    # block (4,096 sequences, the benchmark's launch); the oracle checks a
+    # seeded sample, properties are checked on every sequence
+    w = W.WORKLOADS["l16_rht1024_grad"]
+    s = W.sequences(w.name)
+    temp = w.temps[0]
+    sd = _dev(s)
+    ones = torch.ones_like(sd)
+    soft, lz, g = tcq.bcjr_soft_and_grad(sd, 16, temp, ones)
+    soft_sep, lz_sep = tcq.bcjr_soft(sd, 16, temp)
+    torch.cuda.synchronize()
+    soft, g, soft_sep = soft.cpu().numpy(), g.cpu().numpy(), soft_sep.cpu().numpy()
+    assert np.all(np.isfinite(g)) and np.all(np.isfinite(soft))
+    assert np.abs(soft - soft_sep).max() <= SOFT_ATOL
+    assert np.abs(lz.cpu().numpy() - lz_sep.cpu().numpy()).max() <= 1e-3
+    # v = 1: sum_u grad_u = (2/temp) Var(sum_t code(x_t)) >= 0
+    assert np.all(g.sum(1) >= -GRAD_RTOL_OF_MAX * np.abs(g).sum(1))
+    idx = np.sort(np.random.default_rng(16).choice(s.shape[0], 2, replace=False))
+    rg, rsoft = oracle.bcjr_vjp(s[idx], np.ones((2, 256)), 16, temp)
+    assert np.abs(soft[idx] - rsoft).max() <= SOFT_ATOL
+    for i, j in enumerate(idx):
+        tol = GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+        assert np.abs(g[j] - rg[i]).max() <= tol, (j, np.abs(g[j] - rg[i]).max(), tol)
 
 
 def test_vjp_random_cotangent_and_autograd(tcq):

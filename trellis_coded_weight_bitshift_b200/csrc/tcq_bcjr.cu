@@ -596,8 +596,9 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       f2_t num2 = f2(0.0f, 0.0f), den2 = num2, n12 = num2, n22 = num2;
       // KB values of this thread's spilled vector at flat index f (KB | f)
       // sub-run width: 4 when the code values come from tensor memory (the
-      // registers they free hold the wider block), else 2
-      constexpr int KB = GQ < 2 ? GQ : (C::TMEMC && GQ >= 4 ? 4 : 2);
+      // registers they free hold the wider block) in the soft pass, else 2
+      // (the gradient pass carries B and Psi, twice the values)
+      constexpr int KB = GQ < 2 ? GQ : (C::TMEMC && GQ >= 4 && !GRAD ? 4 : 2);
       auto spilled_run = [&](int f, float *dst) {
         float4 v;
         if constexpr (PREFETCH) v = avq[PREFETCH ? (f >> 2) : 0];
@@ -772,6 +773,10 @@ using Soft12 = BcjrCfg<12, 8, 1, 0, 2, false, 7>;
 using Soft16 = BcjrCfg<16, 32, 1, 0, 2, false, 1, true>;
 using Grad8 = BcjrCfg<8, 4, 8, 4, 2, true>;
 using Grad12 = BcjrCfg<12, 8, 1, 2, 2, true, 7>;
+// L = 16 gradient: code values in tensor memory as in the soft pass; the two
+// carried vectors (A and Phi, 2 x 64 KiB) fit the shared memory only
+// single-buffered, so each step takes two barriers.
+using Grad16 = BcjrCfg<16, 32, 1, 0, 1, true, 1, true>;
 
 template <class C>
 int grid_for(int64_t n_seq) {
@@ -824,7 +829,7 @@ extern "C" size_t tcq_bcjr_workspace_size(const tcq_trellis_t *tr, int64_t n_seq
     switch (tr->L) {
       case 8: return ws_bytes_for<Grad8>(n_seq, T);
       case 12: return ws_bytes_for<Grad12>(n_seq, T);
-      default: return 0;
+      default: return ws_bytes_for<Grad16>(n_seq, T);
     }
   }
   switch (tr->L) {
@@ -866,7 +871,6 @@ extern "C" tcq_status_t tcq_bcjr_soft_and_grad(const tcq_trellis_t *tr, const fl
                                                size_t ws_bytes, void *stream) {
   tcq_status_t st = check_trellis(tr);
   if (st != TCQ_OK) return st;
-  if (tr->L == 16) return TCQ_ERR_UNSUPPORTED;
   if (!temp_ok(temp)) return TCQ_ERR_INVALID_ARG;
   if (n_seq < 0 || n_seq > (int64_t)INT32_MAX) return TCQ_ERR_INVALID_ARG;
   if (n_seq == 0) return TCQ_OK;
@@ -880,7 +884,8 @@ extern "C" tcq_status_t tcq_bcjr_soft_and_grad(const tcq_trellis_t *tr, const fl
   const int T = tr->seq_len;
   switch (tr->L) {
     case 8: return launch<Grad8>(s, D, n_seq, T, kappa, tot, grad_soft, nullptr, soft, log_z, grad_s, ws, ws_bytes, strm);
-    default: return launch<Grad12>(s, D, n_seq, T, kappa, tot, grad_soft, nullptr, soft, log_z, grad_s, ws, ws_bytes, strm);
+    case 12: return launch<Grad12>(s, D, n_seq, T, kappa, tot, grad_soft, nullptr, soft, log_z, grad_s, ws, ws_bytes, strm);
+    default: return launch<Grad16>(s, D, n_seq, T, kappa, tot, grad_soft, nullptr, soft, log_z, grad_s, ws, ws_bytes, strm);
   }
 }
 
@@ -891,7 +896,6 @@ extern "C" tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *tr, const fl
                                                size_t ws_bytes, void *stream) {
   tcq_status_t st = check_trellis(tr);
   if (st != TCQ_OK) return st;
-  if (tr->L == 16) return TCQ_ERR_UNSUPPORTED;
   if (!temp_ok(temp)) return TCQ_ERR_INVALID_ARG;
   if (n_seq < 0 || n_seq > (int64_t)INT32_MAX) return TCQ_ERR_INVALID_ARG;
   if (n_seq == 0) return TCQ_OK;
@@ -905,6 +909,7 @@ extern "C" tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *tr, const fl
   const int T = tr->seq_len;
   switch (tr->L) {
     case 8: return launch<Grad8>(s, D, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
-    default: return launch<Grad12>(s, D, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
+    case 12: return launch<Grad12>(s, D, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
+    default: return launch<Grad16>(s, D, n_seq, T, kappa, tot, grad_soft, soft, nullptr, nullptr, grad_s, ws, ws_bytes, strm);
   }
 }

@@ -5,6 +5,8 @@ Units of work (per sequence of T = 256 weights on a 2^L-state trellis):
 
   decode (HBM):  64 B of 2-bit stream read + 512 B of fp16 written, i.e.
                  2.25 bytes per weight.  Peak: the measured HBM copy bandwidth.
+  pack + decode: 512 B of walk read, the free-start stream written and read
+                 back (17 words at L = 12), 512 B of fp16 written.
   viterbi (ALU): per state and step, the emission (code - s)^2 (sub, mul), the
                  accumulate (add), and a quarter of the shared 4-way min and
                  argmin of its predecessor group (3 min + 3 compare per group):
@@ -80,6 +82,9 @@ def load_measured_peaks(root: str) -> dict:
 def kernel_work(kernel: str, L: int, n_seq: int, T: int = SEQ_LEN) -> tuple[str, float, str]:
     """(bound, algorithmic work per launch, unit of work) for a benchmark kernel."""
     states = float(1 << L)
+    if kernel.startswith("pack_decode"):    # walks in, free-start stream out and back in, fp16 out
+        words = (T * 2 + L - 2 + 31) // 32
+        return "hbm", n_seq * (T * 2 + 2 * 4 * words + T * 2), "bytes"
     if kernel.startswith("decode_gemv"):    # 2-bit stream in; x and y are a rounding error
         return "hbm", n_seq * (T * 2 / 8), "bytes"
     if kernel.startswith("decode"):
