@@ -40,8 +40,17 @@ MUFU_PER_SM = 16               # special-function results per clock per SM
 # null.  (kernel prefix, workload): (bytes, sequences in the capture, sources)
 _CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 MEASURED_TRAFFIC = {
-    ("bcjr_soft_vjp", "l12_gauss1024"): (2.105408e9 + 2.181073664e9, 1024, {
-        "tcq_bcjr.cu": "6617a7096717c0495f8afc8a697e8984401ea6f4",
+    ("bcjr_soft_vjp", "l12_gauss1024"): (2.104392e9 + 2.179997e9, 1024, {
+        "tcq_bcjr.cu": "5857d9bcba2f10375d49c1fde35f8a3ff9e77512",
+        "tcq_device.cuh": "18b7f3a092c947f32accdefd8d22f8b99f58c38e"}),
+    # 32-sequence capture; every sequence writes and re-reads its own messages
+    ("bcjr_soft_vjp", "l16_rht1024_grad"): (988.288e6 + 1.079279e9, 32, {
+        "tcq_bcjr.cu": "5857d9bcba2f10375d49c1fde35f8a3ff9e77512",
+        "tcq_device.cuh": "18b7f3a092c947f32accdefd8d22f8b99f58c38e"}),
+    # cold-cache capture: about 56 MB of the fp16 output is still dirty in L2
+    # when the kernel ends, so DRAM writes read below the 134 MB written
+    ("decode_tile16", "l16_decode_8192sq"): (16.796416e6 + 78.145024e6, 262144, {
+        "tcq_decode.cu": "f973d336196f0d525904ea381884bc99ad8e4f71",
         "tcq_device.cuh": "18b7f3a092c947f32accdefd8d22f8b99f58c38e"}),
     # three launches (row pass, two column passes) of one 8192 x 8192 rotation
     ("rht", "rht_t5_8192sq"): (269.954048e6 + 226.045952e6 + 268.44288e6 + 206.207232e6
