@@ -1,0 +1,186 @@
+"""Out-of-bounds writes: every C-ABI entry point, called on ragged sizes, writes
+only inside its outputs and its workspace, and leaves its inputs unchanged.
+
+Each output and workspace is carved from a larger device buffer whose bytes
+before and after it (and the padding up to the next 256-byte boundary) hold a
+sentinel pattern; after the call the sentinel must be intact.  This stands in
+for a memory checker, which cannot be run on these GPUs.  Correctness of the
+values is covered by the parity tests.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import tcq_workloads as W
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 4096          # bytes of sentinel on each side (keeps 256-byte alignment)
+FILL = 0xA5
+
+
+@pytest.fixture(scope="module")
+def abi():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from trellis_coded_weight_bitshift_b200 import _abi
+    from trellis_coded_weight_bitshift_b200.build import build
+    build()
+    return _abi
+
+
+class Guarded:
+    """nbytes of device memory with sentinel bytes around it."""
+
+    def __init__(self, nbytes: int):
+        self.n = int(nbytes)
+        body = (self.n + 255) // 256 * 256
+        self.buf = torch.full((GUARD + body + GUARD,), FILL, dtype=torch.uint8, device="cuda")
+        self.ptr = ctypes.c_void_p(self.buf.data_ptr() + GUARD)
+
+    def intact(self) -> bool:
+        torch.cuda.synchronize()
+        return bool((self.buf[:GUARD] == FILL).all()) and bool((self.buf[GUARD + self.n:] == FILL).all())
+
+
+def _inp(a: np.ndarray):
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return t, t.clone(), ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _unchanged(*pairs):
+    torch.cuda.synchronize()
+    return all(torch.equal(a, b) for a, b in pairs)
+
+
+@pytest.mark.parametrize("L,n,T", [(8, 5, 37), (8, 9, 256), (12, 5, 37), (12, 3, 256), (16, 3, 37)])
+@pytest.mark.parametrize("weighted", [False, True])
+def test_viterbi_writes_stay_inside(abi, L, n, T, weighted):
+    lib = abi.lib()
+    tr = abi.trellis(L, T)
+    s, s0, sp = _inp(W.gaussian(n, 900 + T))
+    D, D0, Dp = _inp(W.curvature(n, 901, seq_len=T)) if weighted else (s, s0, None)
+    states, mse = Guarded(n * T * 2), Guarded(n * 4)
+    need = lib.tcq_viterbi_workspace_size(ctypes.byref(tr), n)
+    ws = Guarded(need)
+    rc = lib.tcq_viterbi_encode(ctypes.byref(tr), sp, Dp, n, states.ptr, mse.ptr, ws.ptr, need, _stream())
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert states.intact() and mse.intact() and ws.intact()
+    assert _unchanged((s, s0), (D, D0))
+
+
+@pytest.mark.parametrize("L,n,T", [(8, 5, 48), (12, 3, 48), (16, 2, 256)])
+def test_tailbiting_writes_stay_inside(abi, L, n, T):
+    lib = abi.lib()
+    tr = abi.trellis(L, T)
+    s, s0, sp = _inp(W.gaussian(n, 910 + T))
+    states, mse = Guarded(n * T * 2), Guarded(n * 4)
+    need = lib.tcq_viterbi_workspace_size(ctypes.byref(tr), n)
+    ws = Guarded(need)
+    rc = lib.tcq_viterbi_encode_tailbiting(ctypes.byref(tr), sp, None, n, states.ptr, mse.ptr, ws.ptr,
+                                           need, _stream())
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert states.intact() and mse.intact() and ws.intact()
+    assert _unchanged((s, s0))
+
+
+@pytest.mark.parametrize("L,n,T", [(8, 5, 37), (8, 11, 256), (12, 5, 37), (12, 2, 256), (16, 3, 37),
+                                   (16, 2, 256)])
+def test_bcjr_writes_stay_inside(abi, L, n, T):
+    lib = abi.lib()
+    tr = abi.trellis(L, T)
+    temp = ctypes.c_float(0.2)
+    s, s0, sp = _inp(W.gaussian(n, 920 + T))
+    v, v0, vp = _inp(W.gaussian(n, 921 + T))
+    st = _stream()
+    # soft codeword and log Z
+    soft, logz = Guarded(n * T * 4), Guarded(n * 4)
+    need = lib.tcq_bcjr_workspace_size(ctypes.byref(tr), n, 0)
+    ws = Guarded(need)
+    rc = lib.tcq_bcjr_soft(ctypes.byref(tr), sp, None, n, temp, soft.ptr, logz.ptr, ws.ptr, need, st)
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert soft.intact() and logz.intact() and ws.intact()
+    # separate backward, reading the soft codeword just written
+    grad = Guarded(n * T * 4)
+    needg = lib.tcq_bcjr_workspace_size(ctypes.byref(tr), n, 1)
+    wsg = Guarded(needg)
+    soft_t = soft.buf[GUARD:GUARD + n * T * 4].clone()
+    rc = lib.tcq_bcjr_soft_backward(ctypes.byref(tr), sp, None, n, temp, soft.ptr, vp, grad.ptr,
+                                    wsg.ptr, needg, st)
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert grad.intact() and wsg.intact()
+    assert _unchanged((soft.buf[GUARD:GUARD + n * T * 4], soft_t))
+    # one-sweep soft, log Z and gradient
+    soft2, logz2, grad2 = Guarded(n * T * 4), Guarded(n * 4), Guarded(n * T * 4)
+    wsg2 = Guarded(needg)
+    rc = lib.tcq_bcjr_soft_and_grad(ctypes.byref(tr), sp, None, n, temp, vp, soft2.ptr, logz2.ptr,
+                                    grad2.ptr, wsg2.ptr, needg, st)
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert soft2.intact() and logz2.intact() and grad2.intact() and wsg2.intact()
+    assert _unchanged((s, s0), (v, v0))
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+@pytest.mark.parametrize("T", [37, 256])
+def test_pack_and_decode_writes_stay_inside(abi, L, T):
+    lib = abi.lib()
+    tr = abi.trellis(L, T)
+    n = 7
+    rng = np.random.default_rng(930 + L + T)
+    st = np.empty((n, T), dtype=np.int64)
+    st[:, 0] = rng.integers(0, 1 << L, n)
+    for t in range(1, T):
+        st[:, t] = ((st[:, t - 1] << 2) | rng.integers(0, 4, n)) & ((1 << L) - 1)
+    states, states0, stp = _inp(st.astype(np.uint16).view(np.int16))
+    for layout in (abi.TAILBITING, abi.FREE_START):
+        if layout == abi.TAILBITING and (2 * T) % 32:
+            continue
+        words = lib.tcq_stream_words(ctypes.byref(tr), layout)
+        bits = Guarded(n * words * 4)
+        rc = lib.tcq_pack_states(ctypes.byref(tr), stp, n, layout, bits.ptr, _stream())
+        assert rc == abi.TCQ_OK, abi.status_string(rc)
+        assert bits.intact()
+        out = Guarded(n * T * 2)
+        rc = lib.tcq_decode(ctypes.byref(tr), bits.ptr, n, layout, abi.OUT_SEQ, 0, 0, out.ptr, _stream())
+        assert rc == abi.TCQ_OK, abi.status_string(rc)
+        assert out.intact()
+    assert _unchanged((states, states0))
+
+
+def test_decode_tiles_and_gemv_writes_stay_inside(abi):
+    lib = abi.lib()
+    tr = abi.trellis(16, 256)
+    rows, cols = 48, 96
+    n = (rows // 16) * (cols // 16)
+    words = np.random.default_rng(940).integers(0, 2 ** 32, (n, 16), dtype=np.uint32)
+    bits, bits0, bp = _inp(words.view(np.int32))
+    out = Guarded(rows * cols * 2)
+    rc = lib.tcq_decode(ctypes.byref(tr), bp, n, abi.TAILBITING, abi.OUT_TILE16, rows, cols, out.ptr,
+                        _stream())
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert out.intact()
+    x, x0, xp = _inp(W.gaussian(1, 941, seq_len=cols)[0])
+    y = Guarded(rows * 4)
+    rc = lib.tcq_decode_gemv(ctypes.byref(tr), bp, abi.TAILBITING, rows, cols, xp, y.ptr, _stream())
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert y.intact()
+    assert _unchanged((bits, bits0), (x, x0))
+
+
+@pytest.mark.parametrize("rows,cols", [(64, 128), (32, 8192), (1024, 32)])
+def test_rht_writes_stay_inside(abi, rows, cols):
+    lib = abi.lib()
+    rng = np.random.default_rng(950 + rows)
+    w, w0, wp = _inp(rng.standard_normal((rows, cols)).astype(np.float32))
+    s1, s10, s1p = _inp((rng.integers(0, 2, rows) * 2 - 1).astype(np.float32))
+    s2, s20, s2p = _inp((rng.integers(0, 2, cols) * 2 - 1).astype(np.float32))
+    out = Guarded(rows * cols * 4)
+    rc = lib.tcq_rht(wp, rows, cols, s1p, s2p, out.ptr, _stream())
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert out.intact()
+    assert _unchanged((w, w0), (s1, s10), (s2, s20))
