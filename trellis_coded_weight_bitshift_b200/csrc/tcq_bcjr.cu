@@ -85,6 +85,9 @@ struct BcjrCfg {
   static constexpr int TCPT = TMEMC ? HS * G * 2 : 0;              // TMEM columns per thread
   static constexpr int TCOLS = TCPT * (NT / 128) <= 32 ? 32 : TCPT * (NT / 128);  // per CTA
   static constexpr int NPART = TPS >= 32 ? TPS / 32 : 1;       // partial records per sequence
+  // several warp-aligned sequences in one CTA step independently, each on its
+  // own named barrier; they share one copy of the code values
+  static constexpr bool NAMED = SPC > 1 && TPS % 32 == 0;
   static constexpr int PREC = 8;                                 // floats per partial record
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
   static constexpr int NV = GRAD ? 2 : 1;                        // carried vectors (A | A, Phi)
@@ -112,7 +115,16 @@ struct BcjrCfg {
   static_assert(!TMEMC || (SPC == 1 && NT % 128 == 0 && (TCOLS & (TCOLS - 1)) == 0 && TCOLS <= 512 &&
                            G % 8 == 0), "tensor-memory code layout");
   static_assert(SPILL % 4 == 0, "spill in float4 chunks");
+  static_assert(!NAMED || (SPC <= 15 && !TMEMC), "named barriers 1..15, code values in shared memory");
 };
+
+// Barrier over the threads of one sequence: named barrier 1 + ls when the CTA
+// holds several warp-aligned sequences, else the CTA barrier.
+template <class C>
+__device__ __forceinline__ void seq_sync(int ls) {
+  if constexpr (C::NAMED) asm volatile("bar.sync %0, %1;" ::"r"(1 + ls), "n"(C::TPS) : "memory");
+  else __syncthreads();
+}
 
 // Code values are held as vertical pairs over the predecessor digit:
 // pair (h, i) = (code of state 2h NG + G w + i, code of state (2h+1) NG + G w + i).
@@ -341,27 +353,37 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   float *sums = reinterpret_cast<float *>(spill) + (size_t)T * NV * NG;
   auto prec = [&](int parity) { return part + ((parity * SPC + ls) * NPART) * PREC; };
 
+  if constexpr (C::NAMED) __syncthreads();                 // the shared code values are in place
+  // targets (and curvature, cotangent, centre) of step t of sequence row l
+  auto load_row = [&](int l, int t, int64_t base) {
+    const int64_t sq = base + l;
+    const bool ok = sq < n_seq;
+    ssm[l * 256 + t] = ok ? s[sq * T + t] : 0.0f;
+    ksm[l * 256 + t] = kappa * ((ok && Dw) ? Dw[sq * T + t] : 1.0f);
+    if (GRAD) {
+      vsm[l * 256 + t] = ok ? vgrad[sq * T + t] : 0.0f;
+      // centre of the covariance: the forward soft codeword when given,
+      // else the targets themselves (any per-step constant is exact)
+      fsm[l * 256 + t] = ok ? (soft_in ? soft_in[sq * T + t] : s[sq * T + t]) : 0.0f;
+    }
+  };
   for (int64_t base = (int64_t)blockIdx.x * SPC; base < n_seq; base += (int64_t)gridDim.x * SPC) {
     const int64_t seq = base + ls;
     const bool active = seq < n_seq;
-    __syncthreads();                                       // previous sequence fully done
-    for (int x = tid; x < SPC * T; x += C::NT) {
-      const int l = x / T, t = x - l * T;
-      const int64_t sq = base + l;
-      const bool ok = sq < n_seq;
-      ssm[l * 256 + t] = ok ? s[sq * T + t] : 0.0f;
-      ksm[l * 256 + t] = kappa * ((ok && Dw) ? Dw[sq * T + t] : 1.0f);
-      if (GRAD) {
-        vsm[l * 256 + t] = ok ? vgrad[sq * T + t] : 0.0f;
-        // centre of the covariance: the forward soft codeword when given,
-        // else the targets themselves (any per-step constant is exact)
-        fsm[l * 256 + t] = ok ? (soft_in ? soft_in[sq * T + t] : s[sq * T + t]) : 0.0f;
-      }
+    seq_sync<C>(ls);                                       // previous sequence fully done
+    if constexpr (C::NAMED) {
+      for (int t = w; t < T; t += TPS) load_row(ls, t, base);
+    } else {
+      for (int x = tid; x < SPC * T; x += C::NT) load_row(x / T, x % T, base);
     }
     float *V = Vall + ls * NB * NV * NG;
     for (int x = w; x < NV * NG; x += TPS) V[x] = 0.0f;     // A_0 = 0 (and Phi_0 = 0)
-    for (int x = tid; x < 2 * SPC * NPART * PREC; x += C::NT) part[x] = 0.0f;
-    __syncthreads();
+    if constexpr (C::NAMED) {
+      for (int x = w; x < NPART * PREC; x += TPS) { prec(0)[x] = 0.0f; prec(1)[x] = 0.0f; }
+    } else {
+      for (int x = tid; x < 2 * SPC * NPART * PREC; x += C::NT) part[x] = 0.0f;
+    }
+    seq_sync<C>(ls);
 
     // ---------------- forward ----------------
     // A_t is stored relative to CA_t = c_0 + ... + c_{t-1}, c_t = max of stored A_t.
@@ -397,7 +419,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       }
       if (w == 0) cah[ls * 256 + t - 1] = CA;
       if (t == T) break;
-      if (NB == 1) __syncthreads();
+      if (NB == 1) seq_sync<C>(ls);
       CA += cmax;
       float *Ao = V + (t % NB) * NV * NG;
       const float sv = ssm[ls * 256 + t - 1];
@@ -467,7 +489,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       }
       tmax = seq_max<TPS>(tmax);
       if (plead) prec(t & 1)[pidx * PREC] = tmax;
-      __syncthreads();
+      seq_sync<C>(ls);
     }
     // CA = CA_{T-1}; cmax = max of stored A_{T-1}; spill step T-1 holds A_{T-1}.
 
@@ -506,7 +528,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       vmax = lane_reduce<TPS>(vmax, MaxOp());
       float *pp = prec(0);
       if (plead) pp[pidx * PREC + 5] = vmax;
-      __syncthreads();
+      seq_sync<C>(ls);
       vmax = pp[5];
 #pragma unroll
       for (int x = 1; x < NPART; ++x) vmax = fmaxf(vmax, pp[x * PREC + 5]);
@@ -517,7 +539,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         for (int k = 0; k < GQ; ++k) sum += ex2(vals[a][k] - vmax);
       sum = lane_reduce<TPS>(sum, SumOp());
       if (plead) pp[pidx * PREC + 6] = sum;
-      __syncthreads();
+      seq_sync<C>(ls);
       float tot = 0.0f;
 #pragma unroll
       for (int x = 0; x < NPART; ++x) tot += pp[x * PREC + 6];
@@ -531,7 +553,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     // the posteriors themselves (sum ~ 1).
     float *Bv = V;
     for (int x = w; x < NV * NG; x += TPS) Bv[((T - 1) % NB) * NV * NG + x] = 0.0f;
-    __syncthreads();
+    seq_sync<C>(ls);
     float DB = 0.0f;
     for (int t = T - 2; t >= -1; --t) {
       const int tc = t + 1;                                  // combine step
@@ -583,7 +605,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
                                          (n2 * inv - (num * inv) * (n1 * inv));
         }
       }
-      if (NB == 1) __syncthreads();
+      if (NB == 1) seq_sync<C>(ls);
       const float K = log2Z - cah[ls * 256 + tc] - DB;
       DB += dprev;
       const float sv = ssm[ls * 256 + tc];
@@ -714,7 +736,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         }
         if (plead) pp[0] = tmax;
       }
-      __syncthreads();
+      seq_sync<C>(ls);
     }
     if (C::DEFER && active) {
       // every step's sums are in the workspace (the barrier that closed the
@@ -759,10 +781,14 @@ using namespace tcq_host;
 namespace {
 
 using Soft8 = BcjrCfg<8, 4, 8, 4, 2, false>;
-// L = 12: 128 threads / sequence, 7 per SM (one wave of 1,036); the soft pass
-// reads every code value from shared memory, the gradient pass keeps digits
-// 0 and 1 in registers (the register file allows 72 per thread)
-using Soft12 = BcjrCfg<12, 8, 1, 0, 2, false, 7>;
+// L = 12: 128 threads / sequence, seven sequences in one 896-thread CTA per SM
+// (one wave of 1,036), each stepping on its own named barrier.  Every code
+// value is read from one shared-memory copy that the seven share.  Measured
+// against seven one-sequence CTAs, each with its own copy (the gradient pass
+// then kept digits 0-1 in registers and spilled at 72 registers, and the
+// spills missed L1, which the seven copies had taken): soft 0.977 -> 0.883 ms,
+// soft + gradient 1.517 -> 1.295 ms on 1,024 sequences.
+using Soft12 = BcjrCfg<12, 8, 7, 0, 2, false, 1>;
 // L = 16: one 512-thread CTA per SM; all 2^16 code values sit in tensor memory
 // (128 columns per thread, the whole 512-column allocation), which leaves the
 // shared memory for a double-buffered state vector (one barrier per step).
@@ -772,7 +798,7 @@ using Soft12 = BcjrCfg<12, 8, 1, 0, 2, false, 7>;
 // used here only.
 using Soft16 = BcjrCfg<16, 32, 1, 0, 2, false, 1, true>;
 using Grad8 = BcjrCfg<8, 4, 8, 4, 2, true>;
-using Grad12 = BcjrCfg<12, 8, 1, 2, 2, true, 7>;
+using Grad12 = BcjrCfg<12, 8, 7, 0, 2, true, 1>;
 // L = 16 gradient: code values in tensor memory as in the soft pass; the two
 // carried vectors (A and Phi, 2 x 64 KiB) fit the shared memory only
 // single-buffered, so each step takes two barriers.
