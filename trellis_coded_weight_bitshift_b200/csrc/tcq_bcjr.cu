@@ -100,15 +100,18 @@ struct BcjrCfg {
            + (size_t)2 * SPC * NPART * PREC;                        // partial records
   }
   static constexpr size_t smem_bytes() { return smem_floats() * sizeof(float); }
-  // The soft pass finishes its steps after the backward (the per-step sums go
-  // to the workspace); the gradient pass, short of registers, finishes each
-  // step one step later from the shared partial records.
-  static constexpr bool DEFER = !GRAD;
+  // Steps are finished after the backward: the per-step sums go to the
+  // workspace and the sequence's threads turn them into outputs in parallel
+  // (finishing each step on one thread during the sweep stalls the other warps
+  // of the sequence at the next barrier).
+  static constexpr bool DEFER = true;
+  static constexpr int NQS = GRAD ? 4 : 2;                        // sums per record
   // per resident sequence: the spilled messages, then (DEFER) the per-step
-  // partial sums (numerator, denominator) of each warp; a whole number of
-  // 256-byte units, so that every slot (read as float4) stays 16-byte aligned
+  // partial sums (numerator, denominator; gradient: and the two moments) of
+  // each warp; a whole number of 256-byte units, so that every slot (read as
+  // float4) stays 16-byte aligned
   __host__ __device__ static constexpr size_t ws_floats_per_slot(int T) {
-    return ((size_t)T * NV * NG + (DEFER ? (size_t)T * NPART * 2 : 0) + 63) / 64 * 64;
+    return ((size_t)T * NV * NG + (DEFER ? (size_t)T * NPART * NQS : 0) + 63) / 64 * 64;
   }
   static_assert(NG % G == 0 && G % 4 == 0, "bad split");
   static_assert(AREG % 2 == 0, "code values are held in digit pairs");
@@ -348,8 +351,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   // at this thread's groups r = a*NG/4 + GQ*w + k, flattened as a*GQ + k.
   float4 *spill = reinterpret_cast<float4 *>(ws + (size_t)(blockIdx.x * SPC + ls) *
                                                       C::ws_floats_per_slot(T));
-  // DEFER: [T][NPART] records of (numerator, denominator), read back once the
-  // backward is done
+  // DEFER: [T][NPART] records of NQS sums (numerator, denominator; gradient:
+  // the two moments), read back once the backward is done
   float *sums = reinterpret_cast<float *>(spill) + (size_t)T * NV * NG;
   auto prec = [&](int parity) { return part + ((parity * SPC + ls) * NPART) * PREC; };
 
@@ -731,7 +734,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         const int o = lane & (WL - 1);
         float *pp = prec(tc & 1) + pidx * PREC;
         if ((o & (WL / NQ - 1)) == 0) {                                  // num, den (n1, n2)
-          if constexpr (C::DEFER) sums[((size_t)tc * NPART + pidx) * 2 + o / (WL / NQ)] = mine;
+          if constexpr (C::DEFER) sums[((size_t)tc * NPART + pidx) * C::NQS + o / (WL / NQ)] = mine;
           else pp[1 + o / (WL / NQ)] = mine;
         }
         if (plead) pp[0] = tmax;
@@ -742,13 +745,19 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       // every step's sums are in the workspace (the barrier that closed the
       // last step orders them): the sequence's threads finish them in parallel
       for (int u = w; u < T; u += TPS) {
-        float num = 0.0f, den = 0.0f;
+        float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f;
 #pragma unroll
         for (int x = 0; x < NPART; ++x) {
-          num += sums[((size_t)u * NPART + x) * 2];
-          den += sums[((size_t)u * NPART + x) * 2 + 1];
+          const float *r = sums + ((size_t)u * NPART + x) * C::NQS;
+          num += r[0]; den += r[1];
+          if (GRAD) { n1 += r[GRAD ? 2 : 0]; n2 += r[GRAD ? 3 : 0]; }
         }
         if (soft_out) soft_out[seq * T + u] = num / den;
+        if (GRAD) {   // 2 D_u / temp = 2 ln2 kappa D_u
+          const float inv = 1.0f / den;
+          grad_out[seq * T + u] = (1.3862943611198906f * ksm[ls * 256 + u]) *
+                                  (n2 * inv - (num * inv) * (n1 * inv));
+        }
       }
     }
     if (!C::DEFER && w == 0 && active) {                     // finish step 0
