@@ -205,6 +205,26 @@ def test_bcjr_l12_workload(tcq):
     assert np.all(np.isfinite(soft))
 
 
+def test_bcjr_l12_several_waves(tcq):
+    # more sequences than one wave of the L = 12 CTAs (148 x 7 slots): each CTA
+    # loops, and the last round has only a few active sequences
+    n = 2100
+    s = W.gaussian(n, 1212)
+    v = W.gaussian(n, 1213)
+    sd, vd = _dev(s), _dev(v)
+    soft, lz = tcq.bcjr_soft(sd, 12, 0.1)
+    soft2, lz2, g = tcq.bcjr_soft_and_grad(sd, 12, 0.1, vd)
+    torch.cuda.synchronize()
+    soft, soft2, g = soft.cpu().numpy(), soft2.cpu().numpy(), g.cpu().numpy()
+    assert np.all(np.isfinite(soft)) and np.all(np.isfinite(g))
+    assert np.abs(soft - soft2).max() <= SOFT_ATOL
+    idx = np.array([0, 1035, 1036, 2071, 2072, 2099])
+    rg, rsoft = oracle.bcjr_vjp(s[idx], v[idx], 12, 0.1)
+    assert np.abs(soft[idx] - rsoft).max() <= SOFT_ATOL
+    for i, j in enumerate(idx):
+        assert np.abs(g[j] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+
+
 @pytest.mark.parametrize("temp", [1.0, 0.1, 0.01])
 def test_bcjr_l16_student_t(tcq, temp):
     s = W.sequences("l16_studentt_2048x8192")
