@@ -472,9 +472,10 @@ def _signs(n, seed):
 
 
 # every row-pass width (2^11..2^13 in registers, narrower through shared memory)
-# and every column-pass split (one pass of <= 10 bits; 6+6, 6+7, 7+7 bits)
+# and every column-pass split (one pass of <= 10 bits; 5+6, 6+6, 6+7, 7+7 bits)
 @pytest.mark.parametrize("R,C", [(1024, 1024), (32, 8192), (8192, 32), (256, 64), (64, 2048),
-                                 (32, 4096), (4096, 64), (16384, 32)])
+                                 (32, 4096), (4096, 64), (16384, 32), (2048, 128),
+                                 (8192, 1024)])
 def test_rht_matches_dense_definition(tcq, R, C):
     W = W_ = np.random.default_rng(R * 3 + C).standard_normal((R, C)).astype(np.float32)
     s1, s2 = _signs(R, R), _signs(C, C + 1)
