@@ -184,3 +184,37 @@ def test_rht_writes_stay_inside(abi, rows, cols):
     assert rc == abi.TCQ_OK, abi.status_string(rc)
     assert out.intact()
     assert _unchanged((w, w0), (s1, s10), (s2, s20))
+
+
+def test_concurrent_streams_match_sequential(abi):
+    # calls are re-entrant: the same calls on three streams at once (each with
+    # its own workspace) give the same bits as one after another; the L = 16
+    # kernels on two streams also exercise tensor-memory allocation on
+    # shared SMs
+    import trellis_coded_weight_bitshift_b200 as tcq
+    s16 = torch.from_numpy(W.gaussian(300, 961)).cuda()
+    s12 = torch.from_numpy(W.gaussian(1100, 962)).cuda()
+    v12 = torch.from_numpy(W.gaussian(1100, 963)).cuda()
+
+    def run():
+        return (tcq.viterbi_encode(s16, 16), tcq.bcjr_soft(s16, 16, 0.3),
+                tcq.bcjr_soft_and_grad(s12, 12, 0.1, v12))
+
+    ref = run()
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    cur = torch.cuda.current_stream()
+    for st in streams:
+        st.wait_stream(cur)
+    with torch.cuda.stream(streams[0]):
+        vit = tcq.viterbi_encode(s16, 16)
+    with torch.cuda.stream(streams[1]):
+        soft = tcq.bcjr_soft(s16, 16, 0.3)
+    with torch.cuda.stream(streams[2]):
+        sg = tcq.bcjr_soft_and_grad(s12, 12, 0.1, v12)
+    torch.cuda.synchronize()
+    got = (vit, soft, sg)
+    for a, b in zip(got, ref):
+        for x, y in zip(a, b):
+            assert torch.equal(x.view(torch.int16) if x.dtype == torch.uint16 else x,
+                               y.view(torch.int16) if y.dtype == torch.uint16 else y)
