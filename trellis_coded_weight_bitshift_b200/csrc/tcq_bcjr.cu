@@ -621,9 +621,10 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       f2_t num2 = f2(0.0f, 0.0f), den2 = num2, n12 = num2, n22 = num2;
       // KB values of this thread's spilled vector at flat index f (KB | f)
       // sub-run width: 4 when the code values come from tensor memory (the
-      // registers they free hold the wider block) in the soft pass, else 2
-      // (the gradient pass carries B and Psi, twice the values)
-      constexpr int KB = GQ < 2 ? GQ : (C::TMEMC && GQ >= 4 && !GRAD ? 4 : 2);
+      // registers they free hold the wider block) in the soft pass; 1 in the
+      // L = 16 gradient pass, which holds B and Psi of 32 groups (spills
+      // 124/148 -> 36/60 bytes, sweep -3.7%); else 2
+      constexpr int KB = GQ < 2 ? GQ : (C::TMEMC && GQ >= 4 ? (GRAD ? 1 : 4) : 2);
       auto spilled_run = [&](int f, float *dst) {
         float4 v;
         if constexpr (PREFETCH) v = avq[PREFETCH ? (f >> 2) : 0];
