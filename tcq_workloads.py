@@ -40,12 +40,13 @@ class Workload:
     cols: int = 0
     ops: tuple = field(default=())
     curv_seed: int = 0             # > 0: curvature-weighted search, D drawn from this seed
+    concurrent: bool = False       # independent calls may run on separate streams at once
 
 
 # The five workloads, seeds 1..5.
 WORKLOADS = {
     "l8_gauss64": Workload("l8_gauss64", 8, 64, "gaussian", 1, (1.0, 0.1),
-                           ops=("viterbi", "bcjr")),
+                           ops=("viterbi", "bcjr"), concurrent=True),
     "l12_gauss1024": Workload("l12_gauss1024", 12, 1024, "gaussian", 2, (0.05,),
                               ops=("viterbi", "pack_decode", "bcjr", "bcjr_grad")),
     "l16_rht1024": Workload("l16_rht1024", 16, 4096, "rht_block", 3, (), 1024, 1024,
