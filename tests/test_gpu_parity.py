@@ -250,6 +250,51 @@ def test_bcjr_edge_shapes(tcq, L, T, n):
     assert np.all(np.abs(lz - rlz) <= 1e-5 * np.abs(rlz) + 1e-4)
 
 
+def _extreme_targets(T=40):
+    # zeros (many exact cost ties), beyond the largest code value, far outside
+    # the code range, alternating +-50, and tiny values
+    rows = [np.zeros(T), np.full(T, 3.4506), np.full(T, -10.0), np.full(T, 100.0),
+            np.where(np.arange(T) % 2 == 0, 50.0, -50.0),
+            np.random.default_rng(77).standard_normal(T) * 1e-3]
+    return np.stack(rows).astype(np.float32)
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+def test_viterbi_extreme_targets(tcq, L):
+    s = _extreme_targets()
+    st, mse = _viterbi_gpu(tcq, s, L)
+    rst, rmse = oracle.viterbi_f32(s, L)
+    assert np.array_equal(st, rst)
+    assert np.array_equal(mse.view(np.uint32), rmse.view(np.uint32))
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+@pytest.mark.parametrize("temp", [0.1, 1.0, 1e4])
+def test_bcjr_extreme_targets_and_temperatures(tcq, L, temp):
+    s = _extreme_targets()
+    soft, lz = _bcjr_gpu(tcq, s, L, temp)
+    rsoft, rlz = oracle.bcjr_soft(s, L, temp)
+    assert np.all(np.isfinite(soft)) and np.all(np.isfinite(lz))
+    assert np.abs(soft - rsoft).max() <= SOFT_ATOL, np.abs(soft - rsoft).max(axis=1)
+    assert np.all(np.abs(lz - rlz) <= 1e-5 * np.abs(rlz) + 1e-3)
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+def test_bcjr_extreme_targets_low_temperature(tcq, L):
+    # log2 Z and the removed per-step maxima are summed in fp64, so targets far
+    # outside the code range stay finite and log Z stays accurate at any
+    # temperature.  The emission kappa (c - s)^2 is formed in fp32: with
+    # constant targets many walks tie exactly, and their relative weights carry
+    # its rounding (about kappa (c - s)^2 2^-24 per step, ~0.01 in log2 at
+    # temp 1e-3 and s = -10), so there the soft codeword is only within ~1e-2
+    s = _extreme_targets()
+    soft, lz = _bcjr_gpu(tcq, s, L, 1e-3)
+    rsoft, rlz = oracle.bcjr_soft(s, L, 1e-3)
+    assert np.all(np.isfinite(soft)) and np.all(np.isfinite(lz))
+    assert np.all(np.abs(lz - rlz) <= 1e-5 * np.abs(rlz) + 1e-3)
+    assert np.abs(soft - rsoft).max() <= 2e-2
+
+
 def test_bcjr_low_temperature_matches_viterbi_codeword(tcq):
     # temp -> 0 recovers the hard code: on sequences whose closest Viterbi
     # decision is at least 1e-3 relative apart, temp 1e-4 leaves the runner-up

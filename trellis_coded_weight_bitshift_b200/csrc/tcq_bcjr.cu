@@ -96,7 +96,7 @@ struct BcjrCfg {
     return (size_t)SPC * NBUF * NV * NG                            // state vectors
            + (TMEMC ? 0 : (size_t)ASM * G * TPS)                    // smem code values
            + (size_t)SPC * 256 * (GRAD ? 4 : 2)                     // s, kappa*D (+ v, soft)
-           + (size_t)SPC * 256                                       // CA_t prefix sums
+           + (size_t)SPC * 256                                       // CA_t increments
            + (size_t)2 * SPC * NPART * PREC;                        // partial records
   }
   static constexpr size_t smem_bytes() { return smem_floats() * sizeof(float); }
@@ -300,7 +300,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   float *ksm = ssm + SPC * 256;                            // [SPC][256] kappa * D_t
   float *vsm = ksm + SPC * 256;                            // GRAD: v, soft rows
   float *fsm = vsm + (GRAD ? SPC * 256 : 0);
-  float *cah = fsm + (GRAD ? SPC * 256 : 0);               // [SPC][256] CA_t
+  float *cah = fsm + (GRAD ? SPC * 256 : 0);               // [SPC][256] CA_t - CA_{t-1}
   float *part = cah + SPC * 256;                           // [2][SPC][NPART][PREC]
 
   const int tid = threadIdx.x;
@@ -390,7 +390,11 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
 
     // ---------------- forward ----------------
     // A_t is stored relative to CA_t = c_0 + ... + c_{t-1}, c_t = max of stored A_t.
+    // CA itself is needed only for log Z; the combine takes the increments
+    // c_{t-1} = CA_t - CA_{t-1} (cah[t]), because CA can be huge (it grows by
+    // up to kappa max(e) per step) while what the combine needs is small.
     float CA = 0.0f, cmax = 0.0f;
+    if (w == 0) cah[ls * 256] = 0.0f;
     for (int t = 1; t <= T; ++t) {
       const float *Ai = V + ((t - 1) % NB) * NV * NG;
       float ain[4][GQ], fin[GRAD ? 4 : 1][GQ];
@@ -420,8 +424,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           spill[((size_t)(t - 1) * NCH + c) * TPS + w] =
               make_float4(flat[4 * c], flat[4 * c + 1], flat[4 * c + 2], flat[4 * c + 3]);
       }
-      if (w == 0) cah[ls * 256 + t - 1] = CA;
       if (t == T) break;
+      if (w == 0) cah[ls * 256 + t] = cmax;
       if (NB == 1) seq_sync<C>(ls);
       CA += cmax;
       float *Ao = V + (t % NB) * NV * NG;
@@ -497,7 +501,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     // CA = CA_{T-1}; cmax = max of stored A_{T-1}; spill step T-1 holds A_{T-1}.
 
     // ---------------- log2 Z = LSE over all states at T-1 ----------------
-    float log2Z;
+    float log2Z, log2Zrel;
     {
       const float sT = ssm[ls * 256 + T - 1];
       float vals[4][GQ], vmax = -INFINITY;
@@ -546,18 +550,21 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       float tot = 0.0f;
 #pragma unroll
       for (int x = 0; x < NPART; ++x) tot += pp[x * PREC + 6];
-      log2Z = vmax + lg2(tot) + cmax + CA;
+      log2Zrel = vmax + lg2(tot) + cmax;                  // log2 Z - CA_{T-1}
+      log2Z = log2Zrel + CA;
     }
     if (w == 0 && active && logz_out) logz_out[seq] = log2Z * 0.69314718055994531f;
 
     // ---------------- backward + combine ----------------
     // B_t is stored relative to DB_t (sum of the maxima removed); the combine
     // at step tc uses K = log2Z - CA_tc - DB_tc so that the group weights are
-    // the posteriors themselves (sum ~ 1).
+    // the posteriors themselves (sum ~ 1).  K is carried as a running value,
+    // K_{tc-1} = K_tc + (CA_tc - CA_{tc-1}) - (DB_{tc-1} - DB_tc), starting
+    // from log2 Z - CA_{T-1}, so no two huge sums are ever subtracted.
     float *Bv = V;
     for (int x = w; x < NV * NG; x += TPS) Bv[((T - 1) % NB) * NV * NG + x] = 0.0f;
     seq_sync<C>(ls);
-    float DB = 0.0f;
+    float Krun = log2Zrel;
     for (int t = T - 2; t >= -1; --t) {
       const int tc = t + 1;                                  // combine step
       // this thread's spilled A_tc values (issued first: they come from HBM)
@@ -609,8 +616,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         }
       }
       if (NB == 1) seq_sync<C>(ls);
-      const float K = log2Z - cah[ls * 256 + tc] - DB;
-      DB += dprev;
+      const float K = Krun;
+      Krun += cah[ls * 256 + tc] - dprev;
       const float sv = ssm[ls * 256 + tc];
       const float vv = GRAD ? vsm[ls * 256 + tc] : 0.0f;
       const float fv = GRAD ? fsm[ls * 256 + tc] : 0.0f;
