@@ -417,6 +417,30 @@ def test_weighted_full_workload(tcq):
     gn = g.cpu().numpy()[idx]
     for i in range(10):
         assert np.abs(gn[i] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+    # the one-sweep form the benchmark times
+    soft2, lz2, g2 = tcq.bcjr_soft_and_grad(sd, 12, 0.05, torch.ones_like(sd), D=Dd)
+    torch.cuda.synchronize()
+    assert np.abs(soft2.cpu().numpy()[idx] - rsoft).max() <= SOFT_ATOL
+    assert np.abs(lz2.cpu().numpy() - lz.cpu().numpy()).max() <= 1e-3
+    g2n = g2.cpu().numpy()[idx]
+    for i in range(10):
+        assert np.abs(g2n[i] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+
+
+@pytest.mark.parametrize("L", [8, 12, 16])
+def test_weighted_gradient_random_cotangent(tcq, L):
+    s = W.gaussian(3, 1800 + L, seq_len=48)
+    D = W.curvature(3, 1900 + L, seq_len=48)
+    v = W.gaussian(3, 2000 + L, seq_len=48)
+    sd, Dd, vd = _dev(s), _dev(D), _dev(v)
+    soft, _ = tcq.bcjr_soft(sd, L, 0.2, D=Dd)
+    g1 = tcq.bcjr_soft_backward(sd, L, 0.2, soft, vd, D=Dd)
+    _, _, g2 = tcq.bcjr_soft_and_grad(sd, L, 0.2, vd, D=Dd)
+    torch.cuda.synchronize()
+    rg, _ = oracle.bcjr_vjp(s, v, L, 0.2, D=D)
+    for g in (g1.cpu().numpy(), g2.cpu().numpy()):
+        for i in range(3):
+            assert np.abs(g[i] - rg[i]).max() <= GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
 
 
 @pytest.mark.parametrize("L", [8, 16])
