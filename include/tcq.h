@@ -20,8 +20,8 @@
  *
  * Common conventions
  *   - The trellis is (L, k, V) with V = 1: 2^L states, each step appends k
- *     bits; state j may follow state i iff the top L-k bits of j equal the
- *     bottom L-k bits of i [QTIP, trellis].  Supported: k = 2, V = 1,
+ *     bits; the transitions out of state i go to j = ((i << k) | d) mod 2^L
+ *     for the 2^k digits d [QTIP, trellis].  Supported: k = 2, V = 1,
  *     L in {8, 12, 16}, 1 <= seq_len <= 256.  Anything else returns
  *     TCQ_ERR_UNSUPPORTED.
  *   - The codebook is 1MAD [QTIP, codebook]: code(j) = (bytesum(34038481 j +
@@ -100,7 +100,8 @@ TCQ_API const char *tcq_status_string(tcq_status_t status);
 TCQ_API size_t tcq_stream_words(const tcq_trellis_t *trellis, int layout);
 
 /* ------------------------------------------------------------------------
- * Viterbi encode [QTIP, trellis: the min-MSE walk is a shortest path].
+ * Viterbi encode [QTIP, trellis: Viterbi finds the walk of least squared
+ * error].
  *   cost_0(j) = (code_j - s_0)^2,
  *   cost_t(j) = min_a cost_{t-1}((j >> k) | (a << (L-k))) + (code_j - s_t)^2,
  * free start, free end.  fp32 arithmetic with each operation rounded on its
@@ -109,8 +110,8 @@ TCQ_API size_t tcq_stream_words(const tcq_trellis_t *trellis, int layout);
  *
  *   s          [n_seq][seq_len] fp32 targets (input).
  *   D          [n_seq][seq_len] fp32 per-weight curvature, or NULL for all
- *              ones [XOR-Trellis explainer, "Cliff edges": the search
- *              multiplies each step's squared error by that weight's D].  The
+ *              ones [XOR-Trellis explainer, "Cliff edges": the squared
+ *              error of step t is scaled by the curvature D_t].  The
  *              step cost becomes e = d*d, then e*D_t, each rounded on its own.
  *              D must be >= 0 and finite (other values: unspecified walks).
  *   states     [n_seq][seq_len] uint16: the chosen walk, state (L-bit window)
@@ -128,10 +129,10 @@ TCQ_API tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *trellis, const floa
 
 /* ------------------------------------------------------------------------
  * Tail-biting Viterbi encode [QTIP, "Tail-biting is worth its complexity":
- * the last state's low L-k bits equal the first state's high L-k bits, so a
- * sequence costs exactly k*T bits; the two-run search rotates the sequence by
- * T/2, runs Viterbi, reads the shared bits at the seam and re-runs with both
- * ends pinned to them].
+ * the walk closes on itself (the leading L-k bits of the first state are the
+ * trailing L-k bits of the last one), so the stream holds exactly k*T bits;
+ * the two-run search rotates the sequence by T/2, runs Viterbi, reads the
+ * shared bits at the seam and re-runs with both ends pinned to them].
  *   Same arguments, arithmetic and tie-breaks as tcq_viterbi_encode; the
  *   output walk is tail-biting (pack it with TCQ_TAILBITING) and mse is its
  *   cost / seq_len.  Needs k*seq_len >= L.  Workspace: as tcq_viterbi_encode.
@@ -228,8 +229,8 @@ TCQ_API tcq_status_t tcq_bcjr_soft_and_grad(const tcq_trellis_t *trellis, const 
                                             void *stream);
 
 /* ------------------------------------------------------------------------
- * Pack walks into bitstreams [QTIP, trellis: the state is a sliding L-bit
- * window over the stream].  Stream bits [k t, k t + k) are the top k bits of
+ * Pack walks into bitstreams [QTIP, trellis: state t is the L stream bits
+ * that start at bit k t].  Stream bits [k t, k t + k) are the top k bits of
  * state t; a free-start stream ends with the low L-k bits of the last state.
  * For a valid walk (and, for TCQ_TAILBITING, a circular one) decode of the
  * result returns code(states).
@@ -266,9 +267,10 @@ TCQ_API tcq_status_t tcq_decode_gemv(const tcq_trellis_t *trellis, const uint32_
                                      void *stream);
 
 /* ------------------------------------------------------------------------
- * Random-sign Hadamard rotation [QTIP, trellis section: random signs, then a
- * Hadamard matrix, on both sides of W, so that one data-independent code fits
- * every layer]:
+ * Random-sign Hadamard rotation [QTIP, trellis section: QuIP#'s transform,
+ * +-1 signs and a Hadamard transform applied from the left and the right,
+ * leaves the weights close to i.i.d. Gaussian, so one fixed code serves all
+ * layers]:
  *   out = (H_R / sqrt R) diag(sign_rows) W diag(sign_cols) (H_C / sqrt C)
  * with H_n the Sylvester Hadamard matrix (H_n[i][j] = (-1)^popcount(i & j)).
  *   W [rows][cols] fp32 (input), out [rows][cols] fp32 (output; may equal W),

@@ -401,7 +401,8 @@ def pack(states: np.ndarray, L: int, layout: int, k: int = 2) -> np.ndarray:
 
 # --------------------------------------------------------------------------
 # Random-sign Hadamard rotation (QTIP blog, "The trellis: a stateful codebook":
-# random signs, then a Hadamard matrix, on both sides of W -- from QuIP#).
+# QuIP#'s transform, +-1 signs and a Hadamard transform from the left and the
+# right).
 # --------------------------------------------------------------------------
 def hadamard(n: int) -> np.ndarray:
     """Sylvester Hadamard matrix H_n (n a power of two): H_1 = [1],

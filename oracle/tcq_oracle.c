@@ -23,9 +23,9 @@
  *   succ_b(i) = ((i << k) | b) & (2^L - 1), b in [0, 2^k)
  *   Free start: every state may begin a walk with cost (code - s_0)^2.
  *   D      optional per-weight curvature (NULL = all ones).  [XOR-Trellis
- *          explainer, "Cliff edges": the search multiplies each step's squared
- *          error by that weight's D; states and decoder are unchanged.]  The
- *          step cost becomes D_t (code - s_t)^2.
+ *          explainer, "Cliff edges": the squared error of step t is scaled by
+ *          D_t; the trellis and the code stay as they are.]  The step cost
+ *          becomes D_t (code - s_t)^2.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off (no fast-math), so
  * every float/double operation below is one IEEE-754 operation, correctly
@@ -38,8 +38,8 @@
 
 /* ------------------------------------------------------------------------ */
 /* 1MAD computed codebook   [QTIP-blog, "The codebook is computed"]          */
-/* A 32-bit LCG step, the sum of the four bytes of the result (Irwin-Hall,  */
-/* n = 4), then centre by 510 and scale by 147.8.                           */
+/* One 32-bit LCG step on the state, its byte sum (an Irwin-Hall variable   */
+/* with n = 4), then centring by 510 and scaling by 1/147.8.                */
 /* ------------------------------------------------------------------------ */
 int orc_1mad_bytesum(uint32_t x)
 {
@@ -410,11 +410,11 @@ int64_t orc_bruteforce_f64(int L, int k, int T, double temp, const double *s, co
 
 /* ------------------------------------------------------------------------ */
 /* Tail-biting search   [QTIP-blog, "Tail-biting is worth its complexity"]  */
-/* A tail-biting walk also wraps: the last state's low L-k bits equal the   */
-/* first state's high L-k bits, so the stream is exactly k*T bits.  With    */
-/* that shared value o fixed, the search is a Viterbi run whose first state */
-/* must have top bits o and whose last state must have low bits o; the      */
-/* exact optimum is the best of the 2^(L-k) runs, one per o.                */
+/* A tail-biting walk also wraps: the trailing L-k bits of the last state  */
+/* are the leading L-k bits of the first, so the stream is exactly k*T      */
+/* bits.  With that shared value o fixed, the search is a Viterbi run whose */
+/* first state must have top bits o and whose last state must have low bits */
+/* o; the exact optimum is the best of the 2^(L-k) runs, one per o.         */
 /* orc_viterbi_pinned_*: as orc_viterbi_* (same arithmetic and tie-breaks)  */
 /* with those two restrictions; returns the minimum cost (INFINITY if no    */
 /* walk satisfies them).                                                     */

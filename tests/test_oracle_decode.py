@@ -1,12 +1,12 @@
 """Pins for the oracle's bitstream decode and pack.
 
-The window formula is the page's decode (QTIP blog, "The trellis: a stateful
-codebook"): with the stream as one integer of nbits bits read most significant
-first, weight t is ``(bits >> (nbits - L - t*k)) & (2^L - 1)``.  Here it is
-evaluated with Python integers, a route independent of the oracle's numpy bit
-arrays.  A tail-biting stream (QTIP blog, "Tail-biting is worth its
-complexity") is exactly k*T bits and its windows wrap around; evaluating the
-same formula on the stream with its first L - k bits appended gives them.
+The decode rule (QTIP blog, "The trellis: a stateful codebook"): reading the
+stream most significant bit first, weight t is the L-bit number formed by
+stream bits t*k .. t*k + L - 1.  Here it is evaluated on a string of '0'/'1'
+characters, a route independent of the oracle's numpy bit arrays.  A
+tail-biting stream (QTIP blog, "Tail-biting is worth its complexity") is
+exactly k*T bits and its windows wrap around; the same rule on the stream with
+its first L - k bits appended gives them.
 """
 import numpy as np
 import pytest
@@ -22,7 +22,8 @@ def _to_int(words):
 
 
 def _page_window(bits, nbits, t, L, k):
-    return (bits >> (nbits - L - t * k)) & ((1 << L) - 1)
+    text = format(bits, "b").zfill(nbits)          # stream bits, first bit first
+    return int(text[t * k: t * k + L], 2)
 
 
 @pytest.mark.parametrize("L,T", [(8, 13), (12, 40), (16, 256)])

@@ -1,6 +1,7 @@
 """Pins for the oracle's random-sign Hadamard rotation (QTIP blog, "The
-trellis: a stateful codebook": random signs, then a Hadamard matrix, on both
-sides of W, making the weights approximately i.i.d. Gaussian).
+trellis: a stateful codebook": QuIP#'s transform, +-1 signs and a Hadamard
+transform from the left and the right, leaves the entries close to i.i.d.
+Gaussian).
 
 * H_2 = [[1, 1], [1, -1]] and H_n H_n^T = n I (so the rotation is orthonormal);
 * the rotation preserves the Frobenius norm and is undone by its transpose;

@@ -1,7 +1,7 @@
 """Pins for the tail-biting search (QTIP blog, "Tail-biting is worth its
-complexity"): the last state's low L-k bits equal the first state's high L-k
-bits; exact solving takes 2^(L-k) runs with the shared bits fixed; Algorithm 4
-takes two (rotate by T/2, free run, read the overlap at the seam, re-run with
+complexity"): the walk wraps, the trailing L-k bits of the last state being the
+leading L-k bits of the first; exact solving takes 2^(L-k) runs with the shared
+bits fixed; Algorithm 4 takes two (rotate by T/2, free run, read the overlap at the seam, re-run with
 both ends pinned).
 
 * the pinned runs' best equals brute force over tail-biting walks only;

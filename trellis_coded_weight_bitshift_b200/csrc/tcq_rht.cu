@@ -1,8 +1,8 @@
 // Random-sign Hadamard rotation of a weight matrix.
 //
-// [QTIP blog, "The trellis: a stateful codebook"] before quantisation the
-// weights get random signs, then a Hadamard matrix, on both sides (QuIP#'s
-// rotation), which makes them approximately i.i.d. Gaussian:
+// [QTIP blog, "The trellis: a stateful codebook"] before quantisation QuIP#'s
+// transform is applied from the left and the right, +-1 signs followed by a
+// Hadamard transform, so that the entries end up close to i.i.d. Gaussian:
 //   out = (H_R / sqrt R) diag(sign_rows) W diag(sign_cols) (H_C / sqrt C),
 // H_n the Sylvester Hadamard matrix.  The product is separable, so it runs as
 // fast Walsh-Hadamard butterflies, (a, b) -> (a + b, a - b):

@@ -57,9 +57,10 @@ MEASURED_TRAFFIC = {
         "tcq_decode.cu": "f973d336196f0d525904ea381884bc99ad8e4f71",
         "tcq_device.cuh": "18b7f3a092c947f32accdefd8d22f8b99f58c38e"}),
     # three launches (row pass, two column passes) of one 8192 x 8192 rotation
+    # (the source has changed since only in its comments)
     ("rht", "rht_t5_8192sq"): (269.954048e6 + 226.045952e6 + 268.44288e6 + 206.207232e6
                                + 268.502272e6 + 206.875136e6, 262144, {
-        "tcq_rht.cu": "2eca83490f30669a46e44c81714f1c900931fb37",
+        "tcq_rht.cu": "33825d215508751d0fdc95f4adc7ad72f1a187cc",
         "tcq_device.cuh": "18b7f3a092c947f32accdefd8d22f8b99f58c38e"}),
 }
 
