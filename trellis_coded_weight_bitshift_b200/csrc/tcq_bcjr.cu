@@ -69,7 +69,7 @@ __device__ __forceinline__ float lse4_base2(float x0, float x1, float x2, float 
 }
 
 template <int L_, int G_, int SPC_, int AREG_, int NBUF_, bool GRAD_, int MINB_ = 1,
-          bool TMEMC_ = false>
+          bool TMEMC_ = false, bool MSG2_ = false>
 struct BcjrCfg {
   static constexpr int L = L_, G = G_, SPC = SPC_, AREG = AREG_, NBUF = NBUF_;
   static constexpr int MINB = MINB_;                // CTAs per SM the registers must allow
@@ -92,8 +92,13 @@ struct BcjrCfg {
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
   static constexpr int NV = GRAD ? 2 : 1;                        // carried vectors (A | A, Phi)
   static constexpr int SPILL = NV * G;                           // floats spilled per thread-step
+  // MSG2 (gradient, NBUF = 1): the message vector (A, B) is double-buffered and
+  // read block by block after the step's first barrier; only the expectation
+  // vector (Phi, Psi) is single-buffered and read ahead of it
+  static constexpr bool MSG2 = MSG2_;
+  static constexpr int VPS = MSG2 ? 3 : NBUF * NV;              // state vectors per sequence
   static constexpr size_t smem_floats() {
-    return (size_t)SPC * NBUF * NV * NG                            // state vectors
+    return (size_t)SPC * VPS * NG                                  // state vectors
            + (TMEMC ? 0 : (size_t)ASM * G * TPS)                    // smem code values
            + (size_t)SPC * 256 * (GRAD ? 4 : 2)                     // s, kappa*D (+ v, soft)
            + (size_t)SPC * 256                                       // CA_t increments
@@ -118,6 +123,7 @@ struct BcjrCfg {
   static_assert(!TMEMC || (SPC == 1 && NT % 128 == 0 && (TCOLS & (TCOLS - 1)) == 0 && TCOLS <= 512 &&
                            G % 8 == 0), "tensor-memory code layout");
   static_assert(SPILL % 4 == 0, "spill in float4 chunks");
+  static_assert(!MSG2 || (GRAD && NBUF == 1 && GQ % 4 == 0), "split buffering is for the gradient");
   static_assert(!NAMED || (SPC <= 15 && !TMEMC), "named barriers 1..15, code values in shared memory");
 };
 
@@ -295,7 +301,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   constexpr bool GRAD = C::GRAD;
   extern __shared__ __align__(16) float smem[];
   float *Vall = smem;                                      // [SPC][NB][NV][NG]
-  float2 *Csm = reinterpret_cast<float2 *>(Vall + SPC * NB * NV * NG);  // [HS][G][TPS]
+  float2 *Csm = reinterpret_cast<float2 *>(Vall + SPC * C::VPS * NG);  // [HS][G][TPS]
   float *ssm = reinterpret_cast<float *>(Csm + (C::TMEMC ? 0 : C::HS * G * TPS));  // [SPC][256]
   float *ksm = ssm + SPC * 256;                            // [SPC][256] kappa * D_t
   float *vsm = ksm + SPC * 256;                            // GRAD: v, soft rows
@@ -379,8 +385,22 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     } else {
       for (int x = tid; x < SPC * T; x += C::NT) load_row(x / T, x % T, base);
     }
-    float *V = Vall + ls * NB * NV * NG;
-    for (int x = w; x < NV * NG; x += TPS) V[x] = 0.0f;     // A_0 = 0 (and Phi_0 = 0)
+    float *V = Vall + ls * C::VPS * NG;
+    // the message (A or B) and expectation (Phi or Psi) vectors of step x >= -1
+    auto msg_buf = [&](int x) -> float * {
+      return C::MSG2 ? V + (x & 1) * NG : V + ((x + NB) % NB) * NV * NG;
+    };
+    auto exp_buf = [&](int x) -> float * {
+      return C::MSG2 ? V + 2 * NG : V + ((x + NB) % NB) * NV * NG + NG;
+    };
+    if constexpr (C::MSG2) {
+      for (int x = w; x < NG; x += TPS) {                 // A_0 = 0, Phi_0 = 0
+        msg_buf(0)[x] = 0.0f;
+        exp_buf(0)[x] = 0.0f;
+      }
+    } else {
+      for (int x = w; x < NV * NG; x += TPS) V[x] = 0.0f;   // A_0 = 0 (and Phi_0 = 0)
+    }
     if constexpr (C::NAMED) {
       for (int x = w; x < NPART * PREC; x += TPS) { prec(0)[x] = 0.0f; prec(1)[x] = 0.0f; }
     } else {
@@ -395,13 +415,18 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     // up to kappa max(e) per step) while what the combine needs is small.
     float CA = 0.0f, cmax = 0.0f;
     if (w == 0) cah[ls * 256] = 0.0f;
-    for (int t = 1; t <= T; ++t) {
-      const float *Ai = V + ((t - 1) % NB) * NV * NG;
+    // MSG2: the loop stops before step T, whose spill of A_{T-1} and
+    // Phi_{T-1} follows the loop; inside it A_{t-1} is read (and spilled)
+    // block by block in the step itself
+    constexpr bool lazyA = C::MSG2;
+    for (int t = 1; t <= (C::MSG2 ? T - 1 : T); ++t) {
+      const float *Ai = C::MSG2 ? msg_buf(t - 1) : V + ((t - 1) % NB) * NV * NG;
+      const float *Fi = C::MSG2 ? exp_buf(t - 1) : Ai + NG;
       float ain[4][GQ], fin[GRAD ? 4 : 1][GQ];
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
-        read_run<C>(Ai, a * (NG / 4) + GQ * w, ain[a]);
-        if (GRAD) read_run<C>(Ai + NG, a * (NG / 4) + GQ * w, fin[a < (GRAD ? 4 : 1) ? a : 0]);
+        if (!lazyA) read_run<C>(Ai, a * (NG / 4) + GQ * w, ain[a]);
+        if (GRAD) read_run<C>(Fi, a * (NG / 4) + GQ * w, fin[a < (GRAD ? 4 : 1) ? a : 0]);
       }
       cmax = 0.0f;
       if (t > 1) {
@@ -416,19 +441,21 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int k = 0; k < GQ; ++k) {
-            flat[a * GQ + k] = ain[a][k];
+            flat[a * GQ + k] = lazyA ? 0.0f : ain[a][k];
             if (GRAD) flat[G + a * GQ + k] = fin[a < (GRAD ? 4 : 1) ? a : 0][k];
           }
 #pragma unroll
         for (int c = 0; c < NCH; ++c)
-          spill[((size_t)(t - 1) * NCH + c) * TPS + w] =
-              make_float4(flat[4 * c], flat[4 * c + 1], flat[4 * c + 2], flat[4 * c + 3]);
+          if (!lazyA || 4 * c >= G)
+            spill[((size_t)(t - 1) * NCH + c) * TPS + w] =
+                make_float4(flat[4 * c], flat[4 * c + 1], flat[4 * c + 2], flat[4 * c + 3]);
       }
       if (t == T) break;
       if (w == 0) cah[ls * 256 + t] = cmax;
       if (NB == 1) seq_sync<C>(ls);
       CA += cmax;
-      float *Ao = V + (t % NB) * NV * NG;
+      float *Ao = C::MSG2 ? msg_buf(t) : V + (t % NB) * NV * NG;
+      float *Fo = C::MSG2 ? exp_buf(t) : Ao + NG;
       const float sv = ssm[ls * 256 + t - 1];
       const float vv = GRAD ? vsm[ls * 256 + t - 1] : 0.0f;
       const float fv = GRAD ? fsm[ls * 256 + t - 1] : 0.0f;
@@ -460,6 +487,16 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         const f2_t vv2 = f2(vv, vv), vf2 = f2(vv * fv, vv * fv);
 #pragma unroll
         for (int q = 0; q < GQ; ++q) {
+          if (lazyA && (q & 3) == 0) {                      // A_{t-1} for groups 4q .. 4q + 15
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              const float4 v =
+                  *reinterpret_cast<const float4 *>(Ai + swz<C::SWZ>(a * (NG / 4) + GQ * w + q));
+              ain[a][q] = v.x; ain[a][(q + 1) % GQ] = v.y;
+              ain[a][(q + 2) % GQ] = v.z; ain[a][(q + 3) % GQ] = v.w;
+              spill[((size_t)(t - 1) * NCH + (a * GQ + q) / 4) * TPS + w] = v;
+            }
+          }
           const f2_t am0 = f2sub(f2(ain[0][q], ain[1][q]), cm2);
           const f2_t am1 = f2sub(f2(ain[2][q], ain[3][q]), cm2);
           const f2_t ph0 = f2sub(f2(fin[0][q], fin[1][q]), vf2);
@@ -490,13 +527,33 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           }
           *reinterpret_cast<float4 *>(Ao + swz<C::SWZ>(G * w + 4 * q)) =
               make_float4(outA[0], outA[1], outA[2], outA[3]);
-          *reinterpret_cast<float4 *>(Ao + NG + swz<C::SWZ>(G * w + 4 * q)) =
+          *reinterpret_cast<float4 *>(Fo + swz<C::SWZ>(G * w + 4 * q)) =
               make_float4(outF[0], outF[1], outF[2], outF[3]);
         }
       }
       tmax = seq_max<TPS>(tmax);
       if (plead) prec(t & 1)[pidx * PREC] = tmax;
       seq_sync<C>(ls);
+    }
+    if constexpr (C::MSG2) {                                 // step T: spill A_{T-1}, Phi_{T-1}
+      cmax = 0.0f;
+      if (T > 1) {
+        const float *pp = prec((T - 1) & 1);
+        cmax = pp[0];
+#pragma unroll
+        for (int x = 1; x < NPART; ++x) cmax = fmaxf(cmax, pp[x * PREC]);
+      }
+      const float *Ai = msg_buf(T - 1);
+      const float *Fi = exp_buf(T - 1);
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int q = 0; q < GQ; q += 4) {
+          const float4 va = *reinterpret_cast<const float4 *>(Ai + swz<C::SWZ>(a * (NG / 4) + GQ * w + q));
+          const float4 vf = *reinterpret_cast<const float4 *>(Fi + swz<C::SWZ>(a * (NG / 4) + GQ * w + q));
+          spill[((size_t)(T - 1) * NCH + (a * GQ + q) / 4) * TPS + w] = va;
+          spill[((size_t)(T - 1) * NCH + (G + a * GQ + q) / 4) * TPS + w] = vf;
+        }
     }
     // CA = CA_{T-1}; cmax = max of stored A_{T-1}; spill step T-1 holds A_{T-1}.
 
@@ -562,7 +619,14 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     // K_{tc-1} = K_tc + (CA_tc - CA_{tc-1}) - (DB_{tc-1} - DB_tc), starting
     // from log2 Z - CA_{T-1}, so no two huge sums are ever subtracted.
     float *Bv = V;
-    for (int x = w; x < NV * NG; x += TPS) Bv[((T - 1) % NB) * NV * NG + x] = 0.0f;
+    if constexpr (C::MSG2) {
+      for (int x = w; x < NG; x += TPS) {                 // B_{T-1} = 0, Psi_{T-1} = 0
+        msg_buf(T - 1)[x] = 0.0f;
+        exp_buf(T - 1)[x] = 0.0f;
+      }
+    } else {
+      for (int x = w; x < NV * NG; x += TPS) Bv[((T - 1) % NB) * NV * NG + x] = 0.0f;
+    }
     seq_sync<C>(ls);
     float Krun = log2Zrel;
     for (int t = T - 2; t >= -1; --t) {
@@ -584,14 +648,17 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
             prefetch_global<TCQ_SPILL_PREFETCH_LEVEL>(&spill[((size_t)(tc - 1) * NCH + c) * TPS + w]);
         }
       }
-      const float *Bi = Bv + (tc % NB) * NV * NG;
-      float bin[G], pin[GRAD ? G : 1];
+      const float *Bi = C::MSG2 ? msg_buf(tc) : Bv + (tc % NB) * NV * NG;
+      const float *Pi = C::MSG2 ? exp_buf(tc) : Bi + NG;
+      float bin[C::MSG2 ? 1 : G], pin[GRAD ? G : 1];
 #pragma unroll
       for (int q = 0; q < GQ; ++q) {
-        const float4 v = *reinterpret_cast<const float4 *>(Bi + swz<C::SWZ>(G * w + 4 * q));
-        bin[4 * q] = v.x; bin[4 * q + 1] = v.y; bin[4 * q + 2] = v.z; bin[4 * q + 3] = v.w;
+        if constexpr (!C::MSG2) {                            // MSG2: read where used
+          const float4 v = *reinterpret_cast<const float4 *>(Bi + swz<C::SWZ>(G * w + 4 * q));
+          bin[4 * q] = v.x; bin[4 * q + 1] = v.y; bin[4 * q + 2] = v.z; bin[4 * q + 3] = v.w;
+        }
         if (GRAD) {
-          const float4 f = *reinterpret_cast<const float4 *>(Bi + NG + swz<C::SWZ>(G * w + 4 * q));
+          const float4 f = *reinterpret_cast<const float4 *>(Pi + swz<C::SWZ>(G * w + 4 * q));
           pin[4 * q] = f.x; pin[4 * q + 1] = f.y; pin[4 * q + 2] = f.z; pin[4 * q + 3] = f.w;
         }
       }
@@ -621,7 +688,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       const float sv = ssm[ls * 256 + tc];
       const float vv = GRAD ? vsm[ls * 256 + tc] : 0.0f;
       const float fv = GRAD ? fsm[ls * 256 + tc] : 0.0f;
-      float *Bo = Bv + ((t + NB) % NB) * NV * NG;
+      float *Bo = C::MSG2 ? msg_buf(t) : Bv + ((t + NB) % NB) * NV * NG;
+      float *Po = C::MSG2 ? exp_buf(t) : Bo + NG;
       float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f, tmax = -INFINITY;
       const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + tc], -ksm[ls * 256 + tc]);
       const f2_t K2 = f2(K, K), dp2 = f2(dprev, dprev), vv2 = f2(vv, vv);
@@ -670,10 +738,18 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
             } else {
               codes.template pairs<4>(h, 4 * k, cc);
             }
+            float bk[4];                                     // B_{tc+1} of the successors
+            if constexpr (C::MSG2) {
+              const float4 v = *reinterpret_cast<const float4 *>(Bi + swz<C::SWZ>(G * w + 4 * k));
+              bk[0] = v.x; bk[1] = v.y; bk[2] = v.z; bk[3] = v.w;
+            } else {
+#pragma unroll
+              for (int b = 0; b < 4; ++b) bk[b] = bin[C::MSG2 ? 0 : 4 * k + b];
+            }
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
               const f2_t d = f2sub(cc[b], sv2);
-              y[b] = f2fma(f2mul(d, nk2), d, f2(bin[4 * k + b], bin[4 * k + b]));
+              y[b] = f2fma(f2mul(d, nk2), d, f2(bk[b], bk[b]));
             }
             const float mxl = fmaxf(fmaxf(f2lo(y[0]), f2lo(y[1])), fmaxf(f2lo(y[2]), f2lo(y[3])));
             const float mxh = fmaxf(fmaxf(f2hi(y[0]), f2hi(y[1])), fmaxf(f2hi(y[2]), f2hi(y[3])));
@@ -720,8 +796,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
             write_sub<C, KB>(Bo, bl, outL);
             write_sub<C, KB>(Bo, bh, outH);
             if constexpr (GRAD) {
-              write_sub<C, KB>(Bo + NG, bl, outPL);
-              write_sub<C, KB>(Bo + NG, bh, outPH);
+              write_sub<C, KB>(Po, bl, outPL);
+              write_sub<C, KB>(Po, bh, outPH);
             }
           }
         }
@@ -819,7 +895,7 @@ using Grad12 = BcjrCfg<12, 8, 7, 0, 2, true, 1>;
 // L = 16 gradient: code values in tensor memory as in the soft pass; the two
 // carried vectors (A and Phi, 2 x 64 KiB) fit the shared memory only
 // single-buffered, so each step takes two barriers.
-using Grad16 = BcjrCfg<16, 32, 1, 0, 1, true, 1, true>;
+using Grad16 = BcjrCfg<16, 32, 1, 0, 1, true, 1, true, true>;
 
 template <class C>
 int grid_for(int64_t n_seq) {
