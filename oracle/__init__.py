@@ -104,6 +104,40 @@ def _row_ptr(D, i):
     return None if D is None else _ptr(D[i])
 
 
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:                                  # not Linux
+        return os.cpu_count() or 1
+
+
+def map_rows(fn, arrays, *args, threads: int | None = None, **kw):
+    """Apply a row-wise routine of this module to contiguous row blocks of
+    ``arrays`` (a list of [n, ...] arrays, passed positionally before
+    ``args``) in a thread pool, and join each output along rows.  Keyword
+    arrays with n rows (e.g. ``D``) are cut the same way.  The C routines run
+    without the GIL, so the blocks run on separate cores; every row is still
+    computed by the same plain routine, one at a time."""
+    from concurrent.futures import ThreadPoolExecutor
+    n = arrays[0].shape[0]
+    threads = max(1, min(threads or host_threads(), n))
+    edges = np.linspace(0, n, threads + 1).astype(int)
+
+    def part(i):
+        lo, hi = edges[i], edges[i + 1]
+        kws = {key: (v[lo:hi] if isinstance(v, np.ndarray) and v.ndim >= 1 and v.shape[0] == n else v)
+               for key, v in kw.items()}
+        return fn(*[a[lo:hi] for a in arrays], *args, **kws)
+
+    _lib()                                                  # build and load once, before the threads
+    with ThreadPoolExecutor(threads) as ex:
+        outs = list(ex.map(part, range(threads)))
+    if not isinstance(outs[0], tuple):
+        return np.concatenate(outs)
+    return tuple(np.concatenate([o[j] for o in outs]) for j in range(len(outs[0])))
+
+
 # --------------------------------------------------------------------------
 # 1MAD codebook
 # --------------------------------------------------------------------------
@@ -182,7 +216,8 @@ def viterbi_f64(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = Non
 # --------------------------------------------------------------------------
 # Tail-biting search (QTIP blog, "Tail-biting is worth its complexity")
 # --------------------------------------------------------------------------
-def viterbi_pinned_f32(s: np.ndarray, L: int, overlap, k: int = 2, D=None):
+def viterbi_pinned_f32(s: np.ndarray, L: int, overlap, k: int = 2, D=None,
+                       code: np.ndarray | None = None):
     """fp32 Viterbi with the first state's top L-k bits and the last state's
     low L-k bits both equal to ``overlap`` (per row); returns (states, cost)."""
     s = np.ascontiguousarray(s, dtype=np.float32)
@@ -191,11 +226,29 @@ def viterbi_pinned_f32(s: np.ndarray, L: int, overlap, k: int = 2, D=None):
     n, T = s.shape
     D = _rows(D, n, T, np.float32)
     overlap = np.broadcast_to(np.asarray(overlap, dtype=np.int64), (n,))
-    code = codebook_f32(L)
+    code = codebook_f32(L) if code is None else np.ascontiguousarray(code, dtype=np.float32)
     states = np.empty((n, T), dtype=np.uint16)
     cost = np.empty(n, dtype=np.float32)
     for i in range(n):
         cost[i] = _lib().orc_viterbi_pinned_f32(L, k, T, _ptr(s[i]), _row_ptr(D, i), _ptr(code),
+                                                int(overlap[i]), _ptr(states[i]))
+    return states, cost
+
+
+def viterbi_pinned_f64(s: np.ndarray, L: int, overlap, k: int = 2, D=None,
+                       code: np.ndarray | None = None):
+    """fp64 form of ``viterbi_pinned_f32``; returns (states, cost)."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    if s.ndim == 1:
+        s = s[None]
+    n, T = s.shape
+    D = _rows(D, n, T, np.float64)
+    overlap = np.broadcast_to(np.asarray(overlap, dtype=np.int64), (n,))
+    code = codebook_f64(L) if code is None else np.ascontiguousarray(code, dtype=np.float64)
+    states = np.empty((n, T), dtype=np.uint16)
+    cost = np.empty(n, dtype=np.float64)
+    for i in range(n):
+        cost[i] = _lib().orc_viterbi_pinned_f64(L, k, T, _ptr(s[i]), _row_ptr(D, i), _ptr(code),
                                                 int(overlap[i]), _ptr(states[i]))
     return states, cost
 

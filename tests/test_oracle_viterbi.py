@@ -100,3 +100,108 @@ def test_monotone_code_loses_to_scalar_rounding(L, n):
     m = float(np.mean(mse))
     assert abs(m - g[f"L{L}"]) <= 0.004 + 3 * float(np.std(mse)) / np.sqrt(n), m
     assert m > 0.118    # worse than the 4-level Lloyd-Max scalar quantiser on the page
+
+
+# ---------------------------------------------------------------- tie-break rule
+# The page's Viterbi sketch (QTIP blog, "The trellis: a stateful codebook")
+# takes numpy's argmin, which keeps the FIRST minimum: at every step the
+# lowest predecessor digit a -- the candidates (j >> k) | (a << (L - k)) differ
+# only in their top k bits, so this is also the lowest predecessor state --
+# and, at the end, the lowest state.  Among all minimum-energy walks the
+# returned one is therefore the smallest when walks are compared state by
+# state from the LAST step backwards.  The pins below check that rule by
+# enumerating every walk on codebooks with repeated values, where exact cost
+# ties are everywhere; a `<=` in place of `<` in any argmin of the oracle
+# returns a different walk.
+
+def _walks(L, k, T):
+    """Every walk [2^(L + k(T-1)), T] of the bitshift trellis (free start)."""
+    mask = (1 << L) - 1
+    x0 = np.arange(1 << L, dtype=np.int64)
+    walks = x0[:, None]
+    for _ in range(1, T):
+        nxt = ((walks[:, -1:] << k) | np.arange(1 << k, dtype=np.int64)[None, :]) & mask
+        walks = np.concatenate([np.repeat(walks, 1 << k, axis=0), nxt.reshape(-1, 1)], axis=1)
+    return walks
+
+
+def _energies(walks, s, code, f32):
+    """Energy of each walk summed left to right, each operation rounded in the
+    given precision (the order the recursion adds the step costs in)."""
+    dt = np.float32 if f32 else np.float64
+    c = np.asarray(code, dtype=dt)[walks]
+    acc = np.zeros(walks.shape[0], dtype=dt)
+    for t in range(walks.shape[1]):
+        d = (c[:, t] - dt(s[t])).astype(dt)
+        acc = (acc + (d * d).astype(dt)).astype(dt)
+    return acc
+
+
+def _lowest_min_walk(walks, energies):
+    best = walks[energies == energies.min()]
+    order = np.lexsort(best.T)           # last column is the primary key
+    return best[order[0]]
+
+
+def test_all_ties_give_the_lowest_index_walk_by_hand():
+    # all-zero codebook: every candidate of every decision ties.  Lowest digit
+    # at each step and lowest final state give the all-zero walk; a `<=` slip
+    # in the step argmin gives predecessor 12 (digit 3), in the final argmin
+    # state 15.
+    L, T = 4, 4
+    s = np.array([[0.3, -0.2, 1.5, 0.0]], dtype=np.float32)
+    zero = np.zeros(1 << L)
+    st32, _ = oracle.viterbi_f32(s, L, code=zero.astype(np.float32))
+    st64, _, _ = oracle.viterbi_f64(s, L, code=zero)
+    assert st32[0].tolist() == [0, 0, 0, 0]
+    assert st64[0].tolist() == [0, 0, 0, 0]
+    # pinned to overlap o = 1 (first state's top 2 bits, last state's low 2
+    # bits): step 1 has one finite candidate, digit 1 (state 4 | (j >> 2)),
+    # step 2 ties four ways (digit 0), the end is the lowest state with low
+    # bits 1: walk [4, 0, 1]
+    s3 = s[:, :3]
+    st, _ = oracle.viterbi_pinned_f32(s3, L, 1, code=zero.astype(np.float32))
+    assert st[0].tolist() == [4, 0, 1]
+    st, _ = oracle.viterbi_pinned_f64(s3, L, 1, code=zero)
+    assert st[0].tolist() == [4, 0, 1]
+
+
+@pytest.mark.parametrize("f32", [True, False])
+def test_ties_on_repeated_code_values_match_enumeration(f32):
+    L, k, T = 4, 2, 4
+    rng = np.random.default_rng(4242 + f32)
+    walks = _walks(L, k, T)
+    n_multi = 0
+    for trial in range(40):
+        # three code values and integer targets: many walks share the minimum
+        code = rng.integers(-1, 2, 1 << L).astype(np.float64)
+        s = rng.integers(-1, 2, T).astype(np.float64)
+        E = _energies(walks, s, code, f32)
+        n_multi += int((E == E.min()).sum() > 1)
+        want = _lowest_min_walk(walks, E)
+        if f32:
+            st, _ = oracle.viterbi_f32(s.astype(np.float32)[None], L, code=code.astype(np.float32))
+        else:
+            st, _, _ = oracle.viterbi_f64(s[None], L, code=code)
+        assert st[0].tolist() == want.tolist(), (trial, code, s)
+    assert n_multi >= 30                   # the cases really have tied optima
+
+
+@pytest.mark.parametrize("f32", [True, False])
+def test_pinned_ties_match_enumeration(f32):
+    L, k, T = 4, 2, 4
+    low = (1 << (L - k)) - 1
+    rng = np.random.default_rng(4343 + f32)
+    walks = _walks(L, k, T)
+    for trial in range(30):
+        code = rng.integers(-1, 2, 1 << L).astype(np.float64)
+        s = rng.integers(-1, 2, T).astype(np.float64)
+        o = int(rng.integers(0, 1 << (L - k)))
+        ok = ((walks[:, 0] >> k) == o) & ((walks[:, -1] & low) == o)
+        E = _energies(walks[ok], s, code, f32)
+        want = _lowest_min_walk(walks[ok], E)
+        if f32:
+            st, _ = oracle.viterbi_pinned_f32(s.astype(np.float32)[None], L, o, code=code.astype(np.float32))
+        else:
+            st, _ = oracle.viterbi_pinned_f64(s[None], L, o, code=code)
+        assert st[0].tolist() == want.tolist(), (trial, o, code, s)
