@@ -106,7 +106,8 @@ TCQ_API size_t tcq_stream_words(const tcq_trellis_t *trellis, int layout);
  *   cost_t(j) = min_a cost_{t-1}((j >> k) | (a << (L-k))) + (code_j - s_t)^2,
  * free start, free end.  fp32 arithmetic with each operation rounded on its
  * own (d = code - s, e = d*d, cost = best + e; no fused multiply-add); ties go
- * to the lowest predecessor digit a, and the final argmin to the lowest state.
+ * to the lowest predecessor digit a, and the final argmin to the lowest state
+ * (the first minimum, as the sketch's argmin takes it).
  *
  *   s          [n_seq][seq_len] fp32 targets (input).
  *   D          [n_seq][seq_len] fp32 per-weight curvature, or NULL for all
@@ -117,6 +118,18 @@ TCQ_API size_t tcq_stream_words(const tcq_trellis_t *trellis, int layout);
  *   states     [n_seq][seq_len] uint16: the chosen walk, state (L-bit window)
  *              of every weight (output).
  *   mse        [n_seq] fp32: minimum total cost / seq_len (output).
+ *   min_margin [n_seq] fp32 (output, may be NULL): the smallest relative
+ *              decision margin along the returned walk, so that a caller
+ *              can count the sequences whose walk is decided by a near-tie.
+ *              The decisions are each step's choice among the 2^k
+ *              predecessors of the walk's state (candidates cost_{t-1}) and
+ *              the final choice among all states (candidates cost_{T-1});
+ *              a decision's margin is (second - best) / max(best, 1e-30),
+ *              subtraction and division each rounded to fp32, with "second"
+ *              the smallest candidate strictly above the best (exact ties are
+ *              settled by the index rule and have no margin).  +inf when no
+ *              decision had two distinct candidates.  Computing it re-runs
+ *              the forward recursion once more (about twice the time).
  *   ws         device workspace of at least tcq_viterbi_workspace_size()
  *              bytes, 256-byte aligned; it holds the 2-bit backpointers.
  * Returns TCQ_OK, or an error as described above.
@@ -125,7 +138,8 @@ TCQ_API size_t tcq_viterbi_workspace_size(const tcq_trellis_t *trellis, int64_t 
 
 TCQ_API tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *trellis, const float *s,
                                         const float *D, int64_t n_seq, uint16_t *states,
-                                        float *mse, void *ws, size_t ws_bytes, void *stream);
+                                        float *mse, float *min_margin, void *ws, size_t ws_bytes,
+                                        void *stream);
 
 /* ------------------------------------------------------------------------
  * Tail-biting Viterbi encode [QTIP, "Tail-biting is worth its complexity":

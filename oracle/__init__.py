@@ -69,7 +69,7 @@ def _lib():
     lib.orc_1mad_f32.restype = ctypes.c_float
     lib.orc_codebook_1mad_f64.argtypes = [I, P]
     lib.orc_codebook_1mad_f32.argtypes = [I, P]
-    lib.orc_viterbi_f32.argtypes = [I, I, I, P, P, P, P]
+    lib.orc_viterbi_f32.argtypes = [I, I, I, P, P, P, P, P]
     lib.orc_viterbi_f32.restype = ctypes.c_float
     lib.orc_viterbi_f64.argtypes = [I, I, I, P, P, P, P, P]
     lib.orc_viterbi_f64.restype = D
@@ -169,12 +169,14 @@ def codebook_f16(L: int) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Viterbi
 # --------------------------------------------------------------------------
-def viterbi_f32(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None, D=None):
+def viterbi_f32(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None, D=None,
+                margin: bool = False):
     """fp32-canonical Viterbi on each row of ``s`` [n, T] (optional per-weight
     curvature ``D`` [n, T], step cost D_t (code - s_t)^2).
 
     Returns (states uint16 [n, T], mse float32 [n]) with mse = min cost / T
-    computed in fp32."""
+    computed in fp32; with ``margin=True`` also the smallest fp32 relative
+    decision margin along each returned walk (float32 [n])."""
     s = np.ascontiguousarray(s, dtype=np.float32)
     if s.ndim == 1:
         s = s[None]
@@ -183,13 +185,17 @@ def viterbi_f32(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = Non
     code = codebook_f32(L) if code is None else np.ascontiguousarray(code, dtype=np.float32)
     states = np.empty((n, T), dtype=np.uint16)
     mse = np.empty(n, dtype=np.float32)
+    mrg = np.empty(n, dtype=np.float32)
     lib = _lib()
+    m = ctypes.c_float()
     for i in range(n):
         row = s[i]
         st = states[i]
-        cost = lib.orc_viterbi_f32(L, k, T, _ptr(row), _row_ptr(D, i), _ptr(code), _ptr(st))
+        cost = lib.orc_viterbi_f32(L, k, T, _ptr(row), _row_ptr(D, i), _ptr(code), _ptr(st),
+                                   ctypes.byref(m) if margin else None)
         mse[i] = np.float32(cost) / np.float32(T)
-    return states, mse
+        mrg[i] = m.value if margin else np.nan
+    return (states, mse, mrg) if margin else (states, mse)
 
 
 def viterbi_f64(s: np.ndarray, L: int, k: int = 2, code: np.ndarray | None = None, D=None):

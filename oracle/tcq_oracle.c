@@ -78,14 +78,32 @@ void orc_codebook_1mad_f32(int L, float *out)
 /* multiply-add).  The argmin over a keeps the     */
 /* first (lowest a) minimum, like numpy's argmin; the final argmin keeps the */
 /* lowest state.  Returns the minimum total cost; states[0..T-1] the walk.   */
+/*                                                                           */
+/* min_margin (nullable): the smallest relative decision margin along the   */
+/* returned walk, in fp32.  A decision is each step's choice among the 2^k  */
+/* predecessors of the walk's state (candidates cost_{t-1}(pred_a)) and the */
+/* final choice among all states (candidates cost_{T-1}); its margin is     */
+/* (second - best) / max(best, 1e-30), subtraction and division each        */
+/* rounded to fp32, where "second" is the smallest candidate strictly above */
+/* the best (exact ties are settled by index identically at any precision). */
+/* INFINITY when no decision had two distinct candidates.                   */
 /* ------------------------------------------------------------------------ */
+static float rel_gap_f32(float best, float second)
+{
+    float den = best > 1e-30f ? best : 1e-30f;
+    float gap = second - best;
+    return gap / den;
+}
+
 float orc_viterbi_f32(int L, int k, int T, const float *s, const float *D, const float *code,
-                      uint16_t *states)
+                      uint16_t *states, float *min_margin)
 {
     const int N = 1 << L, A = 1 << k;
-    float *cost = (float *)malloc(sizeof(float) * N);
-    float *next = (float *)malloc(sizeof(float) * N);
+    /* every step's cost vector is kept when margins are wanted, else two */
+    const int keep = min_margin ? T : 2;
+    float *all = (float *)malloc(sizeof(float) * (size_t)keep * N);
     int32_t *back = (int32_t *)malloc(sizeof(int32_t) * (size_t)T * N);
+    float *cost = all, *next = all + N;
 
     for (int j = 0; j < N; ++j) {
         float d = code[j] - s[0];
@@ -93,6 +111,7 @@ float orc_viterbi_f32(int L, int k, int T, const float *s, const float *D, const
         cost[j] = D ? e * D[0] : e;
     }
     for (int t = 1; t < T; ++t) {
+        if (min_margin) next = all + (size_t)t * N;
         for (int j = 0; j < N; ++j) {
             float best = INFINITY;
             int bestp = -1;
@@ -112,12 +131,30 @@ float orc_viterbi_f32(int L, int k, int T, const float *s, const float *D, const
     for (int j = 1; j < N; ++j)
         if (cost[j] < cost[st]) st = j;
     float total = cost[st];
+    float margin = INFINITY;
+    if (min_margin) {   /* final decision: the smallest cost strictly above the best */
+        float second = INFINITY;
+        for (int j = 0; j < N; ++j)
+            if (cost[j] > total && cost[j] < second) second = cost[j];
+        if (second < INFINITY) margin = fminf(margin, rel_gap_f32(total, second));
+    }
     states[T - 1] = (uint16_t)st;
     for (int t = T - 1; t > 0; --t) {
-        st = back[(size_t)t * N + st];
+        int bestp = back[(size_t)t * N + st];
+        if (min_margin) {   /* the walk's decision at step t, over cost_{t-1} */
+            const float *prev = all + (size_t)(t - 1) * N;
+            float best = prev[bestp], second = INFINITY;
+            for (int a = 0; a < A; ++a) {
+                int p = (st >> k) | (a << (L - k));
+                if (prev[p] > best && prev[p] < second) second = prev[p];
+            }
+            if (second < INFINITY) margin = fminf(margin, rel_gap_f32(best, second));
+        }
+        st = bestp;
         states[t - 1] = (uint16_t)st;
     }
-    free(cost); free(next); free(back);
+    if (min_margin) *min_margin = margin;
+    free(all); free(back);
     return total;
 }
 

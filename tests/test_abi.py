@@ -45,26 +45,28 @@ def test_invalid_arguments_return_status_without_launch(L):
     from trellis_coded_weight_bitshift_b200 import _abi
     tr = _abi.trellis(10, 256)                     # unsupported L
     bad = ctypes.c_void_p(16)                      # never dereferenced on these paths
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 1, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_UNSUPPORTED
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 1, bad, bad, None, bad, 1 << 20, None) == _abi.TCQ_ERR_UNSUPPORTED
     tr = _abi.trellis(12, 300)                     # seq_len above 256
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 1, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_UNSUPPORTED
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 1, bad, bad, None, bad, 1 << 20, None) == _abi.TCQ_ERR_UNSUPPORTED
     tr = _abi.trellis(12, 256, k=3)
     assert L.tcq_decode(ctypes.byref(tr), bad, 1, 0, 0, 0, 0, bad, None) == _abi.TCQ_ERR_UNSUPPORTED
     tr = _abi.trellis(12, 256)
     # null pointers
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), None, None, 4, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), None, None, 4, bad, bad, None, bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
     # misaligned pointer
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), ctypes.c_void_p(18), None, 4, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), ctypes.c_void_p(18), None, 4, bad, bad, None, bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
     # workspace too small / missing / misaligned
     need = L.tcq_viterbi_workspace_size(ctypes.byref(tr), 4)
     assert need >= 4 * 255 * 256
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 4, bad, bad, ctypes.c_void_p(256), need - 1, None) == _abi.TCQ_ERR_WORKSPACE
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 4, bad, bad, None, need, None) == _abi.TCQ_ERR_WORKSPACE
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 4, bad, bad, ctypes.c_void_p(128), need, None) == _abi.TCQ_ERR_WORKSPACE
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 4, bad, bad, None, ctypes.c_void_p(256), need - 1, None) == _abi.TCQ_ERR_WORKSPACE
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 4, bad, bad, None, None, need, None) == _abi.TCQ_ERR_WORKSPACE
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 4, bad, bad, None, ctypes.c_void_p(128), need, None) == _abi.TCQ_ERR_WORKSPACE
     # misaligned curvature weights
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, ctypes.c_void_p(20), 4, bad, bad, bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, ctypes.c_void_p(20), 4, bad, bad, None, bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
+    # misaligned decision-margin output
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), bad, None, 4, bad, bad, ctypes.c_void_p(36), bad, 1 << 20, None) == _abi.TCQ_ERR_INVALID_ARG
     # nothing to do
-    assert L.tcq_viterbi_encode(ctypes.byref(tr), None, None, 0, None, None, None, 0, None) == _abi.TCQ_OK
+    assert L.tcq_viterbi_encode(ctypes.byref(tr), None, None, 0, None, None, None, None, 0, None) == _abi.TCQ_OK
     # temperature must be positive and finite
     assert L.tcq_bcjr_soft(ctypes.byref(tr), bad, None, 4, ctypes.c_float(0.0), bad, None, bad, 1 << 30, None) == _abi.TCQ_ERR_INVALID_ARG
     assert L.tcq_bcjr_soft(ctypes.byref(tr), bad, None, 4, ctypes.c_float(float("inf")), bad, None, bad, 1 << 30, None) == _abi.TCQ_ERR_INVALID_ARG

@@ -65,13 +65,21 @@ def test_viterbi_writes_stay_inside(abi, L, n, T, weighted):
     tr = abi.trellis(L, T)
     s, s0, sp = _inp(W.gaussian(n, 900 + T))
     D, D0, Dp = _inp(W.curvature(n, 901, seq_len=T)) if weighted else (s, s0, None)
-    states, mse = Guarded(n * T * 2), Guarded(n * 4)
+    states, mse, margin = Guarded(n * T * 2), Guarded(n * 4), Guarded(n * 4)
     need = lib.tcq_viterbi_workspace_size(ctypes.byref(tr), n)
     ws = Guarded(need)
-    rc = lib.tcq_viterbi_encode(ctypes.byref(tr), sp, Dp, n, states.ptr, mse.ptr, ws.ptr, need, _stream())
+    rc = lib.tcq_viterbi_encode(ctypes.byref(tr), sp, Dp, n, states.ptr, mse.ptr, None, ws.ptr, need,
+                                _stream())
     assert rc == abi.TCQ_OK, abi.status_string(rc)
     assert states.intact() and mse.intact() and ws.intact()
     assert _unchanged((s, s0), (D, D0))
+    # with the decision margins (a second forward pass that reads the walks)
+    st0 = states.buf[GUARD:GUARD + n * T * 2].clone()
+    rc = lib.tcq_viterbi_encode(ctypes.byref(tr), sp, Dp, n, states.ptr, mse.ptr, margin.ptr, ws.ptr,
+                                need, _stream())
+    assert rc == abi.TCQ_OK, abi.status_string(rc)
+    assert states.intact() and mse.intact() and margin.intact() and ws.intact()
+    assert _unchanged((s, s0), (D, D0), (states.buf[GUARD:GUARD + n * T * 2], st0))
 
 
 @pytest.mark.parametrize("L,n,T", [(8, 5, 48), (12, 3, 48), (16, 2, 256)])

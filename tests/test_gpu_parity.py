@@ -117,10 +117,23 @@ def test_pack_matches_oracle_and_roundtrips(tcq, L, layout):
 
 
 # ---------------------------------------------------------------- Viterbi
-def _viterbi_gpu(tcq, s, L):
-    st, mse = tcq.viterbi_encode(_dev(s), L)
+def _viterbi_gpu(tcq, s, L, margin=False, D=None):
+    out = tcq.viterbi_encode(_dev(s), L, margin=margin, D=None if D is None else _dev(D))
     torch.cuda.synchronize()
-    return st.cpu().view(torch.int16).numpy().view(np.uint16), mse.cpu().numpy()
+    st = out[0].cpu().view(torch.int16).numpy().view(np.uint16)
+    return (st,) + tuple(o.cpu().numpy() for o in out[1:])
+
+
+def _same_f32(a, b):
+    """Bit-for-bit equality of fp32 arrays (inf included)."""
+    return np.array_equal(np.asarray(a, np.float32).view(np.uint32), np.asarray(b, np.float32).view(np.uint32))
+
+
+def _margin_bound(m64, T):
+    """|m32 - m64| bound: each fp32 cost carries at most T u relative error
+    (u = 2^-24), plus the rounding of the gap and the division."""
+    u = 2.0 ** -24
+    return 2 * (1 + m64) * T * u + 2 * u * m64
 
 
 @pytest.mark.parametrize("name", ["l8_gauss64", "l12_gauss1024"])
@@ -128,16 +141,24 @@ def test_viterbi_full_workload_bit_exact(tcq, name):
     w = W.WORKLOADS[name]
     s = W.sequences(name)
     st, mse = _viterbi_gpu(tcq, s, w.L)
-    rst, rmse = oracle.map_rows(oracle.viterbi_f32, [s], w.L)
+    rst, rmse, rmg = oracle.map_rows(oracle.viterbi_f32, [s], w.L, margin=True)
     assert np.array_equal(st, rst)
     assert np.array_equal(mse.view(np.uint32), rmse.view(np.uint32))
+    # the decision margins (second pass): same walks, margins bit for bit
+    st2, mse2, mg = _viterbi_gpu(tcq, s, w.L, margin=True)
+    assert np.array_equal(st2, rst) and _same_f32(mse2, rmse)
+    assert _same_f32(mg, rmg)
     # against fp64 on every sequence: walks equal off near-ties (counted and
-    # reported), MSE within 2e-5 relative (fp32 sums of 256 terms)
+    # reported, from the GPU's margins and the fp64 oracle's), MSE within
+    # 2e-5 relative (fp32 sums of 256 terms), margins within their bound
     st64, mse64, margin = oracle.map_rows(oracle.viterbi_f64, [s], w.L)
     near = margin < NEAR_TIE
-    print(f"{name}: {int(near.sum())} near-tie sequences of {s.shape[0]} (fp64 margin < {NEAR_TIE:g})")
+    print(f"{name}: near-tie sequences (margin < {NEAR_TIE:g}): GPU {int((mg < NEAR_TIE).sum())}, "
+          f"fp64 oracle {int(near.sum())} of {s.shape[0]}; smallest GPU margin {mg.min():.3g}")
     assert np.array_equal(st[~near], st64[~near])
     assert np.all(np.abs(mse - mse64) <= 2e-5 * mse64)
+    ok = ~near
+    assert np.all(np.abs(mg[ok].astype(np.float64) - margin[ok]) <= _margin_bound(margin[ok], s.shape[1]))
 
 
 def test_viterbi_l16_rht_block(tcq):
@@ -147,19 +168,25 @@ def test_viterbi_l16_rht_block(tcq):
     assert st.shape == (4096, 256)
     assert np.all(_is_walk(st, 16))
     assert np.array_equal(_seq_mse_f32(s, st, 16).view(np.uint32), mse.view(np.uint32))
+    st2, mse2, mg = _viterbi_gpu(tcq, s, 16, margin=True)          # every sequence's margin
+    assert np.array_equal(st2, st) and _same_f32(mse2, mse)
     idx = np.random.default_rng(3).choice(4096, 62, replace=False)
-    idx = np.concatenate([[0, 4095], idx])
-    rst, rmse = oracle.map_rows(oracle.viterbi_f32, [s[idx]], 16)
+    idx = np.concatenate([[0, 4095, int(np.argmin(mg))], idx])
+    rst, rmse, rmg = oracle.map_rows(oracle.viterbi_f32, [s[idx]], 16, margin=True)
     assert np.array_equal(st[idx], rst)
     assert np.array_equal(mse[idx].view(np.uint32), rmse.view(np.uint32))
+    assert _same_f32(mg[idx], rmg)
     # fp64 oracle on the same sample: walks equal off near-ties (counted and
     # reported), MSE within 2e-5 relative
     st64, mse64, margin = oracle.map_rows(oracle.viterbi_f64, [s[idx]], 16)
     near = margin < NEAR_TIE
-    print(f"l16_rht1024: {int(near.sum())} near-tie sequences of {len(idx)} sampled "
-          f"(fp64 margin < {NEAR_TIE:g}); smallest fp64 margin {margin.min():.3g}")
+    print(f"l16_rht1024: near-tie sequences (margin < {NEAR_TIE:g}): GPU {int((mg < NEAR_TIE).sum())} "
+          f"of 4096 (smallest {mg.min():.3g}); fp64 oracle {int(near.sum())} of {len(idx)} sampled "
+          f"(smallest {margin.min():.3g})")
     assert np.array_equal(st[idx][~near], st64[~near])
     assert np.all(np.abs(mse[idx] - mse64) <= 2e-5 * mse64)
+    ok = ~near
+    assert np.all(np.abs(mg[idx][ok].astype(np.float64) - margin[ok]) <= _margin_bound(margin[ok], 256))
     assert abs(float(mse.mean()) - 0.065) < 0.004       # page: free-start L=16 MSE
 
 
@@ -167,10 +194,11 @@ def test_viterbi_l16_rht_block(tcq):
 @pytest.mark.parametrize("T,n", [(1, 3), (2, 5), (3, 1), (17, 9), (100, 2)])
 def test_viterbi_edge_shapes(tcq, L, T, n):
     s = W.gaussian(n, 500 + T, seq_len=T) * np.float32(1.5)
-    st, mse = _viterbi_gpu(tcq, s, L)
-    rst, rmse = oracle.viterbi_f32(s, L)
+    st, mse, mg = _viterbi_gpu(tcq, s, L, margin=True)
+    rst, rmse, rmg = oracle.viterbi_f32(s, L, margin=True)
     assert np.array_equal(st, rst)
     assert np.array_equal(mse.view(np.uint32), rmse.view(np.uint32))
+    assert _same_f32(mg, rmg)
 
 
 def test_viterbi_ties_resolve_to_lowest_index(tcq):
@@ -178,10 +206,11 @@ def test_viterbi_ties_resolve_to_lowest_index(tcq):
     s = np.zeros((9, 64), dtype=np.float32)
     s[1] = 0.25
     s[2, ::2] = -1.0
-    st, mse = _viterbi_gpu(tcq, s, 8)
-    rst, rmse = oracle.viterbi_f32(s, 8)
+    st, mse, mg = _viterbi_gpu(tcq, s, 8, margin=True)
+    rst, rmse, rmg = oracle.viterbi_f32(s, 8, margin=True)
     assert np.array_equal(st, rst)
     assert np.array_equal(mse.view(np.uint32), rmse.view(np.uint32))
+    assert _same_f32(mg, rmg)             # exact ties have no margin
 
 
 # ---------------------------------------------------------------- BCJR
@@ -278,10 +307,11 @@ def _extreme_targets(T=40):
 @pytest.mark.parametrize("L", [8, 12, 16])
 def test_viterbi_extreme_targets(tcq, L):
     s = _extreme_targets()
-    st, mse = _viterbi_gpu(tcq, s, L)
-    rst, rmse = oracle.viterbi_f32(s, L)
+    st, mse, mg = _viterbi_gpu(tcq, s, L, margin=True)
+    rst, rmse, rmg = oracle.viterbi_f32(s, L, margin=True)
     assert np.array_equal(st, rst)
     assert np.array_equal(mse.view(np.uint32), rmse.view(np.uint32))
+    assert _same_f32(mg, rmg)
 
 
 @pytest.mark.parametrize("L", [8, 12, 16])
@@ -411,9 +441,11 @@ def test_weighted_viterbi_bit_exact(tcq, L, n):
     st, mse = tcq.viterbi_encode(_dev(s), L, D=_dev(D))
     torch.cuda.synchronize()
     st = st.cpu().view(torch.int16).numpy().view(np.uint16)
-    rst, rmse = oracle.viterbi_f32(s, L, D=D)
+    rst, rmse, rmg = oracle.map_rows(oracle.viterbi_f32, [s], L, D=D, margin=True)
     assert np.array_equal(st, rst)
     assert np.array_equal(mse.cpu().numpy().view(np.uint32), rmse.view(np.uint32))
+    _, _, mg = _viterbi_gpu(tcq, s, L, margin=True, D=D)
+    assert _same_f32(mg, rmg)
 
 
 def test_weighted_full_workload(tcq):

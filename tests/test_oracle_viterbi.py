@@ -205,3 +205,86 @@ def test_pinned_ties_match_enumeration(f32):
         else:
             st, _ = oracle.viterbi_pinned_f64(s[None], L, o, code=code)
         assert st[0].tolist() == want.tolist(), (trial, o, code, s)
+
+
+# ---------------------------------------------------------------- decision margins
+def _prefix_minima(s, code, L, k, f32):
+    """P[t][p]: least energy of any walk prefix x_0..x_t ending in state p,
+    summed left to right in the given precision, by enumerating every prefix
+    (rounding is monotone, so the minimum of the rounded sums is what the
+    recursion's rounded minimum gives)."""
+    out = []
+    for t in range(len(s)):
+        walks = _walks(L, k, t + 1)
+        E = _energies(walks, s[:t + 1], code, f32)
+        P = np.full(1 << L, np.inf, dtype=np.float32 if f32 else np.float64)
+        np.minimum.at(P, walks[:, -1], E)
+        out.append(P)
+    return out
+
+
+def _margin_along(walk, P, L, k, f32):
+    dt = np.float32 if f32 else np.float64
+
+    def gap(c):
+        best = c.min()
+        above = c[c > best]
+        if above.size == 0:
+            return np.inf
+        den = best if best > dt(1e-30) else dt(1e-30)
+        return dt(dt(above.min() - best) / den)
+
+    m = gap(P[-1])                                  # the final choice among all states
+    for t in range(len(walk) - 1, 0, -1):           # the walk's choice at step t
+        preds = (walk[t] >> k) | (np.arange(1 << k) << (L - k))
+        m = min(m, gap(P[t - 1][preds]))
+    return m
+
+
+@pytest.mark.parametrize("f32", [True, False])
+def test_decision_margin_matches_enumeration(f32):
+    # QTIP blog, "The trellis: a stateful codebook": the walk is read back from
+    # the argmins; the margin of each argmin along it is (second - best)/best
+    L, k, T = 6, 2, 5
+    rng = np.random.default_rng(77 + f32)
+    code = oracle.codebook_f32(L) if f32 else oracle.codebook_f64(L)
+    for trial in range(6):
+        s = rng.standard_normal(T) * 1.3
+        if f32:
+            s = s.astype(np.float32)
+            st, _, m = oracle.viterbi_f32(s[None], L, margin=True)
+        else:
+            st, _, m = oracle.viterbi_f64(s[None], L)
+        P = _prefix_minima(s, code, L, k, f32)
+        want = _margin_along(st[0].astype(np.int64), P, L, k, f32)
+        assert m[0] == want, (trial, m[0], want)
+        assert 0 < m[0] < np.inf
+
+
+def test_decision_margin_with_ties_and_none():
+    # all-zero codebook: every decision is an exact tie, so no decision has a
+    # second distinct candidate and the margin is infinite
+    s = np.array([[0.3, -0.2, 1.5]], dtype=np.float32)
+    _, _, m = oracle.viterbi_f32(s, 4, code=np.zeros(16, np.float32), margin=True)
+    assert m[0] == np.inf
+    _, _, m = oracle.viterbi_f64(s, 4, code=np.zeros(16))
+    assert m[0] == np.inf
+    # repeated code values: ties everywhere, margins still match enumeration
+    rng = np.random.default_rng(5)
+    for trial in range(10):
+        code = rng.integers(-1, 2, 16).astype(np.float32)
+        s = rng.integers(-1, 2, 4).astype(np.float32)
+        st, _, m = oracle.viterbi_f32(s[None], 4, code=code, margin=True)
+        P = _prefix_minima(s, code, 4, 2, True)
+        assert m[0] == _margin_along(st[0].astype(np.int64), P, 4, 2, True)
+
+
+def test_fp32_margin_close_to_fp64_margin():
+    # the two differ only by the rounding of the costs: each cost carries at
+    # most T u relative error (u = 2^-24), so |m32 - m64| <= 2 (1 + m) T u + 2 u m
+    s = W.gaussian(32, 19, seq_len=128)
+    _, _, m32 = oracle.viterbi_f32(s, 8, margin=True)
+    _, _, m64 = oracle.viterbi_f64(s, 8)
+    u = 2.0 ** -24
+    bound = 2 * (1 + m64) * 128 * u + 2 * u * m64
+    assert np.all(np.abs(m32.astype(np.float64) - m64) <= bound)

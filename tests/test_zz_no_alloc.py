@@ -31,9 +31,13 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
     build()
     lib = _abi.lib()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    # two calls in a row; the second is smaller, so stale backpointers from the
-    # first call remain in the shared buffer beyond what the second one uses
-    for L, n, seed in ((12, 400, 71), (12, 150, 72), (16, 24, 73)):
+    # two calls in a row at each L; the second is smaller, so stale
+    # backpointers from the first call remain in the shared buffer beyond
+    # what the second one uses.  L = 8 runs once at the documented maximum
+    # (8,224 sequences: 8,224 x 255 x 16 bytes fill the 32 MiB buffer to
+    # within 512 bytes).
+    for L, n, seed in ((8, 8224, 70), (8, 64, 74), (12, 400, 71), (12, 150, 72), (16, 24, 73),
+                       (16, 32, 75)):
         s = torch.from_numpy(W.gaussian(n, seed)).cuda()
         ref_states, ref_mse = tcq.viterbi_encode(s, L)          # caller-workspace entry point
         states = torch.empty_like(ref_states)
@@ -47,15 +51,17 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
         assert np.array_equal(mse.cpu().numpy().view(np.uint32), ref_mse.cpu().numpy().view(np.uint32))
 
 
-def test_noalloc_rejects_requests_beyond_its_buffer():
+@pytest.mark.parametrize("L,n", [(16, 33), (16, 40), (12, 515), (8, 8225)])
+def test_noalloc_rejects_requests_beyond_its_buffer(L, n):
+    # one sequence past each documented limit (32 at L = 16, 514 at L = 12,
+    # 8,224 at L = 8) is refused on the host, before anything is launched
     assert torch.cuda.is_available(), "GPU test"
     from trellis_coded_weight_bitshift_b200 import _abi
     lib = _abi.lib()
-    n = 40                                   # 40 x 255 x 4 KiB > 32 MiB at L = 16
     s = torch.zeros((n, 256), dtype=torch.float32, device="cuda")
     states = torch.full((n, 256), 7, dtype=torch.int16, device="cuda")
     mse = torch.full((n,), -1.0, dtype=torch.float32, device="cuda")
-    tr = _abi.trellis(16, 256)
+    tr = _abi.trellis(L, 256)
     rc = lib.tcq_viterbi_encode_noalloc(ctypes.byref(tr), _p(s), n, _p(states), _p(mse),
                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == _abi.TCQ_ERR_WORKSPACE

@@ -80,10 +80,12 @@ def _weights(D: torch.Tensor | None, s: torch.Tensor) -> torch.Tensor | None:
 
 
 def viterbi_encode(s: torch.Tensor, L: int, workspace: torch.Tensor | None = None,
-                   D: torch.Tensor | None = None):
+                   D: torch.Tensor | None = None, margin: bool = False):
     """Min-MSE walk of every row of ``s`` [n, T] (fp32) on the (L, 2, 1)
-    bitshift trellis with the 1MAD code; returns (states uint16, mse fp32).
-    ``D`` (optional, same shape) weights each step's squared error."""
+    bitshift trellis with the 1MAD code; returns (states uint16, mse fp32),
+    and with ``margin=True`` also the smallest relative decision margin along
+    each walk (fp32 [n]; a second forward pass).  ``D`` (optional, same
+    shape) weights each step's squared error."""
     _require_cuda(s)
     D = _weights(D, s)
     if s.dtype != torch.float32 or s.dim() != 2:
@@ -92,11 +94,12 @@ def viterbi_encode(s: torch.Tensor, L: int, workspace: torch.Tensor | None = Non
     tr = trellis(L, T)
     states = torch.empty((n, T), dtype=torch.uint16, device=s.device)
     mse = torch.empty((n,), dtype=torch.float32, device=s.device)
+    mrg = torch.empty((n,), dtype=torch.float32, device=s.device) if margin else None
     need = int(lib().tcq_viterbi_workspace_size(ctypes.byref(tr), n))
     ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
     check(lib().tcq_viterbi_encode(ctypes.byref(tr), _ptr(s), _ptr(D), n, _ptr(states), _ptr(mse),
-                                   _ptr(ws), ws.numel(), _stream()), "tcq_viterbi_encode")
-    return states, mse
+                                   _ptr(mrg), _ptr(ws), ws.numel(), _stream()), "tcq_viterbi_encode")
+    return (states, mse, mrg) if margin else (states, mse)
 
 
 def viterbi_encode_tailbiting(s: torch.Tensor, L: int, workspace: torch.Tensor | None = None,

@@ -57,7 +57,7 @@ def lib() -> ctypes.CDLL:
     L.tcq_viterbi_workspace_size.restype = SZ
     L.tcq_viterbi_workspace_size.argtypes = [TP, I64]
     L.tcq_viterbi_encode.restype = I
-    L.tcq_viterbi_encode.argtypes = [TP, P, P, I64, P, P, P, SZ, P]
+    L.tcq_viterbi_encode.argtypes = [TP, P, P, I64, P, P, P, P, SZ, P]
     L.tcq_viterbi_encode_tailbiting.restype = I
     L.tcq_viterbi_encode_tailbiting.argtypes = [TP, P, P, I64, P, P, P, SZ, P]
     L.tcq_viterbi_encode_noalloc.restype = I

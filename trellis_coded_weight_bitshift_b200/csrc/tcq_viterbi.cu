@@ -48,10 +48,11 @@ struct VitCfg {
   static constexpr bool TMEMC = TMEMC_;
   static constexpr int TCPT = TMEMC ? ASM * G : 0;                 // TMEM columns per thread
   static constexpr int TCOLS = TCPT * (NT / 128) <= 32 ? 32 : TCPT * (NT / 128);
-  static constexpr size_t smem_bytes() {
+  // MARGIN (the decision-margin pass) also stages the walk: SPC x 256 uint16
+  static constexpr size_t smem_bytes(bool margin = false) {
     return sizeof(float) * ((size_t)SPC * NBUF * NG + (TMEMC ? 0 : (size_t)ASM * G * TPS) +
                             (size_t)SPC * 512) +
-           sizeof(unsigned long long) * NT;
+           sizeof(unsigned long long) * NT + (margin ? sizeof(uint16_t) * (size_t)SPC * 256 : 0);
   }
   static_assert(NG % G == 0 && G % 4 == 0, "bad group split");
   static_assert(!TMEMC || (SPC == 1 && NT % 128 == 0 && ASM % 2 == 0 && ASM > 0 &&
@@ -75,11 +76,33 @@ __device__ __forceinline__ void load_run(const float *base, int idx, float *dst)
   }
 }
 
-template <class C, bool WEIGHTED>
+// Relative gap of a decision, (second - best) / max(best, 1e-30), each
+// operation rounded to fp32 (costs are >= 0).
+__device__ __forceinline__ float decision_gap(float best, float second) {
+  return __fdiv_rn(__fsub_rn(second, best), fmaxf(best, 1e-30f));
+}
+
+// Fold candidate v into (best, second distinct above best).
+__device__ __forceinline__ void fold_second(float v, float &b, float &s2) {
+  if (v < b) { s2 = b; b = v; }
+  else if (v > b) s2 = fminf(s2, v);
+}
+
+// MARGIN = false: the forward recursion, backpointers, final argmin and MSE.
+// MARGIN = true (decision-margin pass, run after the traceback on the same
+// inputs): the same recursion with no backpointers or outputs except
+// margin_out[seq], the smallest relative decision margin along the walk in
+// `states` -- at step t the gap between the best and second-best distinct
+// cost_{t-1} over the four predecessors of states[t] (one thread per step
+// reads them from the cost vector in shared memory), and at the end the gap
+// between the two smallest distinct final costs.
+template <class C, bool WEIGHTED, bool MARGIN = false>
 __global__ void __launch_bounds__(C::NT, C::MINB)
 viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n_seq,
                    int T, int rot, const uint16_t *pin_states, int pin_pos,
-                   uint8_t *__restrict__ bp, uint16_t *states, float *__restrict__ mse) {
+                   uint8_t *__restrict__ bp, uint16_t *states, float *__restrict__ mse,
+                   float *__restrict__ margin_out) {
+  static_assert(!MARGIN || (C::NBUF == 2 && C::SPC <= 8), "margin pass: double buffer, <= 8 sequences");
   constexpr int NG = C::NG, G = C::G, GQ = C::GQ, TPS = C::TPS, AREG = C::AREG, ASM = C::ASM;
   constexpr int NB = C::NBUF;
   extern __shared__ __align__(16) float smem[];
@@ -88,6 +111,8 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
   float *ssm = Csm + (C::TMEMC ? 0 : ASM * G * TPS);              // [SPC][256]
   float *dsm = ssm + C::SPC * 256;                                 // [SPC][256] weights
   unsigned long long *red = reinterpret_cast<unsigned long long *>(dsm + C::SPC * 256);
+  uint16_t *wsm = reinterpret_cast<uint16_t *>(red + C::NT);         // MARGIN: [SPC][256] walk
+  __shared__ int smg[MARGIN ? C::SPC : 1];                            // MARGIN: min step gap (bits)
 
   const int tid = threadIdx.x;
   const int ls = tid / TPS, w = tid - ls * TPS;
@@ -161,7 +186,9 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
     if (tr >= T) tr -= T;
     ssm[l * 256 + t] = sq < n_seq ? s[sq * T + tr] : 0.0f;
     if (WEIGHTED) dsm[l * 256 + t] = sq < n_seq ? Dw[sq * T + tr] : 0.0f;
+    if (MARGIN) wsm[l * 256 + t] = sq < n_seq ? states[sq * T + t] : (uint16_t)0;
   }
+  if (MARGIN && tid < C::SPC) smg[tid] = 0x7f800000;                 // +inf
   // Pinned (tail-biting) run: the first state's top L-2 bits and the last
   // state's low L-2 bits must both equal the overlap o, i.e. only group o may
   // start (M_0 = 0 there, +inf elsewhere) and only states with low bits o may
@@ -266,7 +293,23 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
       *reinterpret_cast<float4 *>(Mo + swz<C::SWZ>(G * w + 4 * q)) =
           make_float4(outv[0], outv[1], outv[2], outv[3]);
     }
-    if (active) {
+    if constexpr (MARGIN) {
+      // the walk's decision at step t: its state's four predecessors p, with
+      // cost_{t-1}(p) = M_{t-1}(p >> 2) + e_{t-1}(p), rounded as in the step
+      if (active && t % TPS == w) {
+        const uint32_t q = wsm[ls * 256 + t] >> 2;
+        float b = INFINITY, s2 = INFINITY;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const uint32_t p = q | ((uint32_t)a << (C::L - 2));
+          const float d = __fsub_rn(one_mad_f32(p), sv);
+          float e = __fmul_rn(d, d);
+          if (WEIGHTED) e = __fmul_rn(e, dv);
+          fold_second(__fadd_rn(Mi[swz<C::SWZ>((int)(p >> 2))], e), b, s2);
+        }
+        if (s2 < INFINITY) atomicMin(&smg[ls], __float_as_int(decision_gap(b, s2)));
+      }
+    } else if (active) {
       uint8_t *dst = bps + (int64_t)(t - 1) * (NG / 4) + w * C::BPB;
       if constexpr (C::BPB == 1) *dst = (uint8_t)bits[0];
       else if constexpr (C::BPB == 2) *reinterpret_cast<uint16_t *>(dst) = (uint16_t)bits[0];
@@ -292,6 +335,7 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
   {
     const float sv = ssm[ls * 256 + T - 1];
     unsigned long long best = ~0ull;
+    float fb = INFINITY, fs = INFINITY;                                // MARGIN: best, second
 #pragma unroll
     for (int q = 0; q < GQ; ++q) {
       float4 csm[ASM > 0 ? ASM : 1];
@@ -315,27 +359,52 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
           const float cost = __fadd_rn(min_in[a][q], e);
           const unsigned long long key =
               ((unsigned long long)__float_as_uint(cost) << 32) | (uint32_t)(a * NG + G * w + i);
-          if (o < 0 || G * w + i == o) best = key < best ? key : best;
+          if constexpr (MARGIN) fold_second(cost, fb, fs);
+          else if (o < 0 || G * w + i == o) best = key < best ? key : best;
         }
       }
     }
-    // reduce over the sequence's TPS threads
     constexpr int WL = TPS < 32 ? TPS : 32;
+    if constexpr (MARGIN) {
+      // (best, second distinct) over the sequence's TPS threads, then the
+      // smallest gap of the walk
 #pragma unroll
-    for (int off = WL / 2; off > 0; off >>= 1) {
-      const unsigned long long o = __shfl_xor_sync(0xffffffffu, best, off);
-      best = o < best ? o : best;
-    }
-    red[tid] = best;
-    __syncthreads();
-    if (w == 0 && active) {
-      for (int x = WL; x < TPS; x += WL) {
-        const unsigned long long o = red[tid + x];
+      for (int off = WL / 2; off > 0; off >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, fb, off);
+        const float os = __shfl_xor_sync(0xffffffffu, fs, off);
+        fold_second(ob, fb, fs);
+        fs = fminf(fs, os);
+      }
+      red[tid] = ((unsigned long long)__float_as_uint(fs) << 32) | __float_as_uint(fb);
+      __syncthreads();
+      if (w == 0 && active) {
+        for (int x = WL; x < TPS; x += WL) {
+          const unsigned long long v = red[tid + x];
+          fold_second(__uint_as_float((uint32_t)v), fb, fs);
+          fs = fminf(fs, __uint_as_float((uint32_t)(v >> 32)));
+        }
+        float m = __int_as_float(smg[ls]);
+        if (fs < INFINITY) m = fminf(m, decision_gap(fb, fs));
+        margin_out[seq] = m;
+      }
+    } else {
+      // reduce over the sequence's TPS threads
+#pragma unroll
+      for (int off = WL / 2; off > 0; off >>= 1) {
+        const unsigned long long o = __shfl_xor_sync(0xffffffffu, best, off);
         best = o < best ? o : best;
       }
-      const float cost = __uint_as_float((uint32_t)(best >> 32));
-      states[seq * T + T - 1] = (uint16_t)(best & 0xffffffffu);
-      mse[seq] = __fdiv_rn(cost, (float)T);
+      red[tid] = best;
+      __syncthreads();
+      if (w == 0 && active) {
+        for (int x = WL; x < TPS; x += WL) {
+          const unsigned long long o = red[tid + x];
+          best = o < best ? o : best;
+        }
+        const float cost = __uint_as_float((uint32_t)(best >> 32));
+        states[seq * T + T - 1] = (uint16_t)(best & 0xffffffffu);
+        mse[seq] = __fdiv_rn(cost, (float)T);
+      }
     }
   }
   if constexpr (C::TMEMC) {                                // every thread is done with its lane
@@ -412,20 +481,30 @@ using Vit16 = VitCfg<16, 32, 1, 0, 2, 1, true>;
 
 size_t bp_bytes_per_seq(int L, int T) { return (size_t)(T - 1) * ((size_t)1 << (L - 4)); }
 
-template <class C, bool WEIGHTED>
+template <class C, bool WEIGHTED, bool MARGIN = false>
 tcq_status_t launch_fwd_w(const float *s, const float *D, int64_t n_seq, int T, uint8_t *bp,
                           uint16_t *states, float *mse, cudaStream_t stream, int rot,
-                          const uint16_t *pin_states, int pin_pos) {
-  const size_t smem = C::smem_bytes();
+                          const uint16_t *pin_states, int pin_pos, float *margin = nullptr) {
+  const size_t smem = C::smem_bytes(MARGIN);
   if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(viterbi_fwd_kernel<C, WEIGHTED>,
+    if (cudaFuncSetAttribute(viterbi_fwd_kernel<C, WEIGHTED, MARGIN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return TCQ_ERR_CUDA;
   }
   const int64_t blocks = (n_seq + C::SPC - 1) / C::SPC;
-  viterbi_fwd_kernel<C, WEIGHTED><<<(unsigned)blocks, C::NT, smem, stream>>>(
-      s, D, n_seq, T, rot, pin_states, pin_pos, bp, states, mse);
+  viterbi_fwd_kernel<C, WEIGHTED, MARGIN><<<(unsigned)blocks, C::NT, smem, stream>>>(
+      s, D, n_seq, T, rot, pin_states, pin_pos, bp, states, mse, margin);
   return launch_status();
+}
+
+// Decision-margin pass over finished walks (states holds the walks).
+template <class C>
+tcq_status_t launch_margin(const float *s, const float *D, int64_t n_seq, int T, uint8_t *bp,
+                           uint16_t *states, float *margin, cudaStream_t stream) {
+  return D ? launch_fwd_w<C, true, true>(s, D, n_seq, T, bp, states, nullptr, stream, 0, nullptr, 0,
+                                         margin)
+           : launch_fwd_w<C, false, true>(s, nullptr, n_seq, T, bp, states, nullptr, stream, 0,
+                                          nullptr, 0, margin);
 }
 
 template <class C>
@@ -470,13 +549,14 @@ extern "C" size_t tcq_viterbi_workspace_size(const tcq_trellis_t *tr, int64_t n_
 
 extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float *s,
                                            const float *D, int64_t n_seq, uint16_t *states,
-                                           float *mse, void *ws, size_t ws_bytes, void *stream) {
+                                           float *mse, float *min_margin, void *ws,
+                                           size_t ws_bytes, void *stream) {
   tcq_status_t st = check_trellis(tr);
   if (st != TCQ_OK) return st;
   if (n_seq < 0 || n_seq > (int64_t)INT32_MAX * 8) return TCQ_ERR_INVALID_ARG;
   if (n_seq == 0) return TCQ_OK;
   if (!s || !states || !mse || !aligned16(s) || !aligned16(states) || !aligned16(mse) ||
-      (D && !aligned16(D)))
+      (D && !aligned16(D)) || (min_margin && !aligned16(min_margin)))
     return TCQ_ERR_INVALID_ARG;
   const size_t need = tcq_viterbi_workspace_size(tr, n_seq);
   if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TCQ_ERR_WORKSPACE;
@@ -488,8 +568,14 @@ extern "C" tcq_status_t tcq_viterbi_encode(const tcq_trellis_t *tr, const float 
     case 12: st = launch_fwd<Vit12>(s, n_seq, T, bp, states, mse, strm, D); break;
     default: st = launch_fwd<Vit16>(s, n_seq, T, bp, states, mse, strm, D); break;
   }
-  if (st != TCQ_OK || T == 1) return st;
-  return launch_traceback(tr->L, bp, n_seq, T, states, strm);
+  if (st != TCQ_OK) return st;
+  if (T > 1 && (st = launch_traceback(tr->L, bp, n_seq, T, states, strm)) != TCQ_OK) return st;
+  if (!min_margin) return TCQ_OK;
+  switch (tr->L) {
+    case 8: return launch_margin<Vit8>(s, D, n_seq, T, bp, states, min_margin, strm);
+    case 12: return launch_margin<Vit12>(s, D, n_seq, T, bp, states, min_margin, strm);
+    default: return launch_margin<Vit16>(s, D, n_seq, T, bp, states, min_margin, strm);
+  }
 }
 
 // Tail-biting encode [QTIP blog, "Tail-biting is worth its complexity"]: two
@@ -548,8 +634,13 @@ extern "C" tcq_status_t tcq_viterbi_encode_tailbiting(const tcq_trellis_t *tr, c
 // The buffer below is a host-side symbol as far as host code is concerned:
 // its address on the device must be fetched with cudaGetSymbolAddress, with
 // the device current, before it can be passed to a kernel.  That is done once
-// per device, by the first call on that device, and cached.
-#include <atomic>
+// per device context, by the first call in it, and cached.  The cache is keyed
+// on the context's unique id as well as the device ordinal: cudaDeviceReset
+// destroys the device's primary context, the library's module is loaded again
+// in the next one and the buffer may then sit at another address.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 namespace {
@@ -557,8 +648,35 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB per device
 constexpr int kNoAllocMaxDevices = 64;
 
-std::atomic<uint8_t *> g_noalloc_scratch_ptr[kNoAllocMaxDevices];
+struct NoAllocSlot {
+  uint8_t *ptr = nullptr;
+  unsigned long long ctx_id = 0;      // unique id of the context ptr belongs to
+};
+NoAllocSlot g_noalloc_slot[kNoAllocMaxDevices];
 std::mutex g_noalloc_mutex;
+
+// Unique id of the calling thread's current context, through the driver entry
+// points the runtime hands out (no link-time dependency on the driver
+// library); false if there is no current context or the query fails.
+bool current_context_id(unsigned long long *id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 }  // namespace
 
@@ -568,19 +686,20 @@ static tcq_status_t noalloc_scratch_for_current_device(uint8_t **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return TCQ_ERR_CUDA;
   if (dev < 0 || dev >= kNoAllocMaxDevices) return TCQ_ERR_UNSUPPORTED;
-  uint8_t *p = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    p = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
-    if (p == nullptr) {
-      void *addr = nullptr;
-      if (cudaGetSymbolAddress(&addr, tcq_noalloc_scratch) != cudaSuccess || addr == nullptr)
-        return TCQ_ERR_CUDA;
-      p = static_cast<uint8_t *>(addr);
-      g_noalloc_scratch_ptr[dev].store(p, std::memory_order_release);
-    }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  NoAllocSlot &slot = g_noalloc_slot[dev];
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  if (slot.ptr == nullptr || !have_id || id != slot.ctx_id) {
+    void *addr = nullptr;          // also makes the device's primary context current
+    if (cudaGetSymbolAddress(&addr, tcq_noalloc_scratch) != cudaSuccess || addr == nullptr)
+      return TCQ_ERR_CUDA;
+    slot.ptr = static_cast<uint8_t *>(addr);
+    // the id of the context the address was looked up in (0 = unknown: the
+    // next call looks it up again)
+    slot.ctx_id = current_context_id(&id) ? id : 0;
   }
-  *out = p;
+  *out = slot.ptr;
   return TCQ_OK;
 }
 
