@@ -906,9 +906,11 @@ using Soft12 = BcjrCfg<12, 8, 7, 0, 2, false, 1>;
 using Soft16 = BcjrCfg<16, 32, 1, 0, 2, false, 1, true>;
 using Grad8 = BcjrCfg<8, 4, 8, 4, 2, true>;
 using Grad12 = BcjrCfg<12, 8, 7, 0, 2, true, 1>;
-// L = 16 gradient: code values in tensor memory as in the soft pass; the two
-// carried vectors (A and Phi, 2 x 64 KiB) fit the shared memory only
-// single-buffered, so each step takes two barriers.
+// L = 16 gradient: code values in tensor memory as in the soft pass.  The
+// message vector (A forward, B backward) is double-buffered and read block by
+// block after the step's first barrier; the expectation vector (Phi, Psi) fits
+// only once beside it (192 KiB in all), so it is read ahead of that barrier
+// and each step takes two.
 using Grad16 = BcjrCfg<16, 32, 1, 0, 1, true, 1, true, true>;
 
 template <class C>
