@@ -164,7 +164,16 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
   }
   // code values of digits AREG.. at group block q, from tensor or shared memory
   auto load_csm = [&](int q, float4 (&csm)[ASM > 0 ? ASM : 1]) {
-    if constexpr (C::TMEMC) {
+    if constexpr (C::TMEMC && ASM == 4) {
+      // the block's four digits are 16 consecutive columns: one load, one wait
+      // (L = 16 block of 4,096 sequences: 11.99 -> 11.91 ms)
+      float r16[16];
+      tmem_ld16(taddr + (uint32_t)(q * ASM * 4), r16);
+      tmem_wait_ld();
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+        csm[a & (ASM > 0 ? ASM - 1 : 0)] = make_float4(r16[4 * a], r16[4 * a + 1], r16[4 * a + 2], r16[4 * a + 3]);
+    } else if constexpr (C::TMEMC) {
 #pragma unroll
       for (int a = 0; a < ASM; a += 2) {
         float r8[8];
