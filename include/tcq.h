@@ -191,7 +191,11 @@ TCQ_API tcq_status_t tcq_viterbi_encode_noalloc(const tcq_trellis_t *trellis, co
  *   E(x) = sum_t (code(x_t) - s_t)^2
  * and probability exp(-E/temp)/Z over all walks (free start, free end):
  *   soft[t] = E_p[code(x_t)],   log_z = log Z (natural log).
- * fp32, log domain (base 2 inside), renormalised every step.
+ * fp32, log domain (base 2 inside), renormalised every step.  At a step
+ * whose target lies outside the code range, the emissions are taken relative
+ * to the nearest code bound r: (code - r)(code - (2 s - r)) differs from
+ * (code - s)^2 by a constant of the step, which cancels in every expectation
+ * and is added back to log Z in fp64.
  *
  *   s        [n_seq][seq_len] fp32 (input); temp > 0 and finite.
  *   D        [n_seq][seq_len] fp32 curvature weights (>= 0) or NULL: the
@@ -232,7 +236,9 @@ TCQ_API tcq_status_t tcq_bcjr_soft_backward(const tcq_trellis_t *trellis, const 
  * know the cotangent up front (e.g. the gradient of a fixed loss): one
  * forward-backward sweep yields soft, log Z and grad_s, where the two
  * separate calls take two sweeps.  The covariance is centred at the targets
- * s instead of the soft codeword (an exact identity; only rounding differs).
+ * clamped to the code range instead of at the soft codeword (an exact
+ * identity; only rounding differs, and the clamp keeps it small for targets
+ * far outside the range).
  *   grad_soft [n_seq][seq_len] (input); soft, log_z (outputs, each may be
  *   NULL); grad_s (output).  Workspace: tcq_bcjr_workspace_size(.., 1).
  * ------------------------------------------------------------------------ */

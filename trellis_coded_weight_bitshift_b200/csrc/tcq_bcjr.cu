@@ -36,12 +36,15 @@
 //
 // Gradient (GRAD = true): d soft_t / d s_u = (2/temp) Cov(code(x_t), code(x_u)),
 // so grad_u = (2/temp) Cov(F, code(x_u)) with F = sum_t v_t (code(x_t) - soft_t)
-// (centred by the forward soft codeword).  E[F | x_u = j] splits by the Markov
+// (centred by the forward soft codeword when it is given, else by the target
+// clamped to the code range: any per-step constant leaves the covariance
+// unchanged, and a centre near the codes keeps F small).  E[F | x_u = j] splits by the Markov
 // property into a prefix part phi (forward expectation recursion, weights =
 // the forward softmax over predecessors) and a suffix part psi (backward
 // recursion, weights = the backward softmax over successors); both reuse the
 // exponentials of the log-sum-exps above.
 #include <algorithm>
+#include <mutex>
 
 #include "tcq_device.cuh"
 
@@ -292,7 +295,7 @@ __device__ __forceinline__ void write_sub(float *vec, int base, const float *src
 template <class C>
 __global__ void __launch_bounds__(C::NT, C::MINB)
 bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n_seq, int T,
-            float kappa, float two_over_temp,
+            float kappa, float two_over_temp, float cmin, float cmax_code,
             const float *__restrict__ vgrad, const float *__restrict__ soft_in,
             float *__restrict__ soft_out, float *__restrict__ logz_out,
             float *__restrict__ grad_out, float *__restrict__ ws) {
@@ -371,9 +374,12 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     ksm[l * 256 + t] = kappa * ((ok && Dw) ? Dw[sq * T + t] : 1.0f);
     if (GRAD) {
       vsm[l * 256 + t] = ok ? vgrad[sq * T + t] : 0.0f;
-      // centre of the covariance: the forward soft codeword when given,
-      // else the targets themselves (any per-step constant is exact)
-      fsm[l * 256 + t] = ok ? (soft_in ? soft_in[sq * T + t] : s[sq * T + t]) : 0.0f;
+      // centre of the covariance (any per-step constant is exact): the
+      // forward soft codeword when given, else the target clamped to the
+      // code range, which keeps F small for targets far outside it
+      fsm[l * 256 + t] = ok ? (soft_in ? soft_in[sq * T + t]
+                                       : fminf(fmaxf(s[sq * T + t], cmin), cmax_code))
+                            : 0.0f;
     }
   };
   for (int64_t base = (int64_t)blockIdx.x * SPC; base < n_seq; base += (int64_t)gridDim.x * SPC) {
@@ -462,8 +468,18 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       const float vv = GRAD ? vsm[ls * 256 + t - 1] : 0.0f;
       const float fv = GRAD ? fsm[ls * 256 + t - 1] : 0.0f;
       float tmax = -INFINITY;
-      const f2_t sv2 = f2(sv, sv), cm2 = f2(cmax, cmax);
+      // emissions relative to r, the target clamped to the code range:
+      // -kappa (c - s)^2 = d (-kappa d + beta) - kappa (r - s)^2 with d = c - r,
+      // beta = 2 kappa (s - r).  The last term is the same for every state of
+      // the step (posteriors unchanged; log Z gets it back), and for a target
+      // inside the range r = s, beta = +0 and the two FMAs round exactly like
+      // the plain -kappa d d.  Outside it the states that compete carry small,
+      // accurately rounded emissions.
+      const float rv = fminf(fmaxf(sv, cmin), cmax_code);
+      const f2_t sv2 = f2(rv, rv), cm2 = f2(cmax, cmax);
       const f2_t nk2 = f2(-ksm[ls * 256 + t - 1], -ksm[ls * 256 + t - 1]);
+      const float beta = 2.0f * ksm[ls * 256 + t - 1] * (sv - rv);
+      const f2_t b2 = f2(beta, beta);
       if constexpr (!GRAD) {
         // code pairs of group block q + 1 are loaded from tensor memory while
         // block q computes; the wait at the end of block q completes them
@@ -509,8 +525,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           for (int r = 0; r < 4; ++r) {
             const f2_t d0 = f2sub(cq0[r], sv2);
             const f2_t d1 = f2sub(cq1[r], sv2);
-            const f2_t x0 = f2fma(f2mul(d0, nk2), d0, am0);
-            const f2_t x1 = f2fma(f2mul(d1, nk2), d1, am1);
+            const f2_t x0 = f2fma(d0, f2fma(nk2, d0, b2), am0);
+            const f2_t x1 = f2fma(d1, f2fma(nk2, d1, b2), am1);
             outA[r] = lse4_base2(f2lo(x0), f2hi(x0), f2lo(x1), f2hi(x1));
             tmax = fmaxf(tmax, outA[r]);
           }
@@ -544,8 +560,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
             const f2_t c0 = cq0[r];
             const f2_t c1 = cq1[r];
             const f2_t d0 = f2sub(c0, sv2), d1 = f2sub(c1, sv2);
-            const f2_t x0 = f2fma(f2mul(d0, nk2), d0, am0);
-            const f2_t x1 = f2fma(f2mul(d1, nk2), d1, am1);
+            const f2_t x0 = f2fma(d0, f2fma(nk2, d0, b2), am0);
+            const f2_t x1 = f2fma(d1, f2fma(nk2, d1, b2), am1);
             const f2_t z0 = f2fma(vv2, c0, ph0);            // phi_{t-1}(p) = Phi + v (c - soft)
             const f2_t z1 = f2fma(vv2, c1, ph1);
             const float mx = fmaxf(fmaxf(f2lo(x0), f2hi(x0)), fmaxf(f2lo(x1), f2hi(x1)));
@@ -598,6 +614,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     float log2Z, log2Zrel;
     {
       const float sT = ssm[ls * 256 + T - 1];
+      const float rT = fminf(fmaxf(sT, cmin), cmax_code);          // as in the forward
+      const float bT = 2.0f * ksm[ls * 256 + T - 1] * (sT - rT);
       float vals[4][GQ], vmax = -INFINITY;
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
@@ -617,8 +635,8 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
           codes.template pairs<4>(a >> 1, 4 * k, cp);
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
-            const float d = ((a & 1) ? f2hi(cp[b]) : f2lo(cp[b])) - sT;
-            y[b] = -ksm[ls * 256 + T - 1] * d * d;
+            const float d = ((a & 1) ? f2hi(cp[b]) : f2lo(cp[b])) - rT;
+            y[b] = fmaf(-ksm[ls * 256 + T - 1], d, bT) * d;
           }
           const float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
           const float S = ex2(y[0] - mx) + ex2(y[1] - mx) + ex2(y[2] - mx) + ex2(y[3] - mx);
@@ -647,7 +665,17 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       log2Zrel = vmax + lg2(tot) + cmax;                  // log2 Z - CA_{T-1}
       log2Z = log2Zrel + CA;
     }
-    if (w == 0 && active && logz_out) logz_out[seq] = log2Z * 0.69314718055994531f;
+    if (w == 0 && active && logz_out) {
+      // add back kappa D_u (r_u - s_u)^2, removed from every walk's log2
+      // weight at the steps whose target lies outside the code range
+      double removed = 0.0;
+      for (int u = 0; u < T; ++u) {
+        const float su = ssm[ls * 256 + u];
+        const double e = (double)fminf(fmaxf(su, cmin), cmax_code) - (double)su;
+        removed += (double)ksm[ls * 256 + u] * e * e;
+      }
+      logz_out[seq] = (float)(((double)log2Z - removed) * 0.69314718055994531);
+    }
 
     // ---------------- backward + combine ----------------
     // B_t is stored relative to DB_t (sum of the maxima removed); the combine
@@ -722,13 +750,16 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       if (NB == 1) seq_sync<C>(ls);
       const float K = Krun;
       Krun += cah[ls * 256 + tc] - dprev;
-      const float sv = ssm[ls * 256 + tc];
+      const float s_tc = ssm[ls * 256 + tc];
+      const float sv = fminf(fmaxf(s_tc, cmin), cmax_code);          // r, as in the forward
       const float vv = GRAD ? vsm[ls * 256 + tc] : 0.0f;
       const float fv = GRAD ? fsm[ls * 256 + tc] : 0.0f;
       float *Bo = C::MSG2 ? msg_buf(t) : Bv + ((t + NB) % NB) * NV * NG;
       float *Po = C::MSG2 ? exp_buf(t) : Bo + NG;
       float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f, tmax = -INFINITY;
       const f2_t sv2 = f2(sv, sv), nk2 = f2(-ksm[ls * 256 + tc], -ksm[ls * 256 + tc]);
+      const float beta = 2.0f * ksm[ls * 256 + tc] * (s_tc - sv);
+      const f2_t b2 = f2(beta, beta);
       const f2_t K2 = f2(K, K), dp2 = f2(dprev, dprev), vv2 = f2(vv, vv);
       f2_t num2 = f2(0.0f, 0.0f), den2 = num2, n12 = num2, n22 = num2;
       // KB values of this thread's spilled vector at flat index f (KB | f)
@@ -788,7 +819,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
               const f2_t d = f2sub(cc[b], sv2);
-              y[b] = f2fma(f2mul(d, nk2), d, f2(bk[b], bk[b]));
+              y[b] = f2fma(d, f2fma(nk2, d, b2), f2(bk[b], bk[b]));
             }
             const float mxl = fmaxf(fmaxf(f2lo(y[0]), f2lo(y[1])), fmaxf(f2lo(y[2]), f2lo(y[3])));
             const float mxh = fmaxf(fmaxf(f2hi(y[0]), f2hi(y[1])), fmaxf(f2hi(y[2]), f2hi(y[3])));
@@ -938,6 +969,27 @@ using Grad12 = BcjrCfg<12, 8, 7, 0, 2, true, 1>;
 // and each step takes two.
 using Grad16 = BcjrCfg<16, 32, 1, 0, 1, true, 1, true, true>;
 
+// Smallest and largest fp32 code value of the 2^L states (the same fp64
+// division rounded once to fp32 as the kernels' code values), once per L.
+void code_bounds(int L, float *lo, float *hi) {
+  static float cache[17][2];
+  static std::once_flag once[17];
+  std::call_once(once[L], [L] {
+    float mn = INFINITY, mx = -INFINITY;
+    for (uint32_t x = 0; x < (1u << L); ++x) {
+      const uint32_t y = x * kLcgMul + kLcgAdd;
+      const int bs = (int)(y & 255u) + (int)((y >> 8) & 255u) + (int)((y >> 16) & 255u) + (int)(y >> 24);
+      const float v = (float)((double)(bs - 510) / 147.8);
+      mn = std::min(mn, v);
+      mx = std::max(mx, v);
+    }
+    cache[L][0] = mn;
+    cache[L][1] = mx;
+  });
+  *lo = cache[L][0];
+  *hi = cache[L][1];
+}
+
 template <class C>
 int grid_for(int64_t n_seq) {
   int dev = 0, per_sm = 0;
@@ -974,7 +1026,9 @@ tcq_status_t launch(const float *s, const float *D, int64_t n_seq, int T, float 
   const int grid = grid_for<C>(n_seq);
   const size_t need = (size_t)grid * C::SPC * C::ws_floats_per_slot(T) * sizeof(float);
   if (ws_bytes < need) return TCQ_ERR_WORKSPACE;
-  bcjr_kernel<C><<<grid, C::NT, C::smem_bytes(), stream>>>(s, D, n_seq, T, kappa, two_over_temp, v,
+  float cmin, cmax;
+  code_bounds(C::L, &cmin, &cmax);
+  bcjr_kernel<C><<<grid, C::NT, C::smem_bytes(), stream>>>(s, D, n_seq, T, kappa, two_over_temp, cmin, cmax, v,
                                                            soft_in, soft, logz, grad,
                                                            static_cast<float *>(ws));
   return launch_status();
