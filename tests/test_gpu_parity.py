@@ -706,8 +706,10 @@ def _gemv_ref(bits, rows, cols, x, L=16, layout=0, tile_rows=None):
     return np.concatenate(ys), np.concatenate(bs)
 
 
-@pytest.mark.parametrize("L,layout,rows,cols", [(16, 0, 256, 512), (8, 1, 96, 160), (12, 0, 1024, 2048)])
+@pytest.mark.parametrize("L,layout,rows,cols", [(16, 0, 256, 512), (8, 1, 96, 160), (12, 0, 1024, 2048),
+                                             (12, 1, 32, 16400)])
 def test_decode_gemv_matches_oracle(tcq, L, layout, rows, cols):
+    # 16400 columns: a row of 1,025 tiles, split into runs that do not divide it
     rng = np.random.default_rng(rows + cols + L)
     n = (rows // 16) * (cols // 16)
     nw = oracle.stream_words(L, 2, 256, layout)

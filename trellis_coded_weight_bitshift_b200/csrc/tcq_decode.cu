@@ -230,71 +230,22 @@ extern "C" tcq_status_t tcq_decode(const tcq_trellis_t *tr, const uint32_t *bits
 //   y[i] = sum_j W[i][j] x[j],  W = the fp16 matrix tcq_decode (TILE16) gives,
 // accumulated in fp32.  A warp takes a run of tile-columns along two
 // tile-rows; each lane owns one row of one of them and decodes that row's 16
-// weights in every tile of the run, rounds them to fp16 exactly as the decode
-// does and multiplies by x; the stream words of the next tile are loaded while
-// the current one decodes.  Runs combine by one fp32 atomic add per row into y
-// (zeroed first on the same stream).
+// weights in every tile of the run and multiplies them by x; the stream words
+// of the next tile are loaded while the current one decodes.  Runs combine by
+// one fp32 atomic add per row into y (zeroed first on the same stream).
+//
+// The fp16 code of a weight depends only on the byte sum of its LCG output
+// (1,021 values), so each CTA first fills a shared-memory table of the 1,021
+// fp16 codes (held as fp32, the value the product multiplies), one copy per
+// lane: entry (bs, lane) at float index 32 bs + lane, so a warp's 32 lookups
+// fall in 32 different banks whatever the byte sums are.  One IDP4A with byte
+// weights 128 and accumulator 4 lane gives the entry's byte offset straight
+// from the LCG output.  Products are paired per lane (even and odd weights of
+// the row) and summed in fp32.  One 1024-thread CTA per SM (the table takes
+// 130,688 bytes).  Measured and not kept: x staged in shared memory beside the
+// table (2.1 M more warp instructions, 2 us slower on 8192 x 8192).
 namespace tcq {
 
-template <int L, int LAYOUT>
-__global__ void __launch_bounds__(256) decode_gemv_kernel(const uint32_t *__restrict__ bits,
-                                                          int n_tr, int n_tc, int runs, int wps,
-                                                          const float *__restrict__ x,
-                                                          float *__restrict__ y) {
-  // lane l: tile-row 2*pair + (l >> 4), row r = l & 15 of it; the lane decodes
-  // the 16 weights of its row in every tile of the warp's run and owns y[row]
-  const int lane = threadIdx.x & 31;
-  const int r = lane & 15, half = lane >> 4;
-  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  const int n_pairs = (n_tr + 1) >> 1;
-  const int per_run = (n_tc + runs - 1) / runs;
-  for (int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       wid < (int64_t)n_pairs * runs; wid += warps) {
-    const int pair = (int)(wid / runs), run = (int)(wid - (int64_t)pair * runs);
-    const int tr = min(2 * pair + half, n_tr - 1);
-    const bool owner = 2 * pair + half < n_tr;
-    const int c0 = run * per_run, c1 = min(n_tc, c0 + per_run);
-    if (c0 >= c1) continue;
-    const uint32_t *row_src = bits + (int64_t)tr * n_tc * wps + r;
-    const int r1 = LAYOUT == TCQ_TAILBITING ? (((r + 1) & 15) - r) : 1;   // offset of word r+1
-    uint32_t nw0 = __ldg(row_src + (int64_t)c0 * wps), nw1 = __ldg(row_src + (int64_t)c0 * wps + r1);
-    float acc = 0.0f;
-    for (int tc = c0; tc < c1; ++tc) {
-      const uint32_t w0 = nw0, w1 = nw1;
-      if (tc + 1 < c1) {                               // next tile's words, one tile ahead
-        nw0 = __ldg(row_src + (int64_t)(tc + 1) * wps);
-        nw1 = __ldg(row_src + (int64_t)(tc + 1) * wps + r1);
-      }
-      const float4 *xq = reinterpret_cast<const float4 *>(x + tc * 16);
-      const float4 x0 = __ldg(xq), x1 = __ldg(xq + 1), x2 = __ldg(xq + 2), x3 = __ldg(xq + 3);
-      const float xv[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
-                            x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {                    // weights 2j, 2j+1 of the row
-        const unsigned long long c2 = one_mad_decode_f32x2(window_at<L>(w0, w1, 4 * j),
-                                                           window_at<L>(w0, w1, 4 * j + 2));
-        const __half2 hw = __floats2half2_rn(__uint_as_float((uint32_t)c2),
-                                             __uint_as_float((uint32_t)(c2 >> 32)));
-        const float2 wf = __half22float2(hw);
-        acc = fmaf(wf.x, xv[2 * j], acc);
-        acc = fmaf(wf.y, xv[2 * j + 1], acc);
-      }
-    }
-    if (owner) atomicAdd(y + (int64_t)tr * 16 + r, acc);
-  }
-}
-
-// Table form of the same product.  The fp16 code of a weight depends only on
-// the byte sum of its LCG output (1,021 values), so each CTA first fills a
-// shared-memory table of the 1,021 fp16 codes (held as fp32, the value the
-// product multiplies), one copy per lane: entry (bs, lane) at float index
-// 32 bs + lane, so a warp's 32 lookups fall in 32 different banks whatever the
-// byte sums are.  One IDP4A with byte weights 128 and accumulator 4 lane gives
-// the entry's byte offset straight from the LCG output, and replaces the
-// centring, scaling, fp16 rounding and conversion back of the arithmetic form.
-// Products are paired per lane (even and odd weights of the row) and summed
-// in fp32.  One 1024-thread CTA per SM (the table takes 130,688 bytes); the
-// warps walk the same (tile-row pair, run) items as the arithmetic form.
 constexpr int kGemvLutRows = 1021;
 
 template <int L, int LAYOUT>
@@ -303,12 +254,17 @@ __global__ void __launch_bounds__(1024, 1) decode_gemv_lut_kernel(const uint32_t
                                                                   const float *__restrict__ x,
                                                                   float *__restrict__ y) {
   extern __shared__ __align__(16) float lut[];           // [1021][32]
-  for (int e = threadIdx.x; e < kGemvLutRows * 32; e += blockDim.x) {
-    const float centred = (float)((e >> 5) - 510);
-    lut[e] = __half2float(__float2half_rn(__fmul_rn(centred, 0x1.bb68f6p-8f)));
+  const int lane = threadIdx.x & 31;
+  // thread e computes entry e once and stores its 32 copies as eight 16-byte
+  // chunks, starting at chunk (lane mod 8) so that a warp's stores spread over
+  // all banks
+  for (int e = threadIdx.x; e < kGemvLutRows; e += blockDim.x) {
+    const float v = __half2float(__float2half_rn(__fmul_rn((float)(e - 510), 0x1.bb68f6p-8f)));
+    float4 *dst = reinterpret_cast<float4 *>(lut + e * 32);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) dst[(q + lane) & 7] = make_float4(v, v, v, v);
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
   const int r = lane & 15, half = lane >> 4;
   const uint32_t lane_off = 4u * (uint32_t)lane;
   const char *lut_b = reinterpret_cast<const char *>(lut);
@@ -349,6 +305,24 @@ __global__ void __launch_bounds__(1024, 1) decode_gemv_lut_kernel(const uint32_t
   }
 }
 
+template <int L, int LAYOUT>
+tcq_status_t gemv_launch(const uint32_t *bits, int n_tr, int n_tc, int wps, const float *x, float *y,
+                         cudaStream_t s) {
+  const size_t smem = sizeof(float) * (size_t)kGemvLutRows * 32;
+  if (cudaFuncSetAttribute(decode_gemv_lut_kernel<L, LAYOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return TCQ_ERR_CUDA;
+  // each warp a run of tiles along a tile-row pair, runs per pair chosen so
+  // that every resident warp has work
+  const int64_t n_pairs = (n_tr + 1) / 2;
+  const int64_t resident_warps = (int64_t)sm_count() * 32;
+  const int runs = (int)std::max<int64_t>(1, std::min<int64_t>(n_tc, resident_warps / n_pairs));
+  const int64_t warps = n_pairs * runs;
+  const unsigned blocks = (unsigned)std::min<int64_t>((warps + 31) / 32, (int64_t)sm_count());
+  decode_gemv_lut_kernel<L, LAYOUT><<<blocks, 1024, smem, s>>>(bits, n_tr, n_tc, runs, wps, x, y);
+  return launch_status();
+}
+
 }  // namespace tcq
 
 extern "C" tcq_status_t tcq_decode_gemv(const tcq_trellis_t *tr, const uint32_t *bits, int layout,
@@ -367,72 +341,13 @@ extern "C" tcq_status_t tcq_decode_gemv(const tcq_trellis_t *tr, const uint32_t 
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(y, 0, sizeof(float) * (size_t)rows, s) != cudaSuccess) return TCQ_ERR_CUDA;
   const int n_tr = (int)(rows / 16), n_tc = (int)(cols / 16);
-  {
-    // table form: one 1024-thread CTA per SM, each warp a run of tiles along a
-    // tile-row pair (runs per pair chosen so that every warp has work)
-    const size_t smem = sizeof(float) * kGemvLutRows * 32;
-    const void *fn = nullptr;
-    switch (tr->L) {
-      case 8: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_lut_kernel<8, TCQ_TAILBITING>
-                                            : (const void *)decode_gemv_lut_kernel<8, TCQ_FREE_START>; break;
-      case 12: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_lut_kernel<12, TCQ_TAILBITING>
-                                             : (const void *)decode_gemv_lut_kernel<12, TCQ_FREE_START>; break;
-      default: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_lut_kernel<16, TCQ_TAILBITING>
-                                             : (const void *)decode_gemv_lut_kernel<16, TCQ_FREE_START>; break;
-    }
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return TCQ_ERR_CUDA;
-    const int64_t n_pairs = (n_tr + 1) / 2;
-    const int64_t resident_warps = (int64_t)sm_count() * 32;
-    const int runs = (int)std::max<int64_t>(1, std::min<int64_t>(n_tc, resident_warps / n_pairs));
-    const int64_t warps = n_pairs * runs;
-    const unsigned blocks = (unsigned)std::min<int64_t>((warps + 31) / 32, (int64_t)sm_count());
-#define TCQ_GEMV_LUT(LL)                                                                            \
-  (layout == TCQ_TAILBITING                                                                         \
-       ? decode_gemv_lut_kernel<LL, TCQ_TAILBITING><<<blocks, 1024, smem, s>>>(bits, n_tr, n_tc, runs, \
-                                                                               (int)wps, x, y)        \
-       : decode_gemv_lut_kernel<LL, TCQ_FREE_START><<<blocks, 1024, smem, s>>>(bits, n_tr, n_tc, runs, \
-                                                                               (int)wps, x, y))
-    switch (tr->L) {
-      case 8: TCQ_GEMV_LUT(8); break;
-      case 12: TCQ_GEMV_LUT(12); break;
-      default: TCQ_GEMV_LUT(16); break;
-    }
-#undef TCQ_GEMV_LUT
-    return launch_status();
-  }
-  // One wave: as many warps as can be resident, each a run of tiles along a
-  // tile-row (runs per tile-row chosen so that all runs fit at once).
-  int per_sm = 0;
-  {
-    const void *fn = nullptr;
-    switch (tr->L) {
-      case 8: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_kernel<8, TCQ_TAILBITING>
-                                            : (const void *)decode_gemv_kernel<8, TCQ_FREE_START>; break;
-      case 12: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_kernel<12, TCQ_TAILBITING>
-                                             : (const void *)decode_gemv_kernel<12, TCQ_FREE_START>; break;
-      default: fn = layout == TCQ_TAILBITING ? (const void *)decode_gemv_kernel<16, TCQ_TAILBITING>
-                                             : (const void *)decode_gemv_kernel<16, TCQ_FREE_START>; break;
-    }
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 256, 0) != cudaSuccess || per_sm < 1)
-      per_sm = 1;
-  }
-  const int64_t resident_warps = (int64_t)sm_count() * per_sm * 8;
-  const int64_t n_pairs = (n_tr + 1) / 2;
-  const int runs = (int)std::max<int64_t>(1, std::min<int64_t>(n_tc, resident_warps / n_pairs));
-  const int64_t warps = n_pairs * runs;
-  const unsigned blocks = (unsigned)((warps + 7) / 8);
-#define TCQ_GEMV(LL)                                                                          \
-  (layout == TCQ_TAILBITING                                                                   \
-       ? decode_gemv_kernel<LL, TCQ_TAILBITING><<<blocks, 256, 0, s>>>(bits, n_tr, n_tc, runs, \
-                                                                        (int)wps, x, y)        \
-       : decode_gemv_kernel<LL, TCQ_FREE_START><<<blocks, 256, 0, s>>>(bits, n_tr, n_tc, runs, \
-                                                                        (int)wps, x, y))
+  const bool tb = layout == TCQ_TAILBITING;
   switch (tr->L) {
-    case 8: TCQ_GEMV(8); break;
-    case 12: TCQ_GEMV(12); break;
-    default: TCQ_GEMV(16); break;
+    case 8: return tb ? gemv_launch<8, TCQ_TAILBITING>(bits, n_tr, n_tc, (int)wps, x, y, s)
+                      : gemv_launch<8, TCQ_FREE_START>(bits, n_tr, n_tc, (int)wps, x, y, s);
+    case 12: return tb ? gemv_launch<12, TCQ_TAILBITING>(bits, n_tr, n_tc, (int)wps, x, y, s)
+                       : gemv_launch<12, TCQ_FREE_START>(bits, n_tr, n_tc, (int)wps, x, y, s);
+    default: return tb ? gemv_launch<16, TCQ_TAILBITING>(bits, n_tr, n_tc, (int)wps, x, y, s)
+                       : gemv_launch<16, TCQ_FREE_START>(bits, n_tr, n_tc, (int)wps, x, y, s);
   }
-#undef TCQ_GEMV
-  return launch_status();
 }
