@@ -569,6 +569,31 @@ def test_weighted_bcjr(tcq, L):
     assert np.all(np.abs(lz - rlz) <= 1e-5 * np.abs(rlz) + 1e-4)
 
 
+@pytest.mark.parametrize("L", [12, 16])
+@pytest.mark.parametrize("temp", [0.1, 1e-2])
+def test_weighted_bcjr_outliers(tcq, L, temp):
+    # curvature weights on rows with outliers far outside the code range: the
+    # removed per-step terms kappa D_u (r_u - s_u)^2 carry the weight, and the
+    # gradient of the fused call is centred on the clamped targets
+    s = _outlier_rows(4, 5200 + L)
+    D = W.curvature(4, 5300 + L, seq_len=s.shape[1])
+    v = W.gaussian(4, 5400 + L, seq_len=s.shape[1])
+    soft, lz = _bcjr_gpu_w(tcq, s, L, temp, D)
+    _, _, g = tcq.bcjr_soft_and_grad(_dev(s), L, temp, _dev(v), D=_dev(D))
+    torch.cuda.synchronize()
+    rsoft, rlz = oracle.map_rows(oracle.bcjr_soft, [s], L, temp, D=D)
+    rg, _ = oracle.map_rows(oracle.bcjr_vjp, [s, v], L, temp, D=D)
+    assert np.abs(soft - rsoft).max() <= SOFT_ATOL
+    assert np.all(np.abs(lz - rlz) <= 1e-5 * np.abs(rlz) + 1e-3)
+    g = g.cpu().numpy()
+    cmax = float(np.abs(oracle.codebook_f32(L)).max())
+    for i in range(s.shape[0]):
+        # the floor of the extreme-target VJP test; grad_u carries the factor D_u
+        tol = (GRAD_RTOL_OF_MAX * np.abs(rg[i]).max()
+               + (2.0 / temp) * 2.0 ** -22 * np.abs(v[i]).sum() * cmax * D[i].max())
+        assert np.abs(g[i] - rg[i]).max() <= tol
+
+
 def _bcjr_gpu_w(tcq, s, L, temp, D):
     soft, lz = tcq.bcjr_soft(_dev(s), L, temp, D=_dev(D))
     torch.cuda.synchronize()
