@@ -91,6 +91,9 @@ struct BcjrCfg {
   // several warp-aligned sequences in one CTA step independently, each on its
   // own named barrier; they share one copy of the code values
   static constexpr bool NAMED = SPC > 1 && TPS % 32 == 0;
+  // several sequences per warp (L = 8: 16 threads each): a sequence steps on
+  // a warp barrier, since its threads exchange values only with each other
+  static constexpr bool WARPSEQ = SPC > 1 && TPS < 32 && 32 % TPS == 0;
   static constexpr int PREC = 8;                                 // floats per partial record
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
   static constexpr int NV = GRAD ? 2 : 1;                        // carried vectors (A | A, Phi)
@@ -128,13 +131,16 @@ struct BcjrCfg {
   static_assert(SPILL % 4 == 0, "spill in float4 chunks");
   static_assert(!MSG2 || (GRAD && NBUF == 1 && GQ % 4 == 0), "split buffering is for the gradient");
   static_assert(!NAMED || (SPC <= 15 && !TMEMC), "named barriers 1..15, code values in shared memory");
+  static_assert(!WARPSEQ || !TMEMC, "warp-stepped sequences keep their code values in shared memory");
 };
 
 // Barrier over the threads of one sequence: named barrier 1 + ls when the CTA
-// holds several warp-aligned sequences, else the CTA barrier.
+// holds several warp-aligned sequences, the warp barrier when a warp holds
+// whole sequences, else the CTA barrier.
 template <class C>
 __device__ __forceinline__ void seq_sync(int ls) {
   if constexpr (C::NAMED) asm volatile("bar.sync %0, %1;" ::"r"(1 + ls), "n"(C::TPS) : "memory");
+  else if constexpr (C::WARPSEQ) __syncwarp();
   else __syncthreads();
 }
 
@@ -365,7 +371,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   float *sums = reinterpret_cast<float *>(spill) + (size_t)T * NV * NG;
   auto prec = [&](int parity) { return part + ((parity * SPC + ls) * NPART) * PREC; };
 
-  if constexpr (C::NAMED) __syncthreads();                 // the shared code values are in place
+  if constexpr (C::NAMED || C::WARPSEQ) __syncthreads();   // the shared code values are in place
   // targets (and curvature, cotangent, centre) of step t of sequence row l
   auto load_row = [&](int l, int t, int64_t base) {
     const int64_t sq = base + l;
@@ -386,7 +392,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     const int64_t seq = base + ls;
     const bool active = seq < n_seq;
     seq_sync<C>(ls);                                       // previous sequence fully done
-    if constexpr (C::NAMED) {
+    if constexpr (C::NAMED || C::WARPSEQ) {                // each sequence loads its own rows
       for (int t = w; t < T; t += TPS) load_row(ls, t, base);
     } else {
       for (int x = tid; x < SPC * T; x += C::NT) load_row(x / T, x % T, base);
@@ -407,7 +413,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     } else {
       for (int x = w; x < NV * NG; x += TPS) V[x] = 0.0f;   // A_0 = 0 (and Phi_0 = 0)
     }
-    if constexpr (C::NAMED) {
+    if constexpr (C::NAMED || C::WARPSEQ) {
       for (int x = w; x < NPART * PREC; x += TPS) { prec(0)[x] = 0.0f; prec(1)[x] = 0.0f; }
     } else {
       for (int x = tid; x < 2 * SPC * NPART * PREC; x += C::NT) part[x] = 0.0f;

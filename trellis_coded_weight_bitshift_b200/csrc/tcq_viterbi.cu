@@ -43,6 +43,9 @@ struct VitCfg {
   static constexpr int ASM = 4 - AREG;         // predecessor digits whose codes sit in smem
   static constexpr int BPB = G / 4;            // backpointer bytes per thread per step
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
+  // several sequences per warp (L = 8: 16 threads each): a sequence steps on
+  // a warp barrier, since its threads exchange values only with each other
+  static constexpr bool WARPSEQ = SPC > 1 && TPS < 32 && 32 % TPS == 0;
   // the ASM digits not in registers sit in tensor memory (TMEMC: this thread's
   // lane, columns (q ASM + a - AREG) 4 + r) or in shared memory
   static constexpr bool TMEMC = TMEMC_;
@@ -325,7 +328,8 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
       else if constexpr (C::BPB == 4) *reinterpret_cast<uint32_t *>(dst) = bits[0];
       else *reinterpret_cast<uint2 *>(dst) = make_uint2(bits[0], bits[1]);
     }
-    __syncthreads();
+    if constexpr (C::WARPSEQ) __syncwarp();                       // M_t is this sequence's own
+    else __syncthreads();
   }
 
   // Final decision: cost_{T-1}(p) = M_{T-1}(p >> 2) + e_{T-1}(p); lowest p wins ties.
