@@ -115,14 +115,13 @@ struct BcjrCfg {
   // workspace and the sequence's threads turn them into outputs in parallel
   // (finishing each step on one thread during the sweep stalls the other warps
   // of the sequence at the next barrier).
-  static constexpr bool DEFER = true;
   static constexpr int NQS = GRAD ? 4 : 2;                        // sums per record
-  // per resident sequence: the spilled messages, then (DEFER) the per-step
-  // partial sums (numerator, denominator; gradient: and the two moments) of
-  // each warp; a whole number of 256-byte units, so that every slot (read as
+  // per resident sequence: the spilled messages, then the per-step partial
+  // sums (numerator, denominator; gradient: and the two moments) of each
+  // warp; a whole number of 256-byte units, so that every slot (read as
   // float4) stays 16-byte aligned
   __host__ __device__ static constexpr size_t ws_floats_per_slot(int T) {
-    return ((size_t)T * NV * NG + (DEFER ? (size_t)T * NPART * NQS : 0) + 63) / 64 * 64;
+    return ((size_t)T * NV * NG + (size_t)T * NPART * NQS + 63) / 64 * 64;
   }
   static_assert(NG % G == 0 && G % 4 == 0, "bad split");
   static_assert(AREG % 2 == 0, "code values are held in digit pairs");
@@ -366,7 +365,7 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
   // at this thread's groups r = a*NG/4 + GQ*w + k, flattened as a*GQ + k.
   float4 *spill = reinterpret_cast<float4 *>(ws + (size_t)(blockIdx.x * SPC + ls) *
                                                       C::ws_floats_per_slot(T));
-  // DEFER: [T][NPART] records of NQS sums (numerator, denominator; gradient:
+  // then [T][NPART] records of NQS sums (numerator, denominator; gradient:
   // the two moments), read back once the backward is done
   float *sums = reinterpret_cast<float *>(spill) + (size_t)T * NV * NG;
   auto prec = [&](int parity) { return part + ((parity * SPC + ls) * NPART) * PREC; };
@@ -739,19 +738,6 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         dprev = pp[0];
 #pragma unroll
         for (int x = 1; x < NPART; ++x) dprev = fmaxf(dprev, pp[x * PREC]);
-        if (!C::DEFER && w == 0 && active) {                 // finish step tc + 1
-          float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f;
-#pragma unroll
-          for (int x = 0; x < NPART; ++x) {
-            num += pp[x * PREC + 1]; den += pp[x * PREC + 2];
-            if (GRAD) { n1 += pp[x * PREC + 3]; n2 += pp[x * PREC + 4]; }
-          }
-          const float inv = 1.0f / den;
-          if (soft_out) soft_out[seq * T + tc + 1] = num * inv;
-          if (GRAD)
-            grad_out[seq * T + tc + 1] = (1.3862943611198906f * ksm[ls * 256 + tc + 1]) *
-                                         (n2 * inv - (num * inv) * (n1 * inv));
-        }
       }
       if (NB == 1) seq_sync<C>(ls);
       const float K = Krun;
@@ -893,15 +879,13 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
         const float mine = seq_sums<TPS, NQ>(q4, lane);
         const int o = lane & (WL - 1);
         float *pp = prec(tc & 1) + pidx * PREC;
-        if ((o & (WL / NQ - 1)) == 0) {                                  // num, den (n1, n2)
-          if constexpr (C::DEFER) sums[((size_t)tc * NPART + pidx) * C::NQS + o / (WL / NQ)] = mine;
-          else pp[1 + o / (WL / NQ)] = mine;
-        }
+        if ((o & (WL / NQ - 1)) == 0)                                    // num, den (n1, n2)
+          sums[((size_t)tc * NPART + pidx) * C::NQS + o / (WL / NQ)] = mine;
         if (plead) pp[0] = tmax;
       }
       seq_sync<C>(ls);
     }
-    if (C::DEFER && active) {
+    if (active) {
       // every step's sums are in the workspace (the barrier that closed the
       // last step orders them): the sequence's threads finish them in parallel
       for (int u = w; u < T; u += TPS) {
@@ -919,19 +903,6 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
                                   (n2 * inv - (num * inv) * (n1 * inv));
         }
       }
-    }
-    if (!C::DEFER && w == 0 && active) {                     // finish step 0
-      const float *pp = prec(0);
-      float num = 0.0f, den = 0.0f, n1 = 0.0f, n2 = 0.0f;
-#pragma unroll
-      for (int x = 0; x < NPART; ++x) {
-        num += pp[x * PREC + 1]; den += pp[x * PREC + 2];
-        if (GRAD) { n1 += pp[x * PREC + 3]; n2 += pp[x * PREC + 4]; }
-      }
-      const float inv = 1.0f / den;
-      if (soft_out) soft_out[seq * T] = num * inv;
-      if (GRAD)   // 2 D_u / temp = 2 ln2 kappa D_u
-        grad_out[seq * T] = (1.3862943611198906f * ksm[ls * 256]) * (n2 * inv - (num * inv) * (n1 * inv));
     }
   }
   if constexpr (C::TMEMC) {                                // every thread is done with its lane
