@@ -89,3 +89,32 @@ def test_stream_words(L):
     tr = _abi.trellis(16, 7)                       # 14 bits: too short to wrap a 16-bit window
     assert L.tcq_stream_words(ctypes.byref(tr), _abi.TAILBITING) == 0
     assert L.tcq_stream_words(ctypes.byref(tr), _abi.FREE_START) == 1
+
+
+def test_empty_and_negative_batches_on_every_entry_point(L):
+    # n_seq = 0 is an empty batch: TCQ_OK, nothing enqueued, no pointer read
+    # (all are NULL here).  A negative count is an invalid argument.  Matrix
+    # calls with a zero dimension are invalid (a 16x16 tile needs 16 of each).
+    from trellis_coded_weight_bitshift_b200 import _abi
+    f = ctypes.c_float
+    for Lb in (8, 12, 16):
+        tr = ctypes.byref(_abi.trellis(Lb, 256))
+        calls = {
+            "viterbi": lambda n: L.tcq_viterbi_encode(tr, None, None, n, None, None, None, None, 0, None),
+            "noalloc": lambda n: L.tcq_viterbi_encode_noalloc(tr, None, n, None, None, None),
+            "tailbiting": lambda n: L.tcq_viterbi_encode_tailbiting(tr, None, None, n, None, None, None, 0, None),
+            "soft": lambda n: L.tcq_bcjr_soft(tr, None, None, n, f(0.1), None, None, None, 0, None),
+            "backward": lambda n: L.tcq_bcjr_soft_backward(tr, None, None, n, f(0.1), None, None, None, None, 0,
+                                                           None),
+            "soft_and_grad": lambda n: L.tcq_bcjr_soft_and_grad(tr, None, None, n, f(0.1), None, None, None, None,
+                                                                None, 0, None),
+            "pack": lambda n: L.tcq_pack_states(tr, None, n, _abi.FREE_START, None, None),
+            "decode": lambda n: L.tcq_decode(tr, None, n, _abi.TAILBITING, _abi.OUT_SEQ, 0, 0, None, None),
+        }
+        for name, call in calls.items():
+            assert call(0) == _abi.TCQ_OK, (Lb, name)
+            assert call(-1) == _abi.TCQ_ERR_INVALID_ARG, (Lb, name)
+    tr16 = ctypes.byref(_abi.trellis(16, 256))
+    assert L.tcq_decode_gemv(tr16, None, _abi.TAILBITING, 0, 16, None, None, None) == _abi.TCQ_ERR_INVALID_ARG
+    assert L.tcq_decode_gemv(tr16, None, _abi.TAILBITING, 16, 0, None, None, None) == _abi.TCQ_ERR_INVALID_ARG
+    assert L.tcq_rht(None, 0, 64, None, None, None, None) == _abi.TCQ_ERR_INVALID_ARG
