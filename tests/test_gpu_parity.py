@@ -285,6 +285,31 @@ def test_bcjr_l16_student_t(tcq, temp):
     assert np.all(np.abs(lz[idx] - rlz) <= 1e-5 * np.abs(rlz) + 1e-3)
 
 
+@pytest.mark.parametrize("temp", [1.0, 0.01])
+def test_bcjr_config4_full_properties(tcq, temp):
+    # every one of the 65,536 Student-t sequences, at the temperatures the
+    # workload ends on: the soft codeword is finite and inside the code range,
+    # and log Z lies between the two bounds the Viterbi energy E_min gives
+    # (Z holds the minimum walk, and is a sum over 2^(L + 2 (T - 1)) walks):
+    #   -E_min/temp <= log Z <= -E_min/temp + (L + 2 (T - 1)) ln 2
+    # with E_min = 256 x the walk's MSE, each side within log Z's 1e-5 relative
+    s = W.sequences("l16_studentt_2048x8192")
+    sd = _dev(s)
+    soft, lz = tcq.bcjr_soft(sd, 16, temp)
+    soft, lz = soft.cpu().numpy(), lz.cpu().numpy().astype(np.float64)
+    # Viterbi in chunks of 8,192 sequences (8.5 GB of backpointers each)
+    mse = np.concatenate([tcq.viterbi_encode(sd[i:i + 8192], 16)[1].cpu().numpy()
+                          for i in range(0, sd.shape[0], 8192)])
+    torch.cuda.empty_cache()
+    c = oracle.codebook_f32(16)
+    assert np.all(np.isfinite(soft)) and np.all(np.isfinite(lz))
+    assert soft.min() >= c.min() - 1e-6 and soft.max() <= c.max() + 1e-6
+    lo = -256.0 * mse.astype(np.float64) / temp
+    slack = 1e-5 * np.abs(lo) + 1e-3
+    assert np.all(lz >= lo - slack)
+    assert np.all(lz <= lo + (16 + 2 * 255) * np.log(2.0) + slack)
+
+
 @pytest.mark.parametrize("L", [8, 12, 16])
 @pytest.mark.parametrize("T,n", [(1, 2), (2, 3), (5, 9), (33, 1)])
 def test_bcjr_edge_shapes(tcq, L, T, n):
@@ -732,7 +757,7 @@ def _gemv_ref(bits, rows, cols, x, L=16, layout=0, tile_rows=None):
 
 
 @pytest.mark.parametrize("L,layout,rows,cols", [(16, 0, 256, 512), (8, 1, 96, 160), (12, 0, 1024, 2048),
-                                             (12, 1, 32, 16400)])
+                                             (12, 1, 32, 16400), (16, 1, 80, 272)])
 def test_decode_gemv_matches_oracle(tcq, L, layout, rows, cols):
     # 16400 columns: a row of 1,025 tiles, split into runs that do not divide it
     rng = np.random.default_rng(rows + cols + L)
