@@ -737,6 +737,16 @@ def test_rht_in_place_and_8192_square_sampled(tcq):
     ref = oracle.rht_entries(W, s1, s2, ri, ci)
     assert np.abs(got[ri][:, ci] - ref).max() <= 4 * RHT_ATOL * np.sqrt(5 / 3)
     assert abs(float(np.linalg.norm(got.astype(np.float64))) / float(np.linalg.norm(W.astype(np.float64))) - 1) < 1e-5
+    # the rotation is orthonormal and (H/sqrt n)^2 = I: rotating the result
+    # again with unit signs gives diag(s1) W diag(s2), on all 67 M entries.
+    # Each of the 2 x 26 butterfly levels rounds once, at 2^-24 of values that
+    # stay within sqrt(2)^26 of the entries' scale only in the worst case;
+    # the bound below is 64 roundings of the largest entry.
+    tcq.rht(d, _dev(np.ones(R, np.float32)), _dev(np.ones(C, np.float32)), out=d)
+    back = d * _dev(s1)[:, None] * _dev(s2)[None, :]
+    err = float((back - _dev(W)).abs().max())
+    print(f"rht round trip on 8192 x 8192: max |error| {err:.3g}, max |W| {np.abs(W).max():.3g}")
+    assert err <= 64 * 2.0 ** -24 * float(np.abs(W).max())
 
 
 # ---------------------------------------------------------------- decode fused into a GEMV
