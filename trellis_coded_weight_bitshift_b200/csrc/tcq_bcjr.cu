@@ -94,6 +94,12 @@ struct BcjrCfg {
   // several sequences per warp (L = 8: 16 threads each): a sequence steps on
   // a warp barrier, since its threads exchange values only with each other
   static constexpr bool WARPSEQ = SPC > 1 && TPS < 32 && 32 % TPS == 0;
+  // backward exponents against the combine's reference, so that the four
+  // successor terms are posteriors (one ex2 and a maximum fewer per group);
+  // it puts the spilled A on the B recursion's path, which L = 8 cannot hide
+  // (soft pass 0.158 -> 0.171 ms on 64 sequences), while L = 12 and 16 gain
+  // 1-3% (soft) and 3% (soft + VJP)
+  static constexpr bool POSTB = !WARPSEQ;
   static constexpr int PREC = 8;                                 // floats per partial record
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
   static constexpr int NV = GRAD ? 2 : 1;                        // carried vectors (A | A, Phi)
@@ -813,48 +819,93 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
               const f2_t d = f2sub(cc[b], sv2);
               y[b] = f2fma(d, f2fma(nk2, d, b2), f2(bk[b], bk[b]));
             }
-            // exponents taken against the combine's reference K: with
-            // aK = A_tc(r) - K, 2^(aK + y_b) is the posterior of successor
-            // state 4r + b at step tc (at most 1, so no maximum is needed).
-            // Their sums give the combine's weights directly,
-            // B_t(r) = lg2(sum) - aK - dp and (gradient) Psi_t(r) = the
-            // weighted mean of z: four ex2 and one lg2 per group, where a
-            // maximum-relative log-sum-exp and a separate group weight take
-            // five ex2.  A term that underflows is a state whose posterior is
-            // below 2^-126; the paths through it change no output.
-            const f2_t aK = f2sub(f2(avl[j], avh[j]), K2);
-            f2_t S, sc, sz, scz;
+            if constexpr (C::POSTB) {
+              // exponents taken against the combine's reference K: with
+              // aK = A_tc(r) - K, 2^(aK + y_b) is the posterior of successor
+              // state 4r + b at step tc (at most 1, so no maximum is needed).
+              // Their sums give the combine's weights directly,
+              // B_t(r) = lg2(sum) - aK - dp and (gradient) Psi_t(r) = the
+              // weighted mean of z: four ex2 and one lg2 per group, where a
+              // maximum-relative log-sum-exp and a separate group weight take
+              // five ex2.  A term that underflows is a state whose posterior is
+              // below 2^-126; the paths through it change no output.
+              const f2_t aK = f2sub(f2(avl[j], avh[j]), K2);
+              f2_t S, sc, sz, scz;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-              const f2_t e = f2add(y[b], aK);
-              const f2_t v = f2(ex2(f2lo(e)), ex2(f2hi(e)));
-              S = b == 0 ? v : f2add(S, v);
-              if constexpr (!GRAD) {
-                sc = b == 0 ? f2mul(v, cc[b]) : f2fma(v, cc[b], sc);
-              } else {
-                const f2_t vc = f2mul(v, cc[b]);
-                sc = b == 0 ? vc : f2add(sc, vc);
-                // z_b = psi_{tc}(succ) + v_tc (c_b - soft_tc)
-                const float pz = pin[4 * k + b] + nvf;
-                const f2_t z = f2fma(vv2, cc[b], f2(pz, pz));
-                sz = b == 0 ? f2mul(v, z) : f2fma(v, z, sz);
-                scz = b == 0 ? f2mul(vc, z) : f2fma(vc, z, scz);
+              for (int b = 0; b < 4; ++b) {
+                const f2_t e = f2add(y[b], aK);
+                const f2_t v = f2(ex2(f2lo(e)), ex2(f2hi(e)));
+                S = b == 0 ? v : f2add(S, v);
+                if constexpr (!GRAD) {
+                  sc = b == 0 ? f2mul(v, cc[b]) : f2fma(v, cc[b], sc);
+                } else {
+                  const f2_t vc = f2mul(v, cc[b]);
+                  sc = b == 0 ? vc : f2add(sc, vc);
+                  // z_b = psi_{tc}(succ) + v_tc (c_b - soft_tc)
+                  const float pz = pin[4 * k + b] + nvf;
+                  const f2_t z = f2fma(vv2, cc[b], f2(pz, pz));
+                  sz = b == 0 ? f2mul(v, z) : f2fma(v, z, sz);
+                  scz = b == 0 ? f2mul(vc, z) : f2fma(vc, z, scz);
+                }
               }
-            }
-            const f2_t ob = f2sub(f2(lg2(f2lo(S)), lg2(f2hi(S))), f2add(aK, dp2));
-            outL[j] = f2lo(ob);
-            outH[j] = f2hi(ob);
-            tmax = fmaxf(tmax, fmaxf(outL[j], outH[j]));
-            den2 = f2add(den2, S);
-            num2 = f2add(num2, sc);
-            if constexpr (GRAD) {
-              // Psi_t(r) = sz / S, and 0 where every successor underflowed
-              // (their weight is 0 wherever the value is used)
-              outPL[j] = f2lo(S) > 0.0f ? f2lo(sz) * rcp(f2lo(S)) : 0.0f;
-              outPH[j] = f2hi(S) > 0.0f ? f2hi(sz) * rcp(f2hi(S)) : 0.0f;
-              const f2_t fa2 = f2(fal[j], fah[j]);
-              n12 = f2add(n12, f2fma(fa2, S, sz));
-              n22 = f2add(n22, f2fma(fa2, sc, scz));
+              const f2_t ob = f2sub(f2(lg2(f2lo(S)), lg2(f2hi(S))), f2add(aK, dp2));
+              outL[j] = f2lo(ob);
+              outH[j] = f2hi(ob);
+              tmax = fmaxf(tmax, fmaxf(outL[j], outH[j]));
+              den2 = f2add(den2, S);
+              num2 = f2add(num2, sc);
+              if constexpr (GRAD) {
+                // Psi_t(r) = sz / S, and 0 where every successor underflowed
+                // (their weight is 0 wherever the value is used)
+                outPL[j] = f2lo(S) > 0.0f ? f2lo(sz) * rcp(f2lo(S)) : 0.0f;
+                outPH[j] = f2hi(S) > 0.0f ? f2hi(sz) * rcp(f2hi(S)) : 0.0f;
+                const f2_t fa2 = f2(fal[j], fah[j]);
+                n12 = f2add(n12, f2fma(fa2, S, sz));
+                n22 = f2add(n22, f2fma(fa2, sc, scz));
+              }
+            } else {
+              // maximum-relative log-sum-exp and a separate group weight: the
+              // B recursion does not wait on the spilled A (L = 8, where one
+              // warp per scheduler leaves that latency exposed)
+              const float mxl = fmaxf(fmaxf(f2lo(y[0]), f2lo(y[1])), fmaxf(f2lo(y[2]), f2lo(y[3])));
+              const float mxh = fmaxf(fmaxf(f2hi(y[0]), f2hi(y[1])), fmaxf(f2hi(y[2]), f2hi(y[3])));
+              const f2_t mx2 = f2(mxl, mxh);
+              // sums over the four successors, accumulated one successor at a
+              // time (fewer live registers than four separate weights)
+              f2_t su, sc, sz, scz;
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const f2_t e = f2sub(y[b], mx2);
+                const f2_t u = f2(ex2(f2lo(e)), ex2(f2hi(e)));
+                su = b == 0 ? u : f2add(su, u);
+                if constexpr (!GRAD) {
+                  sc = b == 0 ? f2mul(u, cc[b]) : f2fma(u, cc[b], sc);
+                } else {
+                  const f2_t uc = f2mul(u, cc[b]);
+                  sc = b == 0 ? uc : f2add(sc, uc);
+                  // z_b = psi_{tc}(succ) + v_tc (c_b - soft_tc)
+                  const float pz = pin[4 * k + b] + nvf;
+                  const f2_t z = f2fma(vv2, cc[b], f2(pz, pz));
+                  sz = b == 0 ? f2mul(u, z) : f2fma(u, z, sz);
+                  scz = b == 0 ? f2mul(uc, z) : f2fma(uc, z, scz);
+                }
+              }
+              const f2_t ob = f2add(f2sub(mx2, dp2), f2(lg2(f2lo(su)), lg2(f2hi(su))));
+              outL[j] = f2lo(ob);
+              outH[j] = f2hi(ob);
+              tmax = fmaxf(tmax, fmaxf(outL[j], outH[j]));
+              const f2_t wv = f2add(f2sub(f2(avl[j], avh[j]), K2), mx2);
+              const f2_t wgt = f2(ex2(f2lo(wv)), ex2(f2hi(wv)));
+              den2 = f2fma(wgt, su, den2);
+              num2 = f2fma(wgt, sc, num2);
+              if constexpr (GRAD) {
+                const f2_t op = f2mul(sz, f2(rcp(f2lo(su)), rcp(f2hi(su))));
+                outPL[j] = f2lo(op);
+                outPH[j] = f2hi(op);
+                const f2_t fa2 = f2(fal[j], fah[j]);
+                n12 = f2fma(wgt, f2fma(fa2, su, sz), n12);
+                n22 = f2fma(wgt, f2fma(fa2, sc, scz), n22);
+              }
             }
           }
           if (t >= 0) {
