@@ -25,7 +25,10 @@
 //     the mirror image of the forward step);
 //   * combine: alpha_{t+1}(4r+b) + beta_{t+1}(4r+b) = A_{t+1}(r) + y_b where
 //     y_b are the four inputs of the backward log-sum-exp for r, so the soft
-//     codeword reuses those four exponentials plus one for the group weight;
+//     codeword reuses those four exponentials: taken against the combine's
+//     exponent reference K they are the posteriors themselves (L = 12, 16),
+//     or, relative to their maximum, they take one more for the group weight
+//     (L = 8);
 //   * A_t is renormalised every step by the running maximum (a constant per
 //     step, global over the sequence), and so is B; the constants are tracked
 //     to place the combine's exponent reference K_t = log2 Z - (constants)
