@@ -10,7 +10,12 @@
 //   beta_{T-1} = 0,             beta_t(i)  = LSE_b [beta_{t+1}(succ_b i) - e_{t+1}(succ_b i)/temp]
 //   soft_t = sum_j softmax_j(alpha_t + beta_t) code_j
 // Everything here runs in base 2 (kappa = log2(e)/temp scales the energy) on
-// the MUFU ex2/lg2 units, fp32.
+// the MUFU ex2/lg2 units, fp32.  Each step's emission is taken relative to r,
+// the target clamped to the code range: -kappa (c - s)^2 differs from
+// d (-kappa d + 2 kappa (s - r)), d = c - r, by a constant of the step, which
+// cancels in every expectation and is added back to log Z in fp64; for a
+// target outside the range the states that compete then carry small,
+// accurately rounded emissions.
 //
 // Structure (k = 2, the same one as the Viterbi kernel):
 //   * forward: the four states j = 4q + b share one log-sum-exp over their
@@ -41,8 +46,9 @@
 // so grad_u = (2/temp) Cov(F, code(x_u)) with F = sum_t v_t (code(x_t) - soft_t)
 // (centred by the forward soft codeword when it is given, else by the target
 // clamped to the code range: any per-step constant leaves the covariance
-// unchanged, and a centre near the codes keeps F small).  E[F | x_u = j] splits by the Markov
-// property into a prefix part phi (forward expectation recursion, weights =
+// unchanged, and a centre near the codes keeps F small).  E[F | x_u = j]
+// splits by the Markov property into a prefix part phi (forward expectation
+// recursion, weights =
 // the forward softmax over predecessors) and a suffix part psi (backward
 // recursion, weights = the backward softmax over successors); both reuse the
 // exponentials of the log-sum-exps above.
