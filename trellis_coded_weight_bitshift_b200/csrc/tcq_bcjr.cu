@@ -48,10 +48,9 @@
 // clamped to the code range: any per-step constant leaves the covariance
 // unchanged, and a centre near the codes keeps F small).  E[F | x_u = j]
 // splits by the Markov property into a prefix part phi (forward expectation
-// recursion, weights =
-// the forward softmax over predecessors) and a suffix part psi (backward
-// recursion, weights = the backward softmax over successors); both reuse the
-// exponentials of the log-sum-exps above.
+// recursion, weights = the forward softmax over predecessors) and a suffix
+// part psi (backward recursion, weights = the backward softmax over
+// successors); both reuse the exponentials of the log-sum-exps above.
 #include <algorithm>
 #include <mutex>
 
