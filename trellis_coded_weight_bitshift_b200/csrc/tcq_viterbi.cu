@@ -249,7 +249,10 @@ viterbi_fwd_kernel(const float *__restrict__ s, const float *__restrict__ Dw, in
     // Two neighbouring groups i, i+1 with the same predecessor digit a share
     // the input M(q), so their candidate costs are computed as a packed pair:
     // d = c - s, e = d*d (written fma(d, d, +0)), cost = M + e, each lane
-    // rounded exactly like the scalar operation.
+    // rounded exactly like the scalar operation.  A packed multiply followed
+    // by the packed add is fused into one fused multiply-add by the compiler
+    // (one rounding instead of two): written as a multiply, the MSE moved by
+    // an ulp against the oracle's separately rounded operations.
     const f2_t sv2 = f2(sv, sv);
     const float dv = WEIGHTED ? dsm[ls * 256 + t - 1] : 1.0f;
     const f2_t dv2 = f2(dv, dv);
