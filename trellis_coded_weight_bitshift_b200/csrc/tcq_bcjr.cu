@@ -104,10 +104,12 @@ struct BcjrCfg {
   static constexpr bool WARPSEQ = SPC > 1 && TPS < 32 && 32 % TPS == 0;
   // backward exponents against the combine's reference, so that the four
   // successor terms are posteriors (one ex2 and a maximum fewer per group);
-  // it puts the spilled A on the B recursion's path, which L = 8 cannot hide
-  // (soft pass 0.158 -> 0.171 ms on 64 sequences), while L = 12 and 16 gain
-  // 1-3% (soft) and 3% (soft + VJP)
-  static constexpr bool POSTB = !WARPSEQ;
+  // it puts the spilled A on the B recursion's path, which the L = 8
+  // gradient (its spill read inside the step) cannot hide; the soft passes
+  // read it from registers loaded a step ahead (L = 8 soft with the spill
+  // read in the step: 0.158 -> 0.171 ms on 64 sequences; L = 12 and 16 gain
+  // 1-3% soft and 3% soft + VJP)
+  static constexpr bool POSTB = !WARPSEQ || !GRAD;
   static constexpr int PREC = 8;                                 // floats per partial record
   static constexpr int SWZ = (GQ >= 8 ? 7 : GQ - 1);
   static constexpr int NV = GRAD ? 2 : 1;                        // carried vectors (A | A, Phi)
@@ -713,15 +715,26 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
     }
     seq_sync<C>(ls);
     float Krun = log2Zrel;
+    // soft pass with G <= 16: the thread's spilled A of each backward step
+    // sits in registers, loaded one step ahead
+    constexpr bool PREFETCH = !GRAD && G <= 16;
+    [[maybe_unused]] float4 avn[PREFETCH ? NCH : 1];
+    if constexpr (PREFETCH) {
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) avn[c] = spill[((size_t)(T - 1) * NCH + c) * TPS + w];
+    }
     for (int t = T - 2; t >= -1; --t) {
       const int tc = t + 1;                                  // combine step
       // this thread's spilled A_tc values (issued first: they come from HBM)
       // (the gradient pass carries twice the values and would spill registers)
-      constexpr bool PREFETCH = !GRAD && G <= 16;
       float4 avq[PREFETCH ? NCH : 1];
-      if constexpr (PREFETCH) {
+      if constexpr (PREFETCH) {                              // this step's, loaded a step ago
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) avq[c] = spill[((size_t)tc * NCH + c) * TPS + w];
+        for (int c = 0; c < NCH; ++c) avq[c] = avn[c];
+        if (tc > 0) {
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) avn[c] = spill[((size_t)(tc - 1) * NCH + c) * TPS + w];
+        }
       }
       // the next step's spilled chunks are read a whole step from now: start
       // bringing them on chip (register prefetch covers the small soft case)
