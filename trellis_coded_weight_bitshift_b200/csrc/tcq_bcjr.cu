@@ -782,13 +782,12 @@ bcjr_kernel(const float *__restrict__ s, const float *__restrict__ Dw, int64_t n
       const f2_t K2 = f2(K, K), dp2 = f2(dprev, dprev), vv2 = f2(vv, vv);
       f2_t num2 = f2(0.0f, 0.0f), den2 = num2, n12 = num2, n22 = num2;
       // KB values of this thread's spilled vector at flat index f (KB | f)
-      // sub-run width: 4 when the code values come from tensor memory (the
-      // registers they free hold the wider block) in the soft pass; 2 in the
-      // L = 16 gradient pass, which holds Psi of 32 groups across the step's
-      // first barrier (1 and 4 were measured: 1 spilled fewer registers but
-      // read every spilled float4 twice, 24.2 vs 23.5 ms on 1,036
-      // sequences); else 2
-      constexpr int KB = GQ < 2 ? GQ : (C::TMEMC && GQ >= 4 ? (GRAD ? 2 : 4) : 2);
+      // sub-run width 2.  Measured at L = 16: in the gradient pass, which
+      // holds Psi of 32 groups across the step's first barrier, 1 spilled
+      // fewer registers but read every spilled float4 twice (24.2 vs 23.5 ms
+      // on 1,036 sequences); in the soft pass, 4 ran 60.0 against 58.2 ms on
+      // 4,440 sequences
+      constexpr int KB = GQ < 2 ? GQ : 2;
       auto spilled_run = [&](int f, float *dst) {
         float4 v;
         if constexpr (PREFETCH) v = avq[PREFETCH ? (f >> 2) : 0];
