@@ -33,6 +33,23 @@ def test_irwin_hall_closed_form_of_the_constants():
     assert round(math.sqrt(var), 1) == c["scale"]
 
 
+def test_special_states_follow_the_printed_constants():
+    # Two states whose LCG output the printed constants fix without the
+    # multiplication: at x = 0 the output is the increment itself, and at
+    # x = 2^31 an odd multiplier gives a x = 2^31 (mod 2^32), so the output is
+    # the increment with its top bit flipped.  The increment 76625530 =
+    # 0x0491367A has bytes 4, 145, 54, 122 (sum 325); flipping its top bit
+    # raises the top byte from 4 to 132 (sum 453).
+    inc = GOLD["one_mad_constants"]["lcg_increment"]
+    assert inc == 0x0491367A
+    assert oracle.bytesum_1mad(0) == 4 + 145 + 54 + 122 == 325
+    assert oracle.bytesum_1mad(2 ** 31) == 132 + 145 + 54 + 122 == 453
+    # the table is indexed by the state itself: entry 0 is that value, centred
+    # and scaled, at every L
+    for L in (8, 12, 16):
+        assert oracle.codebook_f64(L)[0] == (325.0 - 510.0) / 147.8
+
+
 def test_bytesum_distribution_matches_irwin_hall():
     # sample uniform 32-bit inputs; by the bijection above the oracle's byte sum
     # must follow the n=4 discrete uniform-sum law (mean 510, var 21845).

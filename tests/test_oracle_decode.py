@@ -81,6 +81,31 @@ def test_pack_then_decode_is_identity_tailbiting(L):
     assert np.array_equal(oracle.pack(st, L, oracle.TAILBITING), words)
 
 
+@pytest.mark.parametrize("L,k,T", [(4, 2, 3), (4, 2, 4), (6, 2, 3), (4, 1, 4)])
+def test_stream_lengths_count_the_walks(L, k, T):
+    # Every sequence of T states, kept when each state is its predecessor
+    # shifted left by k bits with k new low bits (a walk of the bitshift
+    # trellis).  Pack is one-to-one on walks and decode turns every stream into
+    # a walk, so a layout of n stream bits must hold exactly 2^n walks: free
+    # start, L bits for the first state and k per later step; tail-biting,
+    # the walks whose last state's low L-k bits are the first state's high
+    # L-k bits, exactly k*T bits.
+    grid = np.stack(np.meshgrid(*[np.arange(1 << L)] * T, indexing="ij"), -1).reshape(-1, T)
+    low = (1 << (L - k)) - 1
+    walks = grid[np.all((grid[:, 1:] >> k) == (grid[:, :-1] & low), axis=1)]
+    circ = walks[(walks[:, 0] >> k) == (walks[:, -1] & low)]
+    assert len(walks) == 2 ** oracle.stream_nbits(L, k, T, oracle.FREE_START)
+    assert len(circ) == 2 ** oracle.stream_nbits(L, k, T, oracle.TAILBITING) == 2 ** (k * T)
+    for layout, w in ((oracle.FREE_START, walks), (oracle.TAILBITING, circ)):
+        words = oracle.pack(w, L, layout, k=k)
+        nb = oracle.stream_nbits(L, k, T, layout)
+        pad = 32 * words.shape[1] - nb
+        ints = [_to_int(r) for r in words]
+        assert len(set(ints)) == len(w)                      # distinct streams
+        assert all(v & ((1 << pad) - 1) == 0 for v in ints)  # only the first nb bits used
+        assert np.array_equal(oracle.windows(words, L, k, T, layout), w)
+
+
 def test_tile_layout():
     rng = np.random.default_rng(9)
     words = rng.integers(0, 2 ** 32, (4 * 6, 16), dtype=np.uint32)
