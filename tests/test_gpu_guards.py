@@ -226,3 +226,54 @@ def test_concurrent_streams_match_sequential(abi):
         for x, y in zip(a, b):
             assert torch.equal(x.view(torch.int16) if x.dtype == torch.uint16 else x,
                                y.view(torch.int16) if y.dtype == torch.uint16 else y)
+
+
+def test_binding_checks_callers_buffers_before_launch(abi):
+    # The library sees only pointers, so the Python binding refuses, before
+    # any launch, a caller's output that the kernels would write past (wrong
+    # shape or dtype) or that is host memory, a host workspace, and
+    # cotangents of the wrong dtype.  A caller's workspace of any dtype that
+    # holds enough bytes is used and gives the same bits as an internal one.
+    import trellis_coded_weight_bitshift_b200 as tcq
+    bits = torch.zeros(4, 16, dtype=torch.int32, device="cuda").view(torch.uint32)
+    for out in (torch.empty(4, 255, dtype=torch.float16, device="cuda"),
+                torch.empty(4, 256, dtype=torch.float32, device="cuda"),
+                torch.empty(4, 256, dtype=torch.float16)):
+        with pytest.raises(ValueError, match="out must be|CUDA"):
+            tcq.decode(bits, 16, 256, tcq.TAILBITING, tcq.OUT_SEQ, out=out)
+    with pytest.raises(ValueError, match="out must be"):
+        tcq.decode(bits, 16, 256, tcq.TAILBITING, tcq.OUT_TILE16, 32, 32,
+                   out=torch.empty(32, 16, dtype=torch.float16, device="cuda"))
+    wm = torch.zeros(16, 32, device="cuda")
+    sr, sc = torch.ones(16, device="cuda"), torch.ones(32, device="cuda")
+    for out in (torch.empty(32, 16, device="cuda"),
+                torch.empty(16, 32, dtype=torch.float64, device="cuda"),
+                torch.empty(16, 32)):
+        with pytest.raises(ValueError, match="out must be|CUDA"):
+            tcq.rht(wm, sr, sc, out=out)
+    x = torch.zeros(32, device="cuda")
+    for out in (torch.empty(31, device="cuda"),
+                torch.empty(32, dtype=torch.float16, device="cuda"),
+                torch.empty(32)):
+        with pytest.raises(ValueError, match="out must be|CUDA"):
+            tcq.decode_gemv(bits, x, 32, 32, out=out)
+
+    s = torch.from_numpy(W.gaussian(3, 964)).cuda()
+    with pytest.raises(ValueError, match="float32"):
+        tcq.bcjr_soft_backward(s, 12, 1.0, s, s.half())
+    with pytest.raises(ValueError, match="float32"):
+        tcq.bcjr_soft_and_grad(s, 12, 1.0, s.double())
+    with pytest.raises(ValueError, match="CUDA"):
+        tcq.viterbi_encode(s, 12, workspace=torch.empty(1 << 20, dtype=torch.uint8))
+
+    need_v = tcq.viterbi_workspace_size(12, 256, 3)
+    need_b = tcq.bcjr_workspace_size(12, 256, 3)
+    ws_v = torch.empty((need_v + 3) // 4, dtype=torch.float32, device="cuda")
+    ws_b = torch.empty((need_b + 3) // 4, dtype=torch.float32, device="cuda")
+    got = (tcq.viterbi_encode(s, 12, workspace=ws_v), tcq.bcjr_soft(s, 12, 0.5, workspace=ws_b))
+    ref = (tcq.viterbi_encode(s, 12), tcq.bcjr_soft(s, 12, 0.5))
+    torch.cuda.synchronize()
+    for a, b in zip(got, ref):
+        for u, v in zip(a, b):
+            assert torch.equal(u.view(torch.int16) if u.dtype == torch.uint16 else u,
+                               v.view(torch.int16) if v.dtype == torch.uint16 else v)

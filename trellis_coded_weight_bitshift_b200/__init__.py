@@ -36,12 +36,39 @@ __all__ = [
 ]
 
 
-def _require_cuda(*tensors: torch.Tensor) -> None:
+def _require_cuda(*tensors: "torch.Tensor | None") -> None:
+    """Every tensor a call hands to the library (None entries skipped) is
+    contiguous and on the current CUDA device, the one the library launches
+    on: a host pointer, or another device's, would reach the kernels."""
+    dev = None
     for t in tensors:
+        if t is None:
+            continue
         if not t.is_cuda:
             raise ValueError("tensors must be CUDA tensors (no CPU fallback)")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors must all be on one device ({dev} and {t.device})")
+    if dev is not None and dev.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {dev} but the current device is "
+                         f"cuda:{torch.cuda.current_device()} (select it with torch.cuda.device)")
+
+
+def _out(out: torch.Tensor, shape, dtype, *like: torch.Tensor) -> torch.Tensor:
+    """A caller's output tensor, checked before any launch: the kernels
+    write all of ``shape`` in ``dtype`` through its pointer."""
+    if tuple(out.shape) != tuple(shape) or out.dtype != dtype:
+        raise ValueError(f"out must be a {dtype} tensor of shape {tuple(shape)}, "
+                         f"not {out.dtype} {tuple(out.shape)}")
+    _require_cuda(out, *like)
+    return out
+
+
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
 
 
 def _stream() -> ctypes.c_void_p:
@@ -55,6 +82,16 @@ def _ptr(t: "torch.Tensor | None") -> ctypes.c_void_p:
 def _workspace(nbytes: int, device) -> torch.Tensor:
     # 256-byte aligned: the caching allocator hands out 512-byte aligned blocks
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _use_workspace(workspace: "torch.Tensor | None", need: int, like: torch.Tensor) -> torch.Tensor:
+    """The caller's workspace (any dtype, counted in bytes) when it holds
+    ``need`` bytes, else a fresh one on ``like``'s device."""
+    if workspace is not None:
+        _require_cuda(workspace, like)
+        if _nbytes(workspace) >= need:
+            return workspace
+    return _workspace(need, like.device)
 
 
 def stream_words(L: int, seq_len: int, layout: int) -> int:
@@ -73,7 +110,7 @@ def bcjr_workspace_size(L: int, seq_len: int, n_seq: int, with_grad: bool = Fals
 def _weights(D: torch.Tensor | None, s: torch.Tensor) -> torch.Tensor | None:
     if D is None:
         return None
-    _require_cuda(D)
+    _require_cuda(D, s)
     if D.shape != s.shape or D.dtype != torch.float32:
         raise ValueError("D must be a float32 tensor shaped like s")
     return D
@@ -96,9 +133,9 @@ def viterbi_encode(s: torch.Tensor, L: int, workspace: torch.Tensor | None = Non
     mse = torch.empty((n,), dtype=torch.float32, device=s.device)
     mrg = torch.empty((n,), dtype=torch.float32, device=s.device) if margin else None
     need = int(lib().tcq_viterbi_workspace_size(ctypes.byref(tr), n))
-    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    ws = _use_workspace(workspace, need, s)
     check(lib().tcq_viterbi_encode(ctypes.byref(tr), _ptr(s), _ptr(D), n, _ptr(states), _ptr(mse),
-                                   _ptr(mrg), _ptr(ws), ws.numel(), _stream()), "tcq_viterbi_encode")
+                                   _ptr(mrg), _ptr(ws), _nbytes(ws), _stream()), "tcq_viterbi_encode")
     return (states, mse, mrg) if margin else (states, mse)
 
 
@@ -116,9 +153,9 @@ def viterbi_encode_tailbiting(s: torch.Tensor, L: int, workspace: torch.Tensor |
     states = torch.empty((n, T), dtype=torch.uint16, device=s.device)
     mse = torch.empty((n,), dtype=torch.float32, device=s.device)
     need = int(lib().tcq_viterbi_workspace_size(ctypes.byref(tr), n))
-    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    ws = _use_workspace(workspace, need, s)
     check(lib().tcq_viterbi_encode_tailbiting(ctypes.byref(tr), _ptr(s), _ptr(D), n, _ptr(states),
-                                              _ptr(mse), _ptr(ws), ws.numel(), _stream()),
+                                              _ptr(mse), _ptr(ws), _nbytes(ws), _stream()),
           "tcq_viterbi_encode_tailbiting")
     return states, mse
 
@@ -136,9 +173,9 @@ def bcjr_soft(s: torch.Tensor, L: int, temp: float, workspace: torch.Tensor | No
     soft = torch.empty_like(s)
     logz = torch.empty((n,), dtype=torch.float32, device=s.device)
     need = int(lib().tcq_bcjr_workspace_size(ctypes.byref(tr), n, 0))
-    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    ws = _use_workspace(workspace, need, s)
     check(lib().tcq_bcjr_soft(ctypes.byref(tr), _ptr(s), _ptr(D), n, float(temp), _ptr(soft),
-                              _ptr(logz), _ptr(ws), ws.numel(), _stream()), "tcq_bcjr_soft")
+                              _ptr(logz), _ptr(ws), _nbytes(ws), _stream()), "tcq_bcjr_soft")
     return soft, logz
 
 
@@ -148,16 +185,17 @@ def bcjr_soft_backward(s: torch.Tensor, L: int, temp: float, soft: torch.Tensor,
     """Vector-Jacobian product: grad_s[u] = sum_t grad_soft[t] d soft[t] / d s[u]."""
     _require_cuda(s, soft, grad_soft)
     D = _weights(D, s)
-    if s.shape != soft.shape or s.shape != grad_soft.shape:
-        raise ValueError("s, soft and grad_soft must have the same shape")
+    if (s.dim() != 2 or s.shape != soft.shape or s.shape != grad_soft.shape
+            or any(t.dtype != torch.float32 for t in (s, soft, grad_soft))):
+        raise ValueError("s, soft and grad_soft must be float32 tensors of one shape [n_seq, seq_len]")
     n, T = s.shape
     tr = trellis(L, T)
     grad = torch.empty_like(s)
     need = int(lib().tcq_bcjr_workspace_size(ctypes.byref(tr), n, 1))
-    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    ws = _use_workspace(workspace, need, s)
     check(lib().tcq_bcjr_soft_backward(ctypes.byref(tr), _ptr(s), _ptr(D), n, float(temp),
                                        _ptr(soft), _ptr(grad_soft), _ptr(grad), _ptr(ws),
-                                       ws.numel(), _stream()), "tcq_bcjr_soft_backward")
+                                       _nbytes(ws), _stream()), "tcq_bcjr_soft_backward")
     return grad
 
 
@@ -168,18 +206,19 @@ def bcjr_soft_and_grad(s: torch.Tensor, L: int, temp: float, grad_soft: torch.Te
     (soft, log_z, grad_s)."""
     _require_cuda(s, grad_soft)
     D = _weights(D, s)
-    if s.shape != grad_soft.shape or s.dtype != torch.float32:
-        raise ValueError("s and grad_soft must be float32 tensors of the same shape")
+    if (s.dim() != 2 or s.shape != grad_soft.shape or s.dtype != torch.float32
+            or grad_soft.dtype != torch.float32):
+        raise ValueError("s and grad_soft must be float32 tensors of one shape [n_seq, seq_len]")
     n, T = s.shape
     tr = trellis(L, T)
     soft = torch.empty_like(s)
     logz = torch.empty((n,), dtype=torch.float32, device=s.device)
     grad = torch.empty_like(s)
     need = int(lib().tcq_bcjr_workspace_size(ctypes.byref(tr), n, 1))
-    ws = workspace if workspace is not None and workspace.numel() >= need else _workspace(need, s.device)
+    ws = _use_workspace(workspace, need, s)
     check(lib().tcq_bcjr_soft_and_grad(ctypes.byref(tr), _ptr(s), _ptr(D), n, float(temp),
                                        _ptr(grad_soft), _ptr(soft), _ptr(logz), _ptr(grad),
-                                       _ptr(ws), ws.numel(), _stream()), "tcq_bcjr_soft_and_grad")
+                                       _ptr(ws), _nbytes(ws), _stream()), "tcq_bcjr_soft_and_grad")
     return soft, logz, grad
 
 
@@ -230,10 +269,11 @@ def decode(bits: torch.Tensor, L: int, seq_len: int = 256, layout: int = TAILBIT
         raise TcqError(_abi.TCQ_ERR_UNSUPPORTED, "tcq_stream_words")
     if bits.shape[1] != words:
         raise ValueError(f"bits must have {words} words per sequence for this trellis and layout")
+    shape = (rows, cols) if out_layout == OUT_TILE16 else (n, seq_len)
     if out is None:
-        shape = (rows, cols) if out_layout == OUT_TILE16 else (n, seq_len)
         out = torch.empty(shape, dtype=torch.float16, device=bits.device)
-    _require_cuda(out)
+    else:
+        _out(out, shape, torch.float16, bits)
     check(lib().tcq_decode(ctypes.byref(tr), _ptr(bits), n, int(layout), int(out_layout), int(rows),
                            int(cols), _ptr(out), _stream()), "tcq_decode")
     return out
@@ -249,8 +289,7 @@ def rht(W: torch.Tensor, sign_rows: torch.Tensor, sign_cols: torch.Tensor,
     R, C = W.shape
     if sign_rows.shape != (R,) or sign_cols.shape != (C,):
         raise ValueError("sign vectors must match W's rows and columns")
-    out = torch.empty_like(W) if out is None else out
-    _require_cuda(out)
+    out = torch.empty_like(W) if out is None else _out(out, (R, C), torch.float32, W)
     check(lib().tcq_rht(_ptr(W), R, C, _ptr(sign_rows.float().contiguous()),
                         _ptr(sign_cols.float().contiguous()), _ptr(out), _stream()), "tcq_rht")
     return out
@@ -267,7 +306,8 @@ def decode_gemv(bits: torch.Tensor, x: torch.Tensor, rows: int, cols: int, L: in
     words = int(lib().tcq_stream_words(ctypes.byref(tr), int(layout)))
     if bits.shape != ((rows // 16) * (cols // 16), words):
         raise ValueError("bits must hold one stream per 16x16 tile")
-    y = torch.empty((rows,), dtype=torch.float32, device=x.device) if out is None else out
+    y = (torch.empty((rows,), dtype=torch.float32, device=x.device) if out is None
+         else _out(out, (rows,), torch.float32, x))
     check(lib().tcq_decode_gemv(ctypes.byref(tr), _ptr(bits), int(layout), int(rows), int(cols),
                                 _ptr(x), _ptr(y), _stream()), "tcq_decode_gemv")
     return y
