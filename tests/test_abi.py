@@ -118,3 +118,21 @@ def test_empty_and_negative_batches_on_every_entry_point(L):
     assert L.tcq_decode_gemv(tr16, None, _abi.TAILBITING, 0, 16, None, None, None) == _abi.TCQ_ERR_INVALID_ARG
     assert L.tcq_decode_gemv(tr16, None, _abi.TAILBITING, 16, 0, None, None, None) == _abi.TCQ_ERR_INVALID_ARG
     assert L.tcq_rht(None, 0, 64, None, None, None, None) == _abi.TCQ_ERR_INVALID_ARG
+
+
+def test_rht_arguments(L):
+    # sizes: powers of two (else an invalid argument), 32 <= cols <= 8192 and
+    # 32 <= rows <= 2^20 (else unsupported); every pointer non-null and
+    # 16-byte aligned.  None of these calls reaches a launch.
+    from trellis_coded_weight_bitshift_b200 import _abi
+    p = ctypes.c_void_p(256)
+    for rows, cols, want in ((48, 64, _abi.TCQ_ERR_INVALID_ARG), (64, 96, _abi.TCQ_ERR_INVALID_ARG),
+                             (0, 64, _abi.TCQ_ERR_INVALID_ARG), (64, -64, _abi.TCQ_ERR_INVALID_ARG),
+                             (16, 64, _abi.TCQ_ERR_UNSUPPORTED), (64, 16, _abi.TCQ_ERR_UNSUPPORTED),
+                             (64, 16384, _abi.TCQ_ERR_UNSUPPORTED), (1 << 21, 64, _abi.TCQ_ERR_UNSUPPORTED)):
+        assert L.tcq_rht(p, rows, cols, p, p, p, None) == want, (rows, cols)
+    for i in range(4):                              # W, sign_rows, sign_cols, out
+        for bad in (None, ctypes.c_void_p(256 + 4)):
+            args = [p, p, p, p]
+            args[i] = bad
+            assert L.tcq_rht(args[0], 64, 64, args[1], args[2], args[3], None) == _abi.TCQ_ERR_INVALID_ARG, (i, bad)

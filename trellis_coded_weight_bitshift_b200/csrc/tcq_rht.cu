@@ -314,7 +314,7 @@ extern "C" tcq_status_t tcq_rht(const float *W, int64_t rows, int64_t cols, cons
   if (!pow2(rows) || !pow2(cols)) return TCQ_ERR_INVALID_ARG;
   if (rows < 32 || cols < 32 || cols > 8192 || rows > (1 << 20)) return TCQ_ERR_UNSUPPORTED;
   if (!W || !out || !sign_rows || !sign_cols || !aligned16(W) || !aligned16(out) ||
-      !aligned16(sign_cols))
+      !aligned16(sign_rows) || !aligned16(sign_cols))
     return TCQ_ERR_INVALID_ARG;
   cudaStream_t strm = (cudaStream_t)stream;
   const int R = (int)rows, C = (int)cols;
